@@ -1,0 +1,91 @@
+"""Plant plausible mistakes in the oracle (on the CPU, via monkeypatch) and
+check that the pins in test_oracle_pins.py catch each one."""
+import numpy as np
+import pytest
+
+import oracle
+from oracle import markov as om
+from oracle import rounding as orr
+
+import test_oracle_pins as pins
+
+
+def _fails(fn, *a, **kw):
+    with pytest.raises(AssertionError):
+        fn(*a, **kw)
+
+
+def test_transposed_w2_is_caught(monkeypatch):
+    monkeypatch.setattr(om, "project_bias", lambda latent, w2: np.asarray(latent, float) @ np.asarray(w2, float))
+    _fails(pins.test_bigram_special_case_is_a_table_lookup)
+
+
+def test_dropped_bias_is_caught(monkeypatch):
+    monkeypatch.setattr(om, "compute_step_bias",
+                        lambda w1, w2, ids, hidden_states=None: np.zeros((np.size(ids), np.shape(w2)[0])))
+    _fails(pins.test_worked_example_apply, "bf16")
+
+
+def test_double_rounding_is_caught(monkeypatch):
+    real = orr.round_to_bfloat16
+    monkeypatch.setattr(orr, "round_to_bfloat16", lambda x: real(np.asarray(x, float).astype(np.float32)))
+    monkeypatch.setattr(oracle, "round_to_bfloat16", orr.round_to_bfloat16)
+    _fails(pins.test_bf16_hand_cases)
+
+
+def test_truncating_rounding_is_caught(monkeypatch):
+    def trunc(x):
+        x = np.asarray(x, np.float32)
+        return (x.view(np.uint32) & np.uint32(0xFFFF0000)).view(np.float32).astype(np.float64)
+    monkeypatch.setattr(oracle, "round_to_bfloat16", trunc)
+    _fails(pins.test_bf16_matches_torch_on_binary32_inputs)
+
+
+def test_unbiased_chain_feedback_is_caught(monkeypatch):
+    """Feeding the argmax of the base logits (not of the corrected logits)
+    to the next step."""
+    def unbiased_choice(base_logits, w1, w2, first_prev, out_dtype, temperature=0.0, seed=0, hidden_states=None):
+        base = np.asarray(base_logits, float)
+        prev = np.asarray(first_prev)
+        toks, corr = [], []
+        for k in range(base.shape[1]):
+            corr.append(om.apply_step_logits(base[:, k], w1, w2, prev, out_dtype))
+            prev = np.argmax(base[:, k], axis=-1)
+            toks.append(prev)
+        return np.stack(toks, 1), np.stack(corr, 1)
+    monkeypatch.setattr(oracle, "sample_block_tokens", unbiased_choice)
+    _fails(pins.test_worked_example_greedy_chain)
+
+
+def test_off_by_one_prev_is_caught(monkeypatch):
+    """Using the first previous token for every step (no feedback)."""
+    def no_feedback(base_logits, w1, w2, first_prev, out_dtype, temperature=0.0, seed=0, hidden_states=None):
+        base = np.asarray(base_logits, float)
+        b, m, _ = base.shape
+        prev = np.asarray(first_prev)
+        corr = np.stack([om.apply_step_logits(base[:, k], w1, w2, prev, out_dtype) for k in range(m)], 1)
+        toks = np.stack([om.sample_tokens(corr[:, k], temperature, seed, k) for k in range(m)], 1)
+        return toks, corr
+    monkeypatch.setattr(oracle, "sample_block_tokens", no_feedback)
+    _fails(pins.test_greedy_chain_brute_force_bigram)
+
+
+def test_missing_temperature_is_caught(monkeypatch):
+    real = om.gumbel_noise
+    monkeypatch.setattr(om, "temperature_scores",
+                        lambda row, t, seed, b, k: np.asarray(row, float) + real(seed, b, k, np.shape(row)[-1]))
+    _fails(pins.test_temperature_sampling_follows_softmax, 0.5)
+
+
+def test_shared_noise_across_rows_is_caught(monkeypatch):
+    """Dropping the row index b from the Philox counter makes every row draw
+    the same token."""
+    real = om.gumbel_noise
+    monkeypatch.setattr(om, "gumbel_noise", lambda seed, b, k, v: real(seed, 0, k, v))
+    _fails(pins.test_temperature_sampling_follows_softmax, 1.0)
+
+
+def test_highest_index_tie_break_is_caught(monkeypatch):
+    monkeypatch.setattr(om, "select_greedy",
+                        lambda x: (np.shape(x)[-1] - 1 - np.argmax(np.asarray(x)[..., ::-1], axis=-1)))
+    _fails(pins.test_worked_example_greedy_chain)

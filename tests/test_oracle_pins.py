@@ -1,0 +1,346 @@
+"""Pins of the CPU oracle to facts outside itself (no GPU).
+
+Each test ties one part of the oracle to something it does not compute
+itself: hand-worked values (tests/golden), a library routine that covers a
+special case, a closed form, or a distributional law checked by chi-square.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+from scipy import stats
+from scipy.special import softmax
+
+import oracle
+from oracle import markov as om
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _f(s):
+    return float(s) if s in ("inf", "-inf", "nan") else float.fromhex(s)
+
+
+# --------------------------------------------------------------------------
+# bfloat16 rounding
+# --------------------------------------------------------------------------
+
+def test_bf16_hand_cases():
+    cases = json.load(open(os.path.join(GOLDEN, "bf16_rounding.json")))["cases"]
+    x = np.array([_f(c["x"]) for c in cases])
+    want = np.array([_f(c["want"]) for c in cases])
+    got = oracle.round_to_bfloat16(x)
+    for xi, gi, wi, c in zip(x, got, want, cases):
+        if np.isnan(wi):
+            assert np.isnan(gi), c["why"]
+        else:
+            assert gi == wi and np.signbit(gi) == np.signbit(wi), (c["x"], gi.hex(), c["why"])
+
+
+def test_bf16_matches_torch_on_binary32_inputs():
+    """For inputs that are binary32 values there is one rounding either way,
+    so the oracle must agree with torch's float32 -> bfloat16 conversion
+    (round to nearest even) bit for bit."""
+    rng = np.random.default_rng(0)
+    bits = rng.integers(0, 2 ** 32, size=400_000, dtype=np.uint64).astype(np.uint32)
+    x32 = bits.view(np.float32)
+    x32 = x32[np.isfinite(x32)]
+    extra = np.array([1.0, 1.00390625, 1.01171875, 3.3895314e38, -3.3895314e38, 1e-40, -1e-41, 0.0],
+                     dtype=np.float32)
+    x32 = np.concatenate([x32, extra, (rng.standard_normal(100_000) * 4).astype(np.float32)])
+    want = torch.from_numpy(x32.copy()).to(torch.bfloat16).to(torch.float64).numpy()
+    got = oracle.round_to_bfloat16(x32.astype(np.float64))
+    same = (got == want) | (np.isnan(got) & np.isnan(want))
+    assert same.all(), (x32[~same][:5], got[~same][:5], want[~same][:5])
+
+
+def test_bf16_ulp():
+    assert oracle.ulp_bfloat16(np.array([1.0]))[0] == 2 ** -7
+    assert oracle.ulp_bfloat16(np.array([9.5]))[0] == 2 ** -4
+    assert oracle.ulp_bfloat16(np.array([0.0]))[0] == 2 ** -7  # defined at 1 for zero
+    assert oracle.ulp_bfloat16(np.array([1e-40]))[0] == 2 ** -133
+
+
+# --------------------------------------------------------------------------
+# The bias and the add
+# --------------------------------------------------------------------------
+
+def _worked():
+    return json.load(open(os.path.join(GOLDEN, "worked_example.json")))
+
+
+def test_worked_example_bias_table():
+    d = _worked()
+    w1, w2 = np.array(d["w1"], float), np.array(d["w2"], float)
+    got = oracle.compute_step_bias(w1, w2, np.arange(3))
+    np.testing.assert_array_equal(got, np.array(d["bias_table"]["rows"], float))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_worked_example_apply(dtype):
+    d = _worked()
+    w1, w2 = np.array(d["w1"], float), np.array(d["w2"], float)
+    a = d["apply"]
+    got = oracle.apply_block_logits(np.array(a["base"], float), w1, w2, np.array(a["prev_ids"]), dtype)
+    np.testing.assert_array_equal(got, np.array(a["want"], float))
+
+
+def test_worked_example_greedy_chain():
+    d = _worked()
+    w1, w2 = np.array(d["w1"], float), np.array(d["w2"], float)
+    s = d["sample_greedy"]
+    toks, corr = oracle.sample_block_tokens(np.array(s["base"], float), w1, w2, np.array(s["first_prev"]),
+                                            "bf16", temperature=0.0)
+    np.testing.assert_array_equal(toks, np.array(s["want_tokens"]))
+    np.testing.assert_array_equal(corr, np.array(s["want_corrected"], float))
+    # temperature None and below the 1e-5 threshold are greedy too
+    for t in (None, 0.0, 9.9e-6, -1.0):
+        t2, _ = oracle.sample_block_tokens(np.array(s["base"], float), w1, w2, np.array(s["first_prev"]),
+                                           "bf16", temperature=t)
+        np.testing.assert_array_equal(t2, np.array(s["want_tokens"]))
+
+
+def _bigram_case(v=16, seed=0):
+    """W1 = identity (r = V): B(x, v) = W2[v, x], a plain bigram table.
+    Integer weights keep every sum exact."""
+    rng = np.random.default_rng(seed)
+    w1 = np.eye(v)
+    w2 = rng.integers(-8, 9, size=(v, v)).astype(float)  # not symmetric
+    table = w2.T.copy()  # table[x, v] = logit bias of token v after token x
+    return w1, w2, table
+
+
+def test_bigram_special_case_is_a_table_lookup():
+    w1, w2, table = _bigram_case()
+    assert not np.array_equal(w2, w2.T)
+    ids = np.array([3, 0, 15, 3, 7])
+    got = oracle.compute_step_bias(w1, w2, ids)
+    for i, x in enumerate(ids):
+        np.testing.assert_array_equal(got[i], table[x])
+
+
+def test_zero_w2_passes_logits_through_bit_for_bit():
+    rng = np.random.default_rng(1)
+    base = oracle.round_to_bfloat16(rng.standard_normal((3, 4, 5, 64)) * 3)
+    w1 = rng.standard_normal((64, 16))
+    got = oracle.apply_block_logits(base, w1, np.zeros((64, 16)), rng.integers(0, 64, (3, 4, 5)), "bf16")
+    np.testing.assert_array_equal(got, base)
+    toks, corr = oracle.sample_block_tokens(base[:, 0], w1, np.zeros((64, 16)), rng.integers(0, 64, 3), "bf16")
+    np.testing.assert_array_equal(corr, base[:, 0])
+    np.testing.assert_array_equal(toks, np.argmax(base[:, 0], axis=-1))
+
+
+def test_bias_row_by_row_against_explicit_sums():
+    """B(x, v) = sum_j W1[x, j] W2[v, j], summed in exact rational arithmetic
+    on small dyadic values (so any fp64 sum is exact)."""
+    from fractions import Fraction
+    rng = np.random.default_rng(2)
+    w1 = rng.integers(-64, 65, size=(12, 5)) / 32.0
+    w2 = rng.integers(-64, 65, size=(12, 5)) / 16.0
+    ids = rng.integers(0, 12, size=7)
+    got = oracle.compute_step_bias(w1, w2, ids)
+    for i, x in enumerate(ids):
+        for v in range(12):
+            s = sum(Fraction(w1[x, j]) * Fraction(w2[v, j]) for j in range(5))
+            assert Fraction(got[i, v]) == s
+
+
+def test_hidden_states_are_ignored():
+    rng = np.random.default_rng(3)
+    base = rng.standard_normal((2, 3, 4, 32))
+    w1, w2 = rng.standard_normal((32, 8)), rng.standard_normal((32, 8))
+    ids = rng.integers(0, 32, (2, 3, 4))
+    a = oracle.apply_block_logits(base, w1, w2, ids, "bf16")
+    b = oracle.apply_block_logits(base, w1, w2, ids, "bf16", hidden_states=rng.standard_normal((2, 3, 4, 7)))
+    np.testing.assert_array_equal(a, b)
+    t1, c1 = oracle.sample_block_tokens(base[:, 0], w1, w2, ids[:, 0, 0], "bf16", 0.7, seed=5)
+    t2, c2 = oracle.sample_block_tokens(base[:, 0], w1, w2, ids[:, 0, 0], "bf16", 0.7, seed=5,
+                                        hidden_states=rng.standard_normal((2, 4, 9)))
+    np.testing.assert_array_equal(t1, t2)
+    np.testing.assert_array_equal(c1, c2)
+
+
+def test_empty_inputs_return_the_input_object():
+    w1 = np.ones((8, 2))
+    w2 = np.ones((8, 2))
+    e1 = np.zeros((2, 0, 8))
+    assert oracle.apply_block_logits(e1, w1, w2, np.zeros((2, 0), int), "bf16") is e1
+    e2 = np.zeros((0, 3, 8))
+    assert oracle.apply_block_logits(e2, w1, w2, np.zeros((0, 3), int), "bf16") is e2
+    toks, corr = oracle.sample_block_tokens(e1, w1, w2, np.array([1, 2]), "bf16")
+    assert corr is e1 and toks.shape == (2, 0) and toks.dtype == np.int64
+
+
+def test_out_of_range_ids_are_rejected():
+    with pytest.raises(IndexError):
+        oracle.compute_step_bias(np.ones((4, 2)), np.ones((4, 2)), np.array([4]))
+    with pytest.raises(IndexError):
+        oracle.compute_step_bias(np.ones((4, 2)), np.ones((4, 2)), np.array([-1]))
+
+
+def test_greedy_ties_take_the_lowest_index_and_nan_wins():
+    assert oracle.select_greedy(np.array([[1.0, 3.0, 3.0, 2.0]]))[0] == 1
+    assert oracle.select_greedy(np.array([[1.0, np.nan, 3.0, np.nan]]))[0] == 1
+    assert oracle.select_greedy(np.array([[-np.inf, -np.inf]]))[0] == 0
+
+
+# --------------------------------------------------------------------------
+# The greedy chain
+# --------------------------------------------------------------------------
+
+def test_greedy_chain_brute_force_bigram():
+    """V = 16, M = 4, every first token: walk the bigram chain by hand
+    (explicit loops over the table, no matrix product) and compare."""
+    v, m = 16, 4
+    w1, w2, table = _bigram_case(v, seed=4)
+    rng = np.random.default_rng(5)
+    base = rng.integers(-16, 17, size=(v, m, v)).astype(float) / 4  # one block per first token
+    toks, corr = oracle.sample_block_tokens(base, w1, w2, np.arange(v), "bf16", temperature=0.0)
+    for x0 in range(v):
+        prev = x0
+        for k in range(m):
+            row = [base[x0, k, j] + table[prev][j] for j in range(v)]
+            best = max(range(v), key=lambda j: (row[j], -j))
+            assert toks[x0, k] == best
+            assert list(corr[x0, k]) == row
+            prev = best
+
+
+def test_tokens_are_argmax_of_returned_logits():
+    rng = np.random.default_rng(6)
+    base = oracle.round_to_bfloat16(rng.standard_normal((4, 5, 300)) * 2)
+    w1, w2 = rng.standard_normal((300, 16)) * 0.3, rng.standard_normal((300, 16)) * 0.3
+    toks, corr = oracle.sample_block_tokens(base, w1, w2, rng.integers(0, 300, 4), "bf16")
+    np.testing.assert_array_equal(toks, np.argmax(corr, axis=-1))
+
+
+def test_sample_equals_apply_on_its_own_tokens():
+    """The two modes differ only in where x_{k-1} comes from: the corrected
+    logits of a sampled block equal the teacher-forced ones computed with
+    prev = [first_prev, tok_0, ..., tok_{M-2}]."""
+    rng = np.random.default_rng(7)
+    base = oracle.round_to_bfloat16(rng.standard_normal((6, 5, 200)) * 2)
+    w1, w2 = rng.standard_normal((200, 32)) * 0.3, rng.standard_normal((200, 32)) * 0.3
+    first = rng.integers(0, 200, 6)
+    for temp in (0.0, 0.8):
+        toks, corr = oracle.sample_block_tokens(base, w1, w2, first, "bf16", temp, seed=9)
+        prev = np.concatenate([first[:, None], toks[:, :-1]], axis=1)
+        np.testing.assert_array_equal(oracle.apply_block_logits(base, w1, w2, prev, "bf16"), corr)
+
+
+# --------------------------------------------------------------------------
+# Philox4x32-10 and the temperature sampler
+# --------------------------------------------------------------------------
+
+_TRITON_PHILOX = r"""
+import os, sys, json
+os.environ["TRITON_INTERPRET"] = "1"
+import torch, triton, triton.language as tl
+@triton.jit
+def k(out, c0p, c1p, c2p, c3p, k0p, k1p, N: tl.constexpr):
+    i = tl.arange(0, N)
+    a, b, c, d = tl.philox_impl(tl.load(c0p + i), tl.load(c1p + i), tl.load(c2p + i), tl.load(c3p + i),
+                                tl.load(k0p + i), tl.load(k1p + i), 10)
+    tl.store(out + i, a); tl.store(out + N + i, b); tl.store(out + 2 * N + i, c); tl.store(out + 3 * N + i, d)
+cols = json.loads(sys.stdin.read())
+n = len(cols[0])
+t = [torch.tensor(c, dtype=torch.int64).to(torch.uint32) for c in cols]
+out = torch.zeros(4 * n, dtype=torch.uint32)
+k[(1,)](out, *t, n)
+print(json.dumps(out.to(torch.int64).view(4, n).tolist()))
+"""
+
+
+def test_philox_matches_an_independent_library_implementation():
+    """Triton's own Philox4x32 (its CPU interpreter, a library routine the
+    oracle does not share) must give the same words for the same counters and
+    keys, including all-zero and all-ones corners."""
+    import subprocess
+    import sys
+    rng = np.random.default_rng(8)
+    n = 64
+    cols = [rng.integers(0, 2 ** 32, n, dtype=np.uint64) for _ in range(6)]
+    for c in cols:
+        c[0], c[1] = 0, 2 ** 32 - 1
+    cols = [c.astype(np.int64).tolist() for c in cols]
+    env = dict(os.environ, TRITON_INTERPRET="1")
+    res = subprocess.run([sys.executable, "-c", _TRITON_PHILOX], input=json.dumps(cols), capture_output=True,
+                         text=True, env=env, timeout=600)
+    if res.returncode != 0:
+        pytest.skip("triton interpreter unavailable: " + res.stderr[-300:])
+    want = np.array(json.loads(res.stdout.strip().splitlines()[-1]), dtype=np.uint64)
+    c = [np.array(x, dtype=np.uint64).astype(np.uint32) for x in cols]
+    for i in range(n):
+        got = oracle.philox4x32((c[0][i], c[1][i], c[2][i], c[3][i]), (int(c[4][i]), int(c[5][i])))
+        assert [int(w) for w in got] == [int(w) for w in want[:, i]], i
+
+
+def test_philox_words_look_uniform():
+    w = np.concatenate([oracle.noise_words(1234, b, k, 4096) for b in range(4) for k in range(4)])
+    counts = np.bincount((w >> np.uint32(24)).astype(np.int64), minlength=256)
+    assert stats.chisquare(counts).pvalue > 1e-3
+    u = oracle.uniform_from_word(w)
+    assert u.min() > 0 and u.max() < 1
+    # neighbouring ids (same Philox call and across calls) are uncorrelated
+    assert abs(np.corrcoef(u[:-1], u[1:])[0, 1]) < 0.02
+
+
+def test_uniform_mapping_endpoints():
+    u = oracle.uniform_from_word(np.array([0, 0xFFFFFFFF, 0x1FF, 0x200], dtype=np.uint32))
+    assert u[0] == 2.0 ** -24 and u[1] == 1 - 2.0 ** -24
+    assert u[2] == 2.0 ** -24 and u[3] == 3 * 2.0 ** -24
+
+
+def test_noise_layout_four_ids_per_call():
+    seed = (7 << 32) | 99
+    w = oracle.noise_words(seed, b=5, k=3, vocab=10)
+    for v in range(10):
+        words = oracle.philox4x32((np.uint32(v >> 2), np.uint32(3), np.uint32(5), np.uint32(0)), (99, 7))
+        assert int(w[v]) == int(words[v & 3])
+
+
+@pytest.mark.parametrize("temp", [0.5, 0.7, 1.0, 2.0])
+def test_temperature_sampling_follows_softmax(temp):
+    """V = 8, M = 1: many rows of the same logits, each with its own noise
+    (row index b is part of the Philox counter). Counts must fit
+    softmax(c / T) (scipy) by chi-square."""
+    v, rows = 8, 1 << 14
+    rng = np.random.default_rng(10)
+    logits = oracle.round_to_bfloat16(rng.standard_normal(v) * 1.5)
+    w1, w2 = np.zeros((v, 2)), np.zeros((v, 2))
+    base = np.broadcast_to(logits, (rows, 1, v))
+    toks, _ = oracle.sample_block_tokens(base, w1, w2, np.zeros(rows, int), "bf16", temp, seed=1234)
+    counts = np.bincount(toks[:, 0], minlength=v)
+    p = softmax(logits / temp)
+    assert stats.chisquare(counts, p * rows).pvalue > 1e-3
+
+
+def test_chain_joint_distribution_bigram():
+    """V = 4, M = 3, bigram table (W1 = I): the frequencies of all 64 sampled
+    sequences must fit the product of the per-step conditionals
+    softmax((U_k + T[x_{k-1}]) / T), written out with scipy's softmax."""
+    v, m, rows, temp = 4, 3, 1 << 14, 0.9
+    w1 = np.eye(v)
+    w2 = np.array([[1.0, -1, 0, 0.5], [0, 2, -1, 0], [-1, 0, 1.5, -0.5], [0.5, 0, -1, 1]])
+    table = w2.T
+    u = np.array([[0.2, 0.0, -0.3, 0.1], [0.0, 0.5, 0.0, -0.5], [-0.2, 0.1, 0.3, 0.0]])
+    base = np.broadcast_to(u, (rows, m, v))
+    x0 = 2
+    toks, _ = oracle.sample_block_tokens(base, w1, w2, np.full(rows, x0), "fp32", temp, seed=77)
+    idx = toks[:, 0] * 16 + toks[:, 1] * 4 + toks[:, 2]
+    counts = np.bincount(idx, minlength=64)
+    p = np.zeros(64)
+    for a in range(v):
+        for b in range(v):
+            for c in range(v):
+                pa = softmax((u[0] + table[x0]) / temp)[a]
+                pb = softmax((u[1] + table[a]) / temp)[b]
+                pc = softmax((u[2] + table[b]) / temp)[c]
+                p[a * 16 + b * 4 + c] = pa * pb * pc
+    assert abs(p.sum() - 1) < 1e-12
+    keep = p * rows >= 5  # chi-square needs expected counts >= 5
+    obs = np.append(counts[keep], counts[~keep].sum())
+    exp = np.append(p[keep] * rows, p[~keep].sum() * rows)
+    assert stats.chisquare(obs, exp).pvalue > 1e-3
