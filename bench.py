@@ -1,0 +1,464 @@
+#!/usr/bin/env python
+"""Benchmark of the VanillaMarkov head's hot path on B200.
+
+One step = one pass over the whole path on its seeded synthetic workloads:
+  * teacher-forced apply_block_logits, 320 rows (B=4, 16 blocks of 5),
+    V=129280, rank 128, bf16 (the workload the metric is quoted on);
+  * greedy sample_block_tokens, B=32 blocks of M=5, V=129280, rank 128;
+  * temperature sample_block_tokens, B=32, M=8, V=151936, rank 64, T=0.7.
+The metric is corrected-logit rows per second over the step (apply rows plus
+sampled positions), with per-part rows/s, blocks/s, GB/s and roofline
+fractions beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torch.distributed.run, one rank per GPU; every rank runs its
+own copy of the workload (weak scaling, no data-path collective) and the
+step time is the max over ranks. ``--impl reference`` times the CPU fp64
+oracle on the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from rank_markov_draft_vanillamarkov_b200 import workloads as W  # noqa: E402
+
+METRIC = "corrected-logit rows/s + achieved HBM GB/s (% roofline); sampled blocks/s at M=5"
+UNIT = "rows/s"
+FALLBACK_HBM_GBS = 6650.0
+PARTS = (("apply", W.APPLY_320), ("greedy", W.greedy(32)), ("temperature", W.TEMPERATURE))
+EXTRA = (("apply_2560", W.APPLY_2560),)
+L2_BYTES = 126 * 1024 * 1024
+
+
+def part_rows(wl: W.Workload) -> int:
+    return wl.rows if wl.mode == "apply" else wl.batch * wl.proposal_len
+
+
+# --------------------------------------------------------------- helpers --
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profile_traffic(kernel_tag: str):
+    """DRAM bytes per launch from the committed ncu summary of this kernel,
+    valid only while the kernel source it was taken from is unchanged."""
+    path = os.path.join(ROOT, "profiles", f"{kernel_tag}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_b = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    m_h = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    m_f = re.search(r"source_file:\s*(\S+)", text)
+    if not (m_b and m_h and m_f):
+        return None
+    src = os.path.join(ROOT, m_f.group(1))
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != m_h.group(1):
+        return None
+    return float(m_b.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples taken while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.6)
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------- our arm ----
+
+class Part:
+    """Device-resident inputs (several rotating sets, together larger than
+    L2) and outputs of one workload of the step."""
+
+    def __init__(self, name, wl, device, seed_offset, min_bytes=3 * L2_BYTES):
+        from rank_markov_draft_vanillamarkov_b200 import VanillaMarkov
+        self.name, self.wl, self.device = name, wl, device
+        per = wl.bytes_moved()
+        self.nsets = max(2, -(-min_bytes // per))
+        self.sets = []
+        for i in range(self.nsets):
+            d = W.make_inputs(wl.with_(data_seed=wl.data_seed + seed_offset + i))
+            dev = {k: v.to(device) for k, v in d.items() if isinstance(v, torch.Tensor)}
+            dev["head"] = VanillaMarkov(dev["w1"], dev["w2"])
+            if wl.mode == "apply":
+                dev["out"] = torch.empty_like(dev["base"])
+            else:
+                dev["tokens"] = torch.empty(wl.batch, wl.proposal_len, dtype=torch.long, device=device)
+                dev["out"] = torch.empty_like(dev["base"])
+            self.sets.append(dev)
+        self.host = W.make_inputs(wl.with_(data_seed=wl.data_seed + seed_offset))
+
+    def run(self, i):
+        s = self.sets[i % self.nsets]
+        if self.wl.mode == "apply":
+            s["head"].apply_block_logits(s["base"], token_ids=s["prev_ids"], out=s["out"])
+        else:
+            s["head"].sample_block_tokens(s["base"], first_prev_token_ids=s["first_prev"],
+                                          temperature=self.wl.temperature, seed=self.wl.philox_seed,
+                                          out_tokens=s["tokens"], out_logits=s["out"])
+
+    @property
+    def rows(self):
+        return part_rows(self.wl)
+
+
+def time_region(parts, steps, warmup, world):
+    """Warm up, then time exactly `steps` steps between a barrier and a device
+    synchronise on both sides. Returns (region seconds max over ranks, per-part
+    mean kernel seconds)."""
+    import torch.distributed as dist
+    for i in range(warmup):
+        for p in parts:
+            p.run(i)
+    torch.cuda.synchronize()
+    ev = {p.name: [] for p in parts}
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(steps):
+        for p in parts:
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            p.run(warmup + i)
+            b.record()
+            ev[p.name].append((a, b))
+    end.record()
+    torch.cuda.synchronize()
+    region = start.elapsed_time(end) / 1e3
+    per = {k: sum(a.elapsed_time(b) for a, b in v) / len(v) / 1e3 for k, v in ev.items()}
+    if world > 1:
+        t = torch.tensor([region], device=parts[0].device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        region = float(t.item())
+        dist.barrier()
+    return region, per
+
+
+def time_e2e(parts, steps, world):
+    """The same step through the public API with host buffers: each step
+    copies its inputs host->device from pinned memory, runs the three calls
+    and copies every output (corrected logits and tokens) back to pinned host
+    memory; all inside the timed region."""
+    import torch.distributed as dist
+    from rank_markov_draft_vanillamarkov_b200 import VanillaMarkov
+    dev = parts[0].device
+    host, devb, h2d, d2h = [], [], 0, 0
+    for p in parts:
+        h = {k: v.pin_memory() for k, v in p.host.items() if isinstance(v, torch.Tensor) and k not in ("w1", "w2")}
+        d = {k: torch.empty_like(v, device=dev) for k, v in h.items()}
+        d["head"] = VanillaMarkov(p.sets[0]["w1"], p.sets[0]["w2"])
+        out_host = torch.empty_like(p.host["base"]).pin_memory()
+        tok_host = torch.empty(p.wl.batch, p.wl.proposal_len, dtype=torch.long).pin_memory() \
+            if p.wl.mode == "sample" else None
+        keys = ["base", "prev_ids"] if p.wl.mode == "apply" else ["base", "first_prev"]
+        h2d += sum(h[k].numel() * h[k].element_size() for k in keys)
+        d2h += out_host.numel() * out_host.element_size() + (tok_host.numel() * 8 if tok_host is not None else 0)
+        host.append((p, h, keys, out_host, tok_host))
+        devb.append(d)
+
+    def one():
+        for (p, h, keys, out_host, tok_host), d in zip(host, devb):
+            for k in keys:
+                d[k].copy_(h[k], non_blocking=True)
+            if p.wl.mode == "apply":
+                out = d["head"].apply_block_logits(d["base"], token_ids=d["prev_ids"])
+                out_host.copy_(out, non_blocking=True)
+            else:
+                t, c = d["head"].sample_block_tokens(d["base"], first_prev_token_ids=d["first_prev"],
+                                                     temperature=p.wl.temperature, seed=p.wl.philox_seed)
+                out_host.copy_(c, non_blocking=True)
+                tok_host.copy_(t, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    sec = a.elapsed_time(b) / 1e3
+    if world > 1:
+        t = torch.tensor([sec], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        sec = float(t.item())
+    return sec, h2d, d2h
+
+
+# ------------------------------------------------------- oracle (CPU) arm --
+
+def _np(t):
+    return t.to(torch.float64).numpy()
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_full_step(inputs):
+    """The oracle over one whole step (every part at full size)."""
+    import oracle
+    rows = 0
+    for (name, wl), d in zip(PARTS, inputs):
+        if wl.mode == "apply":
+            oracle.apply_block_logits(_np(d["base"]), _np(d["w1"]), _np(d["w2"]), d["prev_ids"].numpy(), "bf16")
+        else:
+            oracle.sample_block_tokens(_np(d["base"]), _np(d["w1"]), _np(d["w2"]), d["first_prev"].numpy(), "bf16",
+                                       wl.temperature, wl.philox_seed)
+        rows += part_rows(wl)
+    return rows
+
+
+class OracleUnits:
+    """The step's work as a sequence of small units in the step's proportions:
+    one apply row, one greedy block or one temperature block per unit."""
+
+    def __init__(self):
+        self.inputs = [W.make_inputs(wl) for _, wl in PARTS]
+        self.np = [{k: (_np(v) if v.is_floating_point() else v.numpy()) for k, v in d.items()} for d in self.inputs]
+        self.units = []
+        for pi, (name, wl) in enumerate(PARTS):
+            n = wl.rows if wl.mode == "apply" else wl.batch
+            self.units += [(pi, j) for j in range(n)]
+
+    def run(self, i):
+        import oracle
+        pi, j = self.units[i % len(self.units)]
+        wl = PARTS[pi][1]
+        d = self.np[pi]
+        if wl.mode == "apply":
+            base = d["base"].reshape(-1, wl.vocab)[j:j + 1]
+            ids = d["prev_ids"].reshape(-1)[j:j + 1]
+            oracle.apply_block_logits(base[None], d["w1"], d["w2"], ids[None], "bf16")
+            return 1
+        oracle.sample_block_tokens(d["base"][j:j + 1], d["w1"], d["w2"], d["first_prev"][j:j + 1], "bf16",
+                                   wl.temperature, wl.philox_seed)
+        return wl.proposal_len
+
+
+def reference_arm(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    units = OracleUnits()
+    for i in range(args.warmup):
+        units.run(i)
+    rows = 0
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        rows += units.run(args.warmup + i)
+    sec = time.perf_counter() - t0
+    value = rows / sec
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+                         "sample": "each step is one unit of the step's work in its proportions (one apply row, "
+                                   "one greedy block of 5 or one temperature block of 8), in order"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_block(n_gpus):
+    return {
+        "workload": "apply_r320_v129280_k128 + greedy_b32_m5_v129280_k128 + temp0.7_b32_m8_v151936_k64",
+        "parts": {name: wl.name for name, wl in PARTS},
+        "logits_dtype": "bf16", "weights_dtype": "bf16", "accumulate": "fp32",
+        "l2": "inputs rotate over >= 3 x L2 of distinct buffers per part, so no step finds its data in L2",
+        "parallelism": f"replicas{n_gpus}" if n_gpus > 1 else "single",
+    }
+
+
+# ----------------------------------------------------------------- main ----
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    world, rank, local = dist_env()
+    if args.gpus != world and world > 1:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+
+    from rank_markov_draft_vanillamarkov_b200 import _native as N
+    from rank_markov_draft_vanillamarkov_b200 import launch_count
+    from rank_markov_draft_vanillamarkov_b200.build import build
+    if rank == 0:
+        build()
+    if world > 1:
+        torch.distributed.barrier()
+    N.load()
+
+    parts = [Part(name, wl, device, seed_offset=1000 * rank) for name, wl in PARTS]
+    extra = [Part(name, wl, device, seed_offset=1000 * rank, min_bytes=2 * L2_BYTES) for name, wl in EXTRA]
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    n0 = launch_count()
+    region, per = time_region(parts, args.steps, args.warmup, world)
+    launches = launch_count() - n0
+    clk = clocks.stop()
+    extra_region, extra_per = time_region(extra, max(20, args.steps // 20), 3, world)
+
+    e2e_sec, h2d, d2h = time_e2e(parts, args.e2e_steps, world)
+
+    rows_step = sum(p.rows for p in parts)
+    value = rows_step * world * args.steps / region
+    hbm_peak, peak_kind = measured_peaks()
+    partinfo = {}
+    for p in parts + extra:
+        t = per.get(p.name, extra_per.get(p.name))
+        gbs = p.wl.bytes_moved() / t / 1e9
+        info = {"us": t * 1e6, "rows_per_s": p.rows / t, "gbps": gbs, "frac_hbm": gbs / hbm_peak,
+                "bytes": p.wl.bytes_moved(), "flops": p.wl.flops()}
+        if p.wl.mode == "sample":
+            info["blocks_per_s"] = p.wl.batch / t
+        partinfo[p.name] = info
+    dom = max(parts, key=lambda p: per[p.name])
+    tag = {"apply": "apply_tc_r320_v129280_k128", "greedy": "sample_tc_greedy_b32_m5_v129280_k128",
+           "temperature": "sample_tc_temp_b32_m8_v151936_k64"}[dom.name]
+    achieved = dom.wl.bytes_moved() / per[dom.name] / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": region / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_block(world),
+        "sampled_blocks_per_s_m5": partinfo["greedy"]["blocks_per_s"] * world,
+        "parts": partinfo,
+        "roofline": {"bound": "hbm", "kernel": dom.name, "achieved": achieved, "peak": hbm_peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm_peak,
+                     "traffic": profile_traffic(tag), "algorithmic_bytes": dom.wl.bytes_moved()},
+        "gpu_launches": launches,
+        "clocks": clk,
+        "e2e": {"value": rows_step * world * args.e2e_steps / e2e_sec, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        inputs = [W.make_inputs(wl) for _, wl in PARTS]
+        t0 = time.perf_counter()
+        rows = oracle_full_step(inputs)
+        sec = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": rows / sec, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+                                "sample": "one full step (all three parts at full size) through the fp64 oracle",
+                                "seconds": sec}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,139 @@
+/*
+ * dspark_markov.h -- C ABI of the B200 (sm_100a) VanillaMarkov transition-bias head.
+ *
+ * The head (markov_head.py, the vendored DSpark-style low-rank Markov sequential
+ * head: module docstring "WHAT THIS IS" and class VanillaMarkov) adds a
+ * rank-r bias that depends only on the previous token to a parallel block
+ * drafter's base logits:
+ *
+ *     corrected_k[v] = U_k[v] + B(x_{k-1}, v),   B(x, v) = sum_j W1[x, j] * W2[v, j]
+ *
+ * W1 is an embedding table and W2 the weight of a bias-free Linear(r, V); both
+ * are stored [V, r] row-major, exactly as the two PyTorch modules store them.
+ *
+ * Conventions shared by every entry point:
+ *   - Every buffer is caller-owned DEVICE memory on the current CUDA device,
+ *     contiguous row-major. The library never frees or keeps a caller pointer
+ *     beyond the call.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ *     stream) and the call returns without synchronising. Results are valid
+ *     once the stream has reached that point.
+ *   - The return value is a DSPARK_* code. Argument errors are detected on the
+ *     host before anything is enqueued. Errors found on the device (a token id
+ *     outside [0, V), a bounded wait that ran out) never trap: they are OR-ed
+ *     into a per-device status word read by dspark_markov_get_status().
+ *   - logits_dtype / weight_dtype are DSPARK_DTYPE_* codes. Sums are
+ *     accumulated in fp32 and the corrected logit is rounded once (round to
+ *     nearest even) to the logits dtype.
+ *   - The library keeps a small per-device workspace (status word, reduction
+ *     keys and a barrier counter for the sampler), allocated on first use and
+ *     grown when a larger sampler call needs it. Calls that use it must not
+ *     run concurrently on one device (issue them on one stream).
+ */
+#ifndef DSPARK_MARKOV_H
+#define DSPARK_MARKOV_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+#define DSPARK_OK 0
+#define DSPARK_ERR_INVALID_ARG 1 /* null pointer, non-positive size, rank <= 0, NaN temperature, ... */
+#define DSPARK_ERR_UNSUPPORTED 2 /* dtype pair or shape this build does not handle */
+#define DSPARK_ERR_CUDA 3        /* a CUDA runtime call or kernel launch failed */
+
+/* Bits of the device status word (dspark_markov_get_status). */
+#define DSPARK_STATUS_TOKEN_RANGE 1u /* a token id was outside [0, V); its bias was taken as 0 */
+#define DSPARK_STATUS_TIMEOUT 2u     /* a bounded device-side wait ran out; outputs are invalid */
+
+/* Element types. */
+#define DSPARK_DTYPE_FP32 0
+#define DSPARK_DTYPE_BF16 1
+
+/* Kernel selection (dspark_markov_set_algo). */
+#define DSPARK_ALGO_AUTO 0         /* tensor-core kernels where the shape allows, else generic */
+#define DSPARK_ALGO_GENERIC 1      /* CUDA-core kernels for any shape and dtype */
+#define DSPARK_ALGO_TENSOR_CORE 2  /* tcgen05 kernels only; other shapes return DSPARK_ERR_UNSUPPORTED */
+
+/*
+ * Teacher-forced corrected logits for every position at once
+ * (VanillaMarkov.apply_block_logits; markov_head API docs: "apply_block_logits").
+ *
+ *   base_logits    [rows, vocab] logits_dtype. The pages' [B, num_blocks, block_size, V]
+ *                  or (R, M, V) layouts flatten to rows = product of the leading dims.
+ *   out            [rows, vocab] logits_dtype. May equal base_logits (in place).
+ *   prev_token_ids [rows] int64: the teacher-forced previous token of each row.
+ *   w1, w2         [vocab, rank] weight_dtype (embedding table; Linear(rank, vocab) weight).
+ *   rank           > 0 (the head requires markov_rank > 0).
+ *
+ * rows == 0 is OK and enqueues nothing (the pages return the input itself when
+ * it is empty). The vanilla head ignores hidden states, so none are passed.
+ * Supported dtype pairs: (fp32, fp32), (bf16, bf16), (fp32 logits, bf16 weights),
+ * (bf16 logits, fp32 weights).
+ */
+int dspark_markov_apply_block_logits(const void* base_logits, void* out, const int64_t* prev_token_ids,
+                                     int64_t rows, int64_t vocab, const void* w1, const void* w2, int32_t rank,
+                                     int32_t logits_dtype, int32_t weight_dtype, void* stream);
+
+/*
+ * Left-to-right sampling of B blocks of M positions
+ * (VanillaMarkov.sample_block_tokens and _sample_tokens; markov_head API docs:
+ * "sample_block_tokens").
+ *
+ *   base_logits          [batch, proposal_len, vocab] logits_dtype.
+ *   first_prev_token_ids [batch] int64: the verified token before position 0.
+ *   sampled_tokens       [batch, proposal_len] int64, written.
+ *   corrected_logits     [batch, proposal_len, vocab] logits_dtype, written; the
+ *                        values before any division by the temperature. Must
+ *                        not overlap base_logits.
+ *
+ * Position k is corrected with the bias of the token chosen at k-1, and its own
+ * choice feeds position k+1 on the device. temperature < 1e-5 means greedy:
+ * the lowest index among the maxima of the ROUNDED corrected logits (NaN counts
+ * as the largest value). Otherwise one draw from softmax(c / T) per (b, k), as
+ * argmax_v(c_v / T + g_v) with Gumbel noise g = -log(-log u), u from
+ * Philox4x32-10 (Salmon et al., SC'11) with key (seed lo, seed hi), counter
+ * (v >> 2, k, b, 0), output word v & 3, and u = (2 * (word >> 9) + 1) * 2^-24.
+ * proposal_len == 0 is OK and enqueues nothing. NaN temperature is
+ * DSPARK_ERR_INVALID_ARG.
+ */
+int dspark_markov_sample_block(const void* base_logits, const int64_t* first_prev_token_ids, int64_t batch,
+                               int64_t proposal_len, int64_t vocab, const void* w1, const void* w2, int32_t rank,
+                               float temperature, uint64_t seed, int64_t* sampled_tokens, void* corrected_logits,
+                               int32_t logits_dtype, int32_t weight_dtype, void* stream);
+
+/*
+ * Synchronise `stream`, then read and clear the current device's status word
+ * (DSPARK_STATUS_* bits) into *status_out. Not part of the hot path.
+ */
+int dspark_markov_get_status(void* stream, int32_t* status_out);
+
+/* Text for a DSPARK_* return code. The string is static. */
+const char* dspark_markov_strerror(int code);
+
+/* Process-wide kernel selection (DSPARK_ALGO_*); returns the previous value. */
+int32_t dspark_markov_set_algo(int32_t algo);
+
+/* Number of kernels this library has launched in this process. */
+int64_t dspark_markov_launch_count(void);
+
+/*
+ * Test hooks. `wait_limit_ns` bounds every device-side wait (0 restores the
+ * default of about two seconds). `flags` bit 0 makes one CTA of the tensor-core
+ * sampler skip its grid-barrier arrival, so that the others' bounded wait runs
+ * out and reports DSPARK_STATUS_TIMEOUT; no GPU fault is involved.
+ */
+#define DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL 1u
+int dspark_markov_set_debug(uint32_t flags, uint64_t wait_limit_ns);
+
+/* Which kernel the last call on this thread selected: 0 none, 1 generic, 2 tensor core. */
+int32_t dspark_markov_last_algo(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSPARK_MARKOV_H */

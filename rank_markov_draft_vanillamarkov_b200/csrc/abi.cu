@@ -1,0 +1,278 @@
+// The C ABI (include/dspark_markov.h): argument checks, per-device state,
+// kernel selection and launches. Nothing here allocates or synchronises on the
+// hot path except the one-time per-device workspace (and its growth for a
+// larger sampler call).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/dspark_markov.h"
+#include "kernels.h"
+
+namespace dspark {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // about two seconds
+
+struct DeviceState {
+  bool ready = false;
+  int num_sms = 0;
+  uint32_t* status = nullptr;               // 1 word
+  unsigned char* workspace = nullptr;       // sampler keys + barrier counter
+  size_t workspace_bytes = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+std::atomic<int64_t> g_launches{0};
+std::atomic<int32_t> g_algo{DSPARK_ALGO_AUTO};
+std::atomic<uint32_t> g_debug_flags{0};
+std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
+thread_local int32_t t_last_algo = 0;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+void load_encoder() {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+          cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+}
+
+// Per-device state of the current device, created on first use.
+DeviceState* device_state(int* err) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    *err = DSPARK_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState& d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaMalloc(&d.status, sizeof(uint32_t)) != cudaSuccess || cudaMemset(d.status, 0, sizeof(uint32_t)) != cudaSuccess) {
+      *err = DSPARK_ERR_CUDA;
+      return nullptr;
+    }
+    d.ready = true;
+  }
+  return &d;
+}
+
+// Workspace of at least `bytes`, grown (never shrunk) on demand.
+unsigned char* workspace(DeviceState* d, size_t bytes) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (d->workspace_bytes < bytes) {
+    if (d->workspace) {
+      cudaDeviceSynchronize();
+      cudaFree(d->workspace);
+      d->workspace = nullptr;
+      d->workspace_bytes = 0;
+    }
+    size_t cap = 4096;
+    while (cap < bytes) cap <<= 1;
+    if (cudaMalloc(&d->workspace, cap) != cudaSuccess) return nullptr;
+    d->workspace_bytes = cap;
+  }
+  return d->workspace;
+}
+
+bool dtype_ok(int32_t t) { return t == DSPARK_DTYPE_FP32 || t == DSPARK_DTYPE_BF16; }
+
+int cuda_code(cudaError_t e) { return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA; }
+
+}  // namespace
+
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t rank, const void* base,
+                       const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                       CUtensorMapSwizzle swizzle) {
+  std::call_once(g_encode_once, load_encoder);
+  if (!g_encode) return false;
+  cuuint32_t elem_strides[5] = {1, 1, 1, 1, 1};
+  const CUresult r = g_encode(map, dtype, rank, const_cast<void*>(base), reinterpret_cast<const cuuint64_t*>(dims),
+                              reinterpret_cast<const cuuint64_t*>(strides_bytes),
+                              reinterpret_cast<const cuuint32_t*>(box), elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace dspark
+
+using namespace dspark;
+
+extern "C" {
+
+int dspark_markov_apply_block_logits(const void* base_logits, void* out, const int64_t* prev_token_ids, int64_t rows,
+                                     int64_t vocab, const void* w1, const void* w2, int32_t rank, int32_t logits_dtype,
+                                     int32_t weight_dtype, void* stream) {
+  t_last_algo = 0;
+  if (rows < 0 || vocab <= 0 || rank <= 0 || !dtype_ok(logits_dtype) || !dtype_ok(weight_dtype))
+    return DSPARK_ERR_INVALID_ARG;
+  if (rows == 0) return DSPARK_OK;
+  if (!base_logits || !out || !prev_token_ids || !w1 || !w2) return DSPARK_ERR_INVALID_ARG;
+  int err = DSPARK_OK;
+  DeviceState* d = device_state(&err);
+  if (!d) return err;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int32_t algo = g_algo.load();
+  const bool tc_ok = tc_apply_supported(rows, vocab, rank, logits_dtype, weight_dtype) &&
+                     (reinterpret_cast<uintptr_t>(base_logits) % 16 == 0) && (reinterpret_cast<uintptr_t>(out) % 16 == 0) &&
+                     (reinterpret_cast<uintptr_t>(w2) % 16 == 0) && (reinterpret_cast<uintptr_t>(w1) % 16 == 0);
+  if (algo == DSPARK_ALGO_TENSOR_CORE && !tc_ok) return DSPARK_ERR_UNSUPPORTED;
+  if (tc_ok && algo != DSPARK_ALGO_GENERIC) {
+    TcApplyArgs a{base_logits, out, prev_token_ids, rows, vocab, w1, w2, rank, d->status, g_wait_limit_ns.load()};
+    t_last_algo = 2;
+    return cuda_code(launch_tc_apply(a, d->num_sms, s));
+  }
+  GenericApplyArgs a{base_logits, out, prev_token_ids, rows, vocab, vocab, vocab, 1, w1, w2, rank, d->status};
+  t_last_algo = 1;
+  return cuda_code(launch_generic_apply(a, logits_dtype, weight_dtype, s));
+}
+
+int dspark_markov_sample_block(const void* base_logits, const int64_t* first_prev_token_ids, int64_t batch,
+                               int64_t proposal_len, int64_t vocab, const void* w1, const void* w2, int32_t rank,
+                               float temperature, uint64_t seed, int64_t* sampled_tokens, void* corrected_logits,
+                               int32_t logits_dtype, int32_t weight_dtype, void* stream) {
+  t_last_algo = 0;
+  if (batch < 0 || proposal_len < 0 || vocab <= 0 || rank <= 0 || !dtype_ok(logits_dtype) ||
+      !dtype_ok(weight_dtype) || std::isnan(temperature))
+    return DSPARK_ERR_INVALID_ARG;
+  if (batch == 0 || proposal_len == 0) return DSPARK_OK;
+  if (!base_logits || !first_prev_token_ids || !w1 || !w2 || !sampled_tokens || !corrected_logits)
+    return DSPARK_ERR_INVALID_ARG;
+  if (vocab > 0xfffffffell || proposal_len > 0x7fffffffll || batch > 0x7fffffffll) return DSPARK_ERR_UNSUPPORTED;
+  const size_t lsize = logits_dtype == DSPARK_DTYPE_BF16 ? 2 : 4;
+  {
+    // The corrected logits are written while base logits are still being read.
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(base_logits), c0 = reinterpret_cast<uintptr_t>(corrected_logits);
+    const uintptr_t n = (uintptr_t)(batch * proposal_len * vocab) * lsize;
+    if (a0 < c0 + n && c0 < a0 + n) return DSPARK_ERR_INVALID_ARG;
+  }
+  int err = DSPARK_OK;
+  DeviceState* d = device_state(&err);
+  if (!d) return err;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool greedy = !(temperature >= 1e-5f);
+  const int32_t algo = g_algo.load();
+  const bool tc_ok = tc_sample_supported(batch, vocab, rank, logits_dtype, weight_dtype) &&
+                     (reinterpret_cast<uintptr_t>(base_logits) % 16 == 0) &&
+                     (reinterpret_cast<uintptr_t>(corrected_logits) % 16 == 0) &&
+                     (reinterpret_cast<uintptr_t>(w2) % 16 == 0) && (reinterpret_cast<uintptr_t>(w1) % 16 == 0);
+  if (algo == DSPARK_ALGO_TENSOR_CORE && !tc_ok) return DSPARK_ERR_UNSUPPORTED;
+  if (tc_ok && algo != DSPARK_ALGO_GENERIC) {
+    const size_t keys_bytes = (size_t)batch * (size_t)proposal_len * sizeof(unsigned long long);
+    unsigned char* ws = workspace(d, keys_bytes + 256);
+    if (!ws) return DSPARK_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, keys_bytes + 256, s) != cudaSuccess) return DSPARK_ERR_CUDA;
+    TcSampleArgs a{};
+    a.base = base_logits;
+    a.first_prev = first_prev_token_ids;
+    a.batch = batch;
+    a.steps = proposal_len;
+    a.vocab = vocab;
+    a.w1 = w1;
+    a.w2 = w2;
+    a.rank = rank;
+    a.temperature = temperature;
+    a.greedy = greedy ? 1 : 0;
+    a.seed = seed;
+    a.tokens = sampled_tokens;
+    a.corrected = corrected_logits;
+    a.keys = reinterpret_cast<unsigned long long*>(ws);
+    a.barrier = reinterpret_cast<uint32_t*>(ws + keys_bytes);
+    a.status = d->status;
+    a.wait_limit_ns = g_wait_limit_ns.load();
+    a.debug_flags = g_debug_flags.load();
+    t_last_algo = 2;
+    return cuda_code(launch_tc_sample(a, d->num_sms, s));
+  }
+  // Generic path: one correction launch and one selection launch per step.
+  t_last_algo = 1;
+  for (int64_t k = 0; k < proposal_len; ++k) {
+    GenericApplyArgs a{};
+    a.base = static_cast<const char*>(base_logits) + (size_t)k * vocab * lsize;
+    a.out = static_cast<char*>(corrected_logits) + (size_t)k * vocab * lsize;
+    a.ids = k == 0 ? first_prev_token_ids : sampled_tokens + (k - 1);
+    a.rows = batch;
+    a.vocab = vocab;
+    a.ld_in = proposal_len * vocab;
+    a.ld_out = proposal_len * vocab;
+    a.ld_id = k == 0 ? 1 : proposal_len;
+    a.w1 = w1;
+    a.w2 = w2;
+    a.rank = rank;
+    a.status = d->status;
+    cudaError_t e = launch_generic_apply(a, logits_dtype, weight_dtype, s);
+    if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+    GenericSelectArgs sel{};
+    sel.corrected = a.out;
+    sel.ld_row = proposal_len * vocab;
+    sel.batch = batch;
+    sel.vocab = vocab;
+    sel.tokens = sampled_tokens + k;
+    sel.ld_tok = proposal_len;
+    sel.temperature = temperature;
+    sel.greedy = greedy ? 1 : 0;
+    sel.seed = seed;
+    sel.step = (uint32_t)k;
+    e = launch_generic_select(sel, logits_dtype, s);
+    if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+  }
+  return DSPARK_OK;
+}
+
+int dspark_markov_get_status(void* stream, int32_t* status_out) {
+  if (!status_out) return DSPARK_ERR_INVALID_ARG;
+  int err = DSPARK_OK;
+  DeviceState* d = device_state(&err);
+  if (!d) return err;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DSPARK_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, d->status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return DSPARK_ERR_CUDA;
+  if (cudaMemset(d->status, 0, sizeof(uint32_t)) != cudaSuccess) return DSPARK_ERR_CUDA;
+  *status_out = (int32_t)v;
+  return DSPARK_OK;
+}
+
+const char* dspark_markov_strerror(int code) {
+  switch (code) {
+    case DSPARK_OK: return "ok";
+    case DSPARK_ERR_INVALID_ARG: return "invalid argument";
+    case DSPARK_ERR_UNSUPPORTED: return "unsupported dtype or shape";
+    case DSPARK_ERR_CUDA: return "CUDA error";
+    default: return "unknown error";
+  }
+}
+
+int32_t dspark_markov_set_algo(int32_t algo) {
+  if (algo != DSPARK_ALGO_AUTO && algo != DSPARK_ALGO_GENERIC && algo != DSPARK_ALGO_TENSOR_CORE) return -1;
+  return g_algo.exchange(algo);
+}
+
+int64_t dspark_markov_launch_count(void) { return g_launches.load(); }
+
+int dspark_markov_set_debug(uint32_t flags, uint64_t wait_limit_ns) {
+  g_debug_flags.store(flags);
+  g_wait_limit_ns.store(wait_limit_ns ? wait_limit_ns : kDefaultWaitLimitNs);
+  return DSPARK_OK;
+}
+
+int32_t dspark_markov_last_algo(void) { return t_last_algo; }
+
+}  // extern "C"

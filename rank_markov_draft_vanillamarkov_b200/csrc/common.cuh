@@ -1,0 +1,92 @@
+// Shared device helpers of the Markov-head kernels: element conversion, the
+// packed argmax key, the device status word and Philox4x32-10.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/dspark_markov.h"
+
+namespace dspark {
+
+// ---------------------------------------------------------------------------
+// Element conversion. Corrected logits are rounded once, round-to-nearest-even.
+// ---------------------------------------------------------------------------
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// ---------------------------------------------------------------------------
+// Argmax key: the score's bits mapped to an unsigned order in the high word and
+// the complement of the vocabulary id in the low word, so that the largest key
+// is the largest score and, among equal scores, the lowest id. NaN is made a
+// single positive quiet NaN, which orders above +inf; -0 is made +0 so that
+// the two zeros tie, as they compare equal.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t orderable_bits(float s) {
+  uint32_t b = __float_as_uint(s);
+  if (s != s) b = 0x7fc00000u;
+  if (s == 0.0f) b = 0u;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ unsigned long long pack_key(float score, uint32_t v) {
+  return ((unsigned long long)orderable_bits(score) << 32) | (unsigned long long)(0xffffffffu - v);
+}
+
+__device__ __forceinline__ uint32_t key_token(unsigned long long key) {
+  return 0xffffffffu - (uint32_t)(key & 0xffffffffull);
+}
+
+__device__ __forceinline__ void report_status(uint32_t* status, uint32_t bits) {
+  if (status) atomicOr(status, bits);
+}
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy
+// as 1, 2, 3", SC'11): ten rounds of two 32x32->64 multiplies per round, the
+// key advanced by two Weyl constants between rounds.
+// ---------------------------------------------------------------------------
+struct Philox4 {
+  uint32_t x, y, z, w;
+};
+
+__device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+                                                 uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    const uint32_t lo0 = 0xD2511F53u * c0, hi0 = __umulhi(0xD2511F53u, c0);
+    const uint32_t lo1 = 0xCD9E8D57u * c2, hi1 = __umulhi(0xCD9E8D57u, c2);
+    const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return Philox4{c0, c1, c2, c3};
+}
+
+__device__ __forceinline__ uint32_t philox_word(const Philox4& p, uint32_t i) {
+  return i == 0 ? p.x : i == 1 ? p.y : i == 2 ? p.z : p.w;
+}
+
+// u = (2 * (w >> 9) + 1) * 2^-24 lies strictly inside (0, 1) and is exact in
+// binary32. The Gumbel variate is g = -log(-log u).
+__device__ __forceinline__ float gumbel_from_word(uint32_t w) {
+  const float u = (float)(2u * (w >> 9) + 1u) * 5.9604644775390625e-08f;  // 2^-24
+  return -logf(-logf(u));
+}
+
+__device__ __forceinline__ float noise_for(uint64_t seed, uint32_t b, uint32_t k, uint32_t v) {
+  const Philox4 p = philox4x32_10(v >> 2, k, b, 0u, (uint32_t)seed, (uint32_t)(seed >> 32));
+  return gumbel_from_word(philox_word(p, v & 3u));
+}
+
+}  // namespace dspark

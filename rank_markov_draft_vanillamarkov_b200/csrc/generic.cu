@@ -1,0 +1,126 @@
+// Generic (CUDA-core) kernels of the Markov head: any vocabulary size, any
+// rank, fp32 or bf16 logits and weights. They serve the fp32 workloads and
+// the shapes the tensor-core kernels do not take (vocab not a multiple of 8,
+// rank not a multiple of 64, batch above 256 in the sampler).
+//
+// apply:  one CTA per (row, 1024-wide vocab slice). The CTA stages the row's
+//         latent W1[prev] in shared memory; each thread forms the fp32 dot
+//         product with W2[v, :] for four ids, adds U and rounds once.
+// select: one CTA per batch row; every thread scans a strided part of the
+//         corrected row keeping the largest packed (score, -id) key, then the
+//         CTA reduces the keys.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dspark {
+
+namespace {
+
+constexpr int kApplyThreads = 256;
+constexpr int kApplyIdsPerThread = 4;
+constexpr int kApplySlice = kApplyThreads * kApplyIdsPerThread;
+constexpr int kSelectThreads = 512;
+
+template <typename TL, typename TW>
+__global__ void __launch_bounds__(kApplyThreads) generic_apply_kernel(GenericApplyArgs a) {
+  extern __shared__ float latent[];
+  const int64_t row = blockIdx.x;
+  const int64_t id = a.ids[row * a.ld_id];
+  const bool valid = id >= 0 && id < a.vocab;
+  if (!valid && threadIdx.x == 0 && blockIdx.y == 0) report_status(a.status, DSPARK_STATUS_TOKEN_RANGE);
+  const TW* w1 = static_cast<const TW*>(a.w1);
+  const TW* w2 = static_cast<const TW*>(a.w2);
+  for (int j = threadIdx.x; j < a.rank; j += blockDim.x) latent[j] = valid ? to_f32(w1[id * a.rank + j]) : 0.0f;
+  __syncthreads();
+  const TL* in = static_cast<const TL*>(a.base) + row * a.ld_in;
+  TL* out = static_cast<TL*>(a.out) + row * a.ld_out;
+  const int64_t v0 = (int64_t)blockIdx.y * kApplySlice + threadIdx.x;
+#pragma unroll
+  for (int i = 0; i < kApplyIdsPerThread; ++i) {
+    const int64_t v = v0 + (int64_t)i * kApplyThreads;
+    if (v >= a.vocab) break;
+    const TW* wrow = w2 + v * a.rank;
+    float acc = 0.0f;
+    for (int j = 0; j < a.rank; ++j) acc = fmaf(latent[j], to_f32(wrow[j]), acc);
+    out[v] = from_f32<TL>(to_f32(in[v]) + acc);
+  }
+}
+
+__device__ __forceinline__ unsigned long long max_u64(unsigned long long a, unsigned long long b) {
+  return a > b ? a : b;
+}
+
+template <typename TL>
+__global__ void __launch_bounds__(kSelectThreads) generic_select_kernel(GenericSelectArgs a) {
+  __shared__ unsigned long long warp_best[kSelectThreads / 32];
+  const int64_t b = blockIdx.x;
+  const TL* row = static_cast<const TL*>(a.corrected) + b * a.ld_row;
+  unsigned long long best = 0ull;
+  for (int64_t v = threadIdx.x; v < a.vocab; v += blockDim.x) {
+    float s = to_f32(row[v]);
+    if (!a.greedy) s = s / a.temperature + noise_for(a.seed, (uint32_t)b, a.step, (uint32_t)v);
+    best = max_u64(best, pack_key(s, (uint32_t)v));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) best = max_u64(best, __shfl_xor_sync(0xffffffffu, best, o));
+  if ((threadIdx.x & 31) == 0) warp_best[threadIdx.x >> 5] = best;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    best = threadIdx.x < kSelectThreads / 32 ? warp_best[threadIdx.x] : 0ull;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) best = max_u64(best, __shfl_xor_sync(0xffffffffu, best, o));
+    if (threadIdx.x == 0) a.tokens[b * a.ld_tok] = (int64_t)key_token(best);
+  }
+}
+
+template <typename TL, typename TW>
+cudaError_t launch_apply_t(const GenericApplyArgs& a, cudaStream_t stream) {
+  const int64_t slices = (a.vocab + kApplySlice - 1) / kApplySlice;
+  if (slices > 65535) return cudaErrorInvalidConfiguration;
+  const size_t smem = (size_t)a.rank * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(generic_apply_kernel<TL, TW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  // Rows go on grid.x (up to 2^31 - 1); chunk anyway to keep offsets simple.
+  const int64_t kMaxRows = 1ll << 30;
+  for (int64_t r0 = 0; r0 < a.rows; r0 += kMaxRows) {
+    GenericApplyArgs c = a;
+    c.rows = a.rows - r0 < kMaxRows ? a.rows - r0 : kMaxRows;
+    c.base = static_cast<const char*>(a.base) + r0 * a.ld_in * (int64_t)sizeof(TL);
+    c.out = static_cast<char*>(a.out) + r0 * a.ld_out * (int64_t)sizeof(TL);
+    c.ids = a.ids + r0 * a.ld_id;
+    dim3 grid((unsigned)c.rows, (unsigned)slices);
+    generic_apply_kernel<TL, TW><<<grid, kApplyThreads, smem, stream>>>(c);
+    note_launch();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_generic_apply(const GenericApplyArgs& a, int logits_dtype, int weight_dtype, cudaStream_t s) {
+  if (a.rows == 0) return cudaSuccess;
+  if (logits_dtype == DSPARK_DTYPE_FP32 && weight_dtype == DSPARK_DTYPE_FP32) return launch_apply_t<float, float>(a, s);
+  if (logits_dtype == DSPARK_DTYPE_BF16 && weight_dtype == DSPARK_DTYPE_BF16)
+    return launch_apply_t<__nv_bfloat16, __nv_bfloat16>(a, s);
+  if (logits_dtype == DSPARK_DTYPE_FP32 && weight_dtype == DSPARK_DTYPE_BF16)
+    return launch_apply_t<float, __nv_bfloat16>(a, s);
+  return launch_apply_t<__nv_bfloat16, float>(a, s);
+}
+
+cudaError_t launch_generic_select(const GenericSelectArgs& a, int logits_dtype, cudaStream_t s) {
+  if (a.batch == 0) return cudaSuccess;
+  if (a.batch > 0x7fffffffll) return cudaErrorInvalidConfiguration;
+  if (logits_dtype == DSPARK_DTYPE_FP32)
+    generic_select_kernel<float><<<(unsigned)a.batch, kSelectThreads, 0, s>>>(a);
+  else
+    generic_select_kernel<__nv_bfloat16><<<(unsigned)a.batch, kSelectThreads, 0, s>>>(a);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace dspark

@@ -1,0 +1,86 @@
+// Internal interface between the C-ABI layer (abi.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dspark {
+
+// Counts kernel launches made by this library (dspark_markov_launch_count).
+void note_launch();
+
+// ---------------------------------------------------------------- generic --
+struct GenericApplyArgs {
+  const void* base;      // row i at base + i * ld_in elements
+  void* out;             // row i at out + i * ld_out elements
+  const int64_t* ids;    // prev id of row i at ids[i * ld_id]
+  int64_t rows, vocab;
+  int64_t ld_in, ld_out, ld_id;
+  const void* w1;
+  const void* w2;
+  int32_t rank;
+  uint32_t* status;
+};
+
+struct GenericSelectArgs {
+  const void* corrected;  // row b at corrected + b * ld_row elements
+  int64_t ld_row;
+  int64_t batch, vocab;
+  int64_t* tokens;  // token of row b at tokens[b * ld_tok]
+  int64_t ld_tok;
+  float temperature;
+  int32_t greedy;
+  uint64_t seed;
+  uint32_t step;
+};
+
+cudaError_t launch_generic_apply(const GenericApplyArgs& a, int logits_dtype, int weight_dtype, cudaStream_t s);
+cudaError_t launch_generic_select(const GenericSelectArgs& a, int logits_dtype, cudaStream_t s);
+
+// ----------------------------------------------------------- tensor core --
+// Teacher-forced apply on tcgen05: bf16 logits, bf16 weights,
+// vocab % 8 == 0, rank in {64, 128, 192, 256}.
+struct TcApplyArgs {
+  const void* base;
+  void* out;
+  const int64_t* ids;
+  int64_t rows, vocab;
+  const void* w1;
+  const void* w2;
+  int32_t rank;
+  uint32_t* status;
+  uint64_t wait_limit_ns;
+};
+bool tc_apply_supported(int64_t rows, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype);
+cudaError_t launch_tc_apply(const TcApplyArgs& a, int num_sms, cudaStream_t s);
+
+// Persistent left-to-right sampler on tcgen05: bf16 logits, bf16 weights,
+// vocab % 8 == 0, rank in {64, 128, 192, 256}, batch <= 256.
+struct TcSampleArgs {
+  const void* base;
+  const int64_t* first_prev;
+  int64_t batch, steps, vocab;
+  const void* w1;
+  const void* w2;
+  int32_t rank;
+  float temperature;
+  int32_t greedy;
+  uint64_t seed;
+  int64_t* tokens;
+  void* corrected;
+  unsigned long long* keys;  // [steps, batch] workspace, zeroed by the launcher
+  uint32_t* barrier;         // grid-barrier counter, zeroed by the launcher
+  uint32_t* status;
+  uint64_t wait_limit_ns;
+  uint32_t debug_flags;
+};
+bool tc_sample_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype);
+cudaError_t launch_tc_sample(const TcSampleArgs& a, int num_sms, cudaStream_t s);
+
+// Encodes a tiled TMA descriptor through the driver entry point.
+bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t rank, const void* base,
+                       const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                       CUtensorMapSwizzle swizzle);
+
+}  // namespace dspark

@@ -1,0 +1,558 @@
+// Left-to-right block sampling on the sm_100a tensor cores
+// (VanillaMarkov.sample_block_tokens and _sample_tokens of the vendored
+// markov_head.py). For k = 0 .. M-1 and every block b:
+//
+//     c_k[b, v] = round_bf16( U[b, k, v] + sum_j W1[x_{k-1}[b], j] * W2[v, j] )
+//     x_k[b]    = argmax_v c_k[b, v]                    (greedy)
+//              or argmax_v c_k[b, v] / T + g(b, k, v)   (Gumbel-max, Philox noise)
+//
+// with x_{-1} = first_prev. One launch covers all M steps. The grid is one
+// CTA per SM (cooperative launch, so all CTAs are resident); CTA c owns a
+// contiguous run of 128-id vocabulary tiles. Per step each CTA
+//   - computes bias^T = W2_tile[128 x r] . X^T[r x B] on tcgen05 (swap-AB:
+//     M = 128 ids, N = B padded to 16, K = r), X = the gathered W1 rows of
+//     x_{k-1}; W2 tiles come from L2 (loaded with an evict-last policy, so
+//     the M steps re-read them from L2, not HBM);
+//   - adds U (TMA-staged [B x 128] tiles, prefetched across step boundaries
+//     since U does not depend on the chain), rounds to bf16, stores c_k, and
+//     keeps the packed (score, -id) maximum per b;
+//   - merges its maxima into a per-(k, b) 64-bit key with atomicMax, then
+//     passes a grid barrier (bounded wait) after which every CTA decodes x_k.
+//
+// Warp roles (288 threads): 0 W2 producer, 1 MMA issuer + TMEM owner, 2 U
+// producer, 3 W1 gather + grid barrier, 4-7 epilogue (thread = vocab id).
+#include "common.cuh"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace dspark {
+namespace {
+
+constexpr int kBV = 128;               // vocabulary ids per tile (MMA M)
+constexpr int kAtomK = 64;             // bf16 elements per 128-byte swizzle row
+constexpr int kW2AtomBytes = 128 * 128;
+constexpr int kThreads = 288;
+constexpr int kMaxStages = 12;
+constexpr int kMaxBatch = 256;
+constexpr size_t kSmemLimit = 232448;  // dynamic shared memory per block on sm_100
+
+struct __align__(64) SampleMaps {
+  CUtensorMap w2;   // [vocab, rank] bf16, box 64 x 128, 128B swizzle
+  CUtensorMap u;    // [batch, steps, vocab] bf16, box 128 x 1 x batch
+  CUtensorMap out;  // same geometry as u
+};
+
+struct SampleParams {
+  const int64_t* first_prev;
+  const __nv_bfloat16* w1;
+  int64_t* tokens;
+  unsigned long long* keys;
+  uint32_t* barrier;
+  uint32_t* status;
+  int32_t batch, batch_pad, steps, rank;
+  int64_t vocab;
+  int32_t vocab_tiles;
+  int32_t w2_slots, u_slots;
+  uint32_t u_slot_bytes, x_bytes;  // x_bytes: one step's gathered operand
+  float temperature;
+  int32_t greedy;
+  uint64_t seed;
+  uint64_t wait_limit_ns;
+  uint32_t debug_flags;
+  uint32_t tmem_cols;
+};
+
+struct SampleTail {
+  uint64_t w2_full[kMaxStages], w2_empty[kMaxStages];
+  uint64_t u_full[kMaxStages], u_empty[kMaxStages];
+  uint64_t x_full[2], x_empty[2];
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int is_last;
+};
+
+__device__ __forceinline__ bool barrier_and(bool v, uint32_t id, uint32_t n) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"((uint32_t)v), "r"(id), "r"(n)
+      : "memory");
+  return out != 0;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ unsigned long long ld_relaxed_gpu(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsigned long long b) {
+  return a > b ? a : b;
+}
+
+// Thirty-two keys per lane in; lane L leaves with the warp-wide maximum of key
+// index L. Each round halves the keys a lane holds: it keeps the half whose
+// index bit matches its own lane bit and trades the other half with the lane
+// across that bit.
+__device__ __forceinline__ unsigned long long transpose_max32(unsigned long long (&k)[32], int lane) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < o; ++j) {
+      const unsigned long long send = upper ? k[j] : k[j + o];
+      const unsigned long long keep = upper ? k[j + o] : k[j];
+      const unsigned long long recv = __shfl_xor_sync(0xffffffffu, send, o);
+      k[j] = umax64(keep, recv);
+    }
+  }
+  return k[0];
+}
+
+template <int KA>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_sample_kernel(const __grid_constant__ SampleMaps maps, const SampleParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* w2_smem = smem;                                            // w2_slots x KA atoms
+  uint8_t* x_smem = w2_smem + (size_t)p.w2_slots * KA * kW2AtomBytes;  // 2 x x_bytes
+  uint8_t* u_smem = x_smem + 2 * (size_t)p.x_bytes;                   // u_slots x u_slot_bytes
+  unsigned long long* red = reinterpret_cast<unsigned long long*>(u_smem + (size_t)p.u_slots * p.u_slot_bytes);
+  SampleTail* sh = reinterpret_cast<SampleTail*>(red + 4 * p.batch_pad);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int G = gridDim.x;
+  const int t_begin = (int)((int64_t)p.vocab_tiles * blockIdx.x / G);
+  const int t_end = (int)((int64_t)p.vocab_tiles * (blockIdx.x + 1) / G);
+  const int nt = t_end - t_begin;
+  const int M = p.steps;
+  const int B = p.batch;
+  const int BB = p.batch_pad;
+  const int64_t items = (int64_t)M * nt;
+  const uint32_t atom_x = (uint32_t)BB * 128u;  // bytes of one X atom
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < p.w2_slots; ++i) {
+      mbar_init(&sh->w2_full[i], 1);
+      mbar_init(&sh->w2_empty[i], 1);
+    }
+    for (int i = 0; i < p.u_slots; ++i) {
+      mbar_init(&sh->u_full[i], 1);
+      mbar_init(&sh->u_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh->x_full[i], 32);
+      mbar_init(&sh->x_empty[i], 1);
+      mbar_init(&sh->acc_full[i], 1);
+      mbar_init(&sh->acc_empty[i], 4);
+    }
+    mbar_init(&sh->drain, 1);
+    sh->abort_flag = 0;
+    sh->is_last = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sh->tmem_base, p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = sh->tmem_base;
+  const WaitCtl ctl{&sh->abort_flag, p.status, p.wait_limit_ns};
+  volatile int never = 0;
+  const WaitCtl drain_ctl{&never, p.status, p.wait_limit_ns};
+
+  if (warp == 0) {
+    // ----------------------------------------------- W2 producer ----
+    if (lane == 0) {
+      prefetch_tensormap(&maps.w2);
+      const uint64_t pol_keep = policy_evict_last();
+      int64_t i = 0;
+      for (; i < items; ++i) {
+        const int t = t_begin + (int)(i % nt);
+        const int w = (int)(i % p.w2_slots);
+        if (!mbar_wait(&sh->w2_empty[w], ((uint32_t)(i / p.w2_slots) & 1u) ^ 1u, ctl)) break;
+        mbar_arrive_expect_tx(&sh->w2_full[w], KA * kW2AtomBytes);
+        uint8_t* dst = w2_smem + (size_t)w * KA * kW2AtomBytes;
+#pragma unroll
+        for (int ka = 0; ka < KA; ++ka)
+          tma_load_2d(dst + ka * kW2AtomBytes, &maps.w2, &sh->w2_full[w], ka * kAtomK, t * kBV, pol_keep);
+      }
+      // Drain: wait for the last fill of every slot this thread started.
+      for (int64_t j = (i > p.w2_slots ? i - p.w2_slots : 0); j < i; ++j)
+        mbar_wait(&sh->w2_full[j % p.w2_slots], (uint32_t)(j / p.w2_slots) & 1u, drain_ctl);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------ U producer ----
+    if (lane == 0) {
+      prefetch_tensormap(&maps.u);
+      prefetch_tensormap(&maps.out);
+      const uint64_t pol_stream = policy_evict_first();
+      int64_t i = 0;
+      for (; i < items; ++i) {
+        const int k = (int)(i / nt);
+        const int t = t_begin + (int)(i % nt);
+        const int s = (int)(i % p.u_slots);
+        if (!mbar_wait(&sh->u_empty[s], ((uint32_t)(i / p.u_slots) & 1u) ^ 1u, ctl)) break;
+        mbar_arrive_expect_tx(&sh->u_full[s], p.u_slot_bytes);
+        tma_load_3d(u_smem + (size_t)s * p.u_slot_bytes, &maps.u, &sh->u_full[s], t * kBV, k, 0, pol_stream);
+      }
+      for (int64_t j = (i > p.u_slots ? i - p.u_slots : 0); j < i; ++j)
+        mbar_wait(&sh->u_full[j % p.u_slots], (uint32_t)(j / p.u_slots) & 1u, drain_ctl);
+    }
+  } else if (warp == 3) {
+    // ------------------------------------ W1 gather + grid barrier ----
+    for (int k = 0; k < M; ++k) {
+      const int xb = k & 1;
+      const uint32_t xe_par = ((uint32_t)(k >> 1) & 1u) ^ 1u;
+      // Lane 0 decides and the warp follows, so the lanes never split around
+      // the warp-wide shuffles below.
+      bool xe_ok = lane == 0 ? mbar_wait(&sh->x_empty[xb], xe_par, ctl) : true;
+      xe_ok = __shfl_sync(0xffffffffu, xe_ok ? 1 : 0, 0) != 0;
+      if (!xe_ok) break;
+      if (lane != 0) mbar_wait(&sh->x_empty[xb], xe_par, ctl);  // already complete
+      if (k > 0) {
+        // Every CTA has merged its step k-1 maxima once the counter reaches k * G.
+        bool ok = true;
+        if (lane == 0) {
+          const uint32_t target = (uint32_t)k * (uint32_t)G;
+          const uint64_t t0 = globaltimer_ns();
+          while (ld_acquire_gpu(p.barrier) < target) {
+            if (*ctl.abort_flag) {
+              ok = false;
+              break;
+            }
+            if (globaltimer_ns() - t0 > p.wait_limit_ns) {
+              *ctl.abort_flag = 1;
+              atomicOr(p.status, DSPARK_STATUS_TIMEOUT);
+              ok = false;
+              break;
+            }
+            __nanosleep(64);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        __syncwarp();
+        if (!ok) break;
+      }
+      uint8_t* xdst = x_smem + (size_t)xb * p.x_bytes;
+      bool bad = false;
+      for (int b0 = 0; b0 < BB; b0 += 32) {
+        int64_t id = -1;
+        const int b = b0 + lane;
+        if (b < B) {
+          id = k == 0 ? p.first_prev[b] : (int64_t)key_token(ld_relaxed_gpu(&p.keys[(size_t)(k - 1) * B + b]));
+          if (k > 0 && blockIdx.x == 0) p.tokens[(size_t)b * M + (k - 1)] = id;
+          if (id < 0 || id >= p.vocab) {
+            bad = true;
+            id = -1;
+          }
+        }
+        // lane j of this pass holds the id of row b0 + j; rows are gathered
+        // 4 at a time per warp pass (8 chunks each).
+        for (int r = 0; r < 32 && b0 + r < BB; r += 4) {
+          const int row = b0 + r + (lane >> 3);
+          const int j = lane & 7;
+          const int64_t rid = __shfl_sync(0xffffffffu, id, r + (lane >> 3));
+#pragma unroll
+          for (int ka = 0; ka < KA; ++ka) {
+            uint4 val = make_uint4(0u, 0u, 0u, 0u);
+            if (rid >= 0) val = ld_nc_v4(p.w1 + rid * p.rank + ka * kAtomK + j * 8);
+            *reinterpret_cast<uint4*>(xdst + ka * atom_x + row * 128 + ((j ^ (row & 7)) << 4)) = val;
+          }
+        }
+      }
+      if (bad) report_status(p.status, DSPARK_STATUS_TOKEN_RANGE);
+      fence_proxy_async_smem();
+      mbar_arrive(&sh->x_full[xb]);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------- MMA issuer ----
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kBV, (uint32_t)BB);
+      const uint32_t w2_addr = smem_u32(w2_smem);
+      const uint32_t x_addr = smem_u32(x_smem);
+      bool ok = true;
+      for (int k = 0; k < M && ok; ++k) {
+        const int xb = k & 1;
+        if (!mbar_wait(&sh->x_full[xb], (uint32_t)(k >> 1) & 1u, ctl)) break;
+        for (int tt = 0; tt < nt; ++tt) {
+          const int64_t i = (int64_t)k * nt + tt;
+          const int w = (int)(i % p.w2_slots);
+          const int abuf = (int)(i & 1);
+          if (!mbar_wait(&sh->w2_full[w], (uint32_t)(i / p.w2_slots) & 1u, ctl) ||
+              !mbar_wait(&sh->acc_empty[abuf], ((uint32_t)(i >> 1) & 1u) ^ 1u, ctl)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t d_tmem = tmem_base + (uint32_t)(abuf * BB);
+#pragma unroll
+          for (int ka = 0; ka < KA; ++ka) {
+#pragma unroll
+            for (int kk = 0; kk < kAtomK / 16; ++kk) {
+              const uint64_t ad = sw128_kmajor_desc(w2_addr + (uint32_t)(w * KA + ka) * kW2AtomBytes + kk * 32);
+              const uint64_t bd = sw128_kmajor_desc(x_addr + (uint32_t)xb * p.x_bytes + ka * atom_x + kk * 32);
+              umma_bf16_ss(d_tmem, ad, bd, idesc, (ka | kk) != 0);
+            }
+          }
+          umma_commit(&sh->w2_empty[w]);
+          umma_commit(&sh->acc_full[abuf]);
+        }
+        if (ok) umma_commit(&sh->x_empty[xb]);
+      }
+      umma_commit(&sh->drain);
+      mbar_wait(&sh->drain, 0, drain_ctl);
+    }
+  } else {
+    // -------------------------------------------------- epilogue ----
+    const int et = threadIdx.x - 128;  // vocabulary id within the tile = TMEM lane
+    const int q = warp & 3;
+    const int groups = (B + 31) >> 5;
+    int prev_s = -1;
+    bool ok = true;
+    for (int k = 0; k < M && ok; ++k) {
+      unsigned long long best[kMaxBatch / 32];
+#pragma unroll
+      for (int g = 0; g < kMaxBatch / 32; ++g) best[g] = 0ull;
+      for (int tt = 0; tt < nt; ++tt) {
+        const int64_t i = (int64_t)k * nt + tt;
+        const int s = (int)(i % p.u_slots);
+        const int abuf = (int)(i & 1);
+        const uint32_t acc_par = (uint32_t)(i >> 1) & 1u;
+        const uint32_t u_par = (uint32_t)(i / p.u_slots) & 1u;
+        bool w_ok = true;
+        if (et == 0) w_ok = mbar_wait(&sh->acc_full[abuf], acc_par, ctl) && mbar_wait(&sh->u_full[s], u_par, ctl);
+        if (!barrier_and(w_ok, 1, 128)) {
+          ok = false;
+          break;
+        }
+        if (et != 0) {
+          mbar_wait(&sh->acc_full[abuf], acc_par, ctl);
+          mbar_wait(&sh->u_full[s], u_par, ctl);
+        }
+        tc_fence_after_sync();
+        const int t = t_begin + tt;
+        const uint32_t v = (uint32_t)(t * kBV + et);
+        const bool valid = (int64_t)v < p.vocab;
+        __nv_bfloat16* slot = reinterpret_cast<__nv_bfloat16*>(u_smem + (size_t)s * p.u_slot_bytes);
+        const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(abuf * BB);
+#pragma unroll
+        for (int g = 0; g < kMaxBatch / 32; ++g) {
+          if (g >= groups) break;
+          uint32_t d[32];
+          tmem_ld_32x32b_x16(tb + 32 * g, *reinterpret_cast<uint32_t(*)[16]>(&d[0]));
+          if (32 * g + 16 < BB) tmem_ld_32x32b_x16(tb + 32 * g + 16, *reinterpret_cast<uint32_t(*)[16]>(&d[16]));
+          tmem_ld_wait();
+          unsigned long long key[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int b = 32 * g + j;
+            key[j] = 0ull;
+            if (b < B) {
+              __nv_bfloat16* e = slot + (size_t)b * kBV + et;
+              const __nv_bfloat16 c = __float2bfloat16_rn(__bfloat162float(*e) + __uint_as_float(d[j]));
+              *e = c;
+              float score = __bfloat162float(c);
+              if (!p.greedy) score = score / p.temperature + noise_for(p.seed, (uint32_t)b, (uint32_t)k, v);
+              if (valid) key[j] = pack_key(score, v);
+            }
+          }
+          best[g] = umax64(best[g], transpose_max32(key, lane));
+        }
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->acc_empty[abuf]);
+        fence_proxy_async_smem();
+        named_barrier_sync(1, 128);
+        if (et == 0) {
+          tma_store_3d(&maps.out, slot, t * kBV, k, 0);
+          bulk_commit_group();
+          if (prev_s >= 0) {
+            bulk_wait_group_read<1>();
+            mbar_arrive(&sh->u_empty[prev_s]);
+          }
+          prev_s = s;
+        }
+      }
+      if (!ok) break;
+      // Merge the four warps' maxima, then this CTA's into the global keys.
+#pragma unroll
+      for (int g = 0; g < kMaxBatch / 32; ++g)
+        if (g < groups) red[q * BB + 32 * g + lane] = best[g];
+      named_barrier_sync(1, 128);
+      for (int b = et; b < B; b += 128) {
+        const unsigned long long m = umax64(umax64(red[b], red[BB + b]), umax64(red[2 * BB + b], red[3 * BB + b]));
+        atomicMax(&p.keys[(size_t)k * B + b], m);
+      }
+      __threadfence();
+      named_barrier_sync(1, 128);
+      if (et == 0) {
+        const bool skip = (p.debug_flags & DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL) && blockIdx.x == 0 && k == 0;
+        int last = 0;
+        if (!skip) {
+          __threadfence();
+          const uint32_t ticket = atomicAdd(p.barrier, 1u);
+          last = (k == M - 1) && ticket == (uint32_t)M * (uint32_t)G - 1u;
+        }
+        sh->is_last = last;
+      }
+      if (k == M - 1) {
+        named_barrier_sync(1, 128);
+        if (sh->is_last) {
+          __threadfence();
+          for (int b = et; b < B; b += 128)
+            p.tokens[(size_t)b * M + (M - 1)] = (int64_t)key_token(ld_relaxed_gpu(&p.keys[(size_t)(M - 1) * B + b]));
+        }
+      }
+    }
+    if (et == 0) bulk_wait_group<0>();
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  if (warp == 1) tmem_dealloc(tmem_base, p.tmem_cols);
+}
+
+struct SampleConfig {
+  int w2_slots, u_slots;
+  uint32_t u_slot_bytes, x_bytes;
+  size_t smem_bytes;
+  bool ok;
+};
+
+size_t align1024(size_t x) { return (x + 1023) & ~size_t(1023); }
+
+SampleConfig plan(int ka, int batch, int batch_pad) {
+  SampleConfig c{};
+  c.u_slot_bytes = (uint32_t)align1024((size_t)batch * kBV * 2);
+  c.x_bytes = (uint32_t)((size_t)ka * batch_pad * 128);
+  const size_t fixed = 1024 + 2 * (size_t)c.x_bytes + 4 * (size_t)batch_pad * 8 + sizeof(SampleTail) + 64;
+  const size_t w2_slot = (size_t)ka * kW2AtomBytes;
+  for (int w = 4; w >= 2; --w) {
+    for (int u = 8; u >= 2; --u) {
+      const size_t total = fixed + w * w2_slot + u * (size_t)c.u_slot_bytes;
+      if (total <= kSmemLimit) {
+        c.w2_slots = w;
+        c.u_slots = u;
+        c.smem_bytes = total;
+        c.ok = true;
+        return c;
+      }
+    }
+  }
+  c.ok = false;
+  return c;
+}
+
+int batch_pad_of(int64_t batch) { return (int)(((batch + 15) / 16) * 16); }
+
+uint32_t tmem_cols_for(int batch_pad) {
+  uint32_t need = 2u * (uint32_t)batch_pad, cols = 32;
+  while (cols < need) cols <<= 1;
+  return cols;
+}
+
+template <int KA>
+cudaError_t launch_ka(const TcSampleArgs& a, int num_sms, cudaStream_t stream) {
+  const int BB = batch_pad_of(a.batch);
+  const SampleConfig c = plan(KA, (int)a.batch, BB);
+  if (!c.ok) return cudaErrorInvalidValue;
+  SampleMaps maps;
+  const uint32_t wbox[2] = {64, 128};
+  const uint64_t wdim[2] = {(uint64_t)a.rank, (uint64_t)a.vocab};
+  const uint64_t wstr[1] = {(uint64_t)a.rank * 2};
+  if (!encode_tensor_map(&maps.w2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.w2, wdim, wstr, wbox,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  const uint64_t udim[3] = {(uint64_t)a.vocab, (uint64_t)a.steps, (uint64_t)a.batch};
+  const uint64_t ustr[2] = {(uint64_t)a.vocab * 2, (uint64_t)a.vocab * 2 * (uint64_t)a.steps};
+  const uint32_t ubox[3] = {(uint32_t)kBV, 1u, (uint32_t)a.batch};
+  if (!encode_tensor_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.base, udim, ustr, ubox,
+                         CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_tensor_map(&maps.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.corrected, udim, ustr, ubox,
+                         CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+
+  SampleParams p{};
+  p.first_prev = a.first_prev;
+  p.w1 = static_cast<const __nv_bfloat16*>(a.w1);
+  p.tokens = a.tokens;
+  p.keys = a.keys;
+  p.barrier = a.barrier;
+  p.status = a.status;
+  p.batch = (int32_t)a.batch;
+  p.batch_pad = BB;
+  p.steps = (int32_t)a.steps;
+  p.rank = a.rank;
+  p.vocab = a.vocab;
+  p.vocab_tiles = (int32_t)((a.vocab + kBV - 1) / kBV);
+  p.w2_slots = c.w2_slots;
+  p.u_slots = c.u_slots;
+  p.u_slot_bytes = c.u_slot_bytes;
+  p.x_bytes = c.x_bytes;
+  p.temperature = a.temperature;
+  p.greedy = a.greedy;
+  p.seed = a.seed;
+  p.wait_limit_ns = a.wait_limit_ns;
+  p.debug_flags = a.debug_flags;
+  p.tmem_cols = tmem_cols_for(BB);
+
+  cudaError_t e = cudaFuncSetAttribute(tc_sample_kernel<KA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)c.smem_bytes);
+  if (e != cudaSuccess) return e;
+  const int grid = p.vocab_tiles < num_sms ? p.vocab_tiles : num_sms;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = c.smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, tc_sample_kernel<KA>, maps, p);
+  note_launch();
+  return e;
+}
+
+}  // namespace
+
+bool tc_sample_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype) {
+  if (logits_dtype != DSPARK_DTYPE_BF16 || weight_dtype != DSPARK_DTYPE_BF16) return false;
+  if (vocab % 8 != 0 || rank % 64 != 0 || rank < 64 || rank > 256) return false;
+  if (batch < 1 || batch > kMaxBatch) return false;
+  if (vocab >= (1ll << 31) - kBV) return false;
+  return plan(rank / 64, (int)batch, batch_pad_of(batch)).ok;
+}
+
+cudaError_t launch_tc_sample(const TcSampleArgs& a, int num_sms, cudaStream_t s) {
+  switch (a.rank / 64) {
+    case 1: return launch_ka<1>(a, num_sms, s);
+    case 2: return launch_ka<2>(a, num_sms, s);
+    case 3: return launch_ka<3>(a, num_sms, s);
+    case 4: return launch_ka<4>(a, num_sms, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace dspark

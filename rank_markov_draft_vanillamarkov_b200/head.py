@@ -1,0 +1,190 @@
+"""``VanillaMarkov``: the rank-r Markov transition-bias head on B200.
+
+Python face of the C ABI: torch tensors supply device memory and the current
+CUDA stream; every step of the computation runs in the library's kernels.
+
+The method (markov_head.py, the vendored DSpark-style low-rank Markov head,
+module docstring "WHAT THIS IS"; nemo_automodel ...speculative.dspark.markov_head
+API docs, ``VanillaMarkov``): a parallel block drafter gives base logits U_k
+for every position k of a block in one pass; the head adds
+B(x_{k-1}, :) = W2(W1[x_{k-1}]) with W1 an embedding [V, r] and W2 a
+bias-free Linear(r, V) (weight [V, r]). Training uses the teacher-forced
+predecessor (``apply_block_logits``); inference samples left to right
+(``sample_block_tokens``).
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional, Tuple
+
+import torch
+
+from . import _native as N
+
+_DT = {torch.float32: N.DSPARK_DTYPE_FP32, torch.bfloat16: N.DSPARK_DTYPE_BF16}
+
+
+def _stream_ptr(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check_cuda(t: torch.Tensor, name: str, device: torch.device) -> None:
+    if not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must be a CUDA tensor on {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+class VanillaMarkov:
+    """Memoryless low-rank transition bias with caller-owned weights.
+
+    ``w1`` (embedding table) and ``w2`` (``Linear(rank, vocab)`` weight) are
+    both ``[vocab, rank]`` CUDA tensors of one dtype (fp32 or bf16). The head
+    requires ``rank > 0`` (``VanillaMarkov.__init__`` asserts it).
+    """
+
+    markov_head_type = "vanilla"
+
+    def __init__(self, w1: torch.Tensor, w2: torch.Tensor):
+        if w1.dim() != 2 or w1.shape != w2.shape:
+            raise ValueError("w1 and w2 must both be [vocab, rank]")
+        if w1.dtype not in _DT or w2.dtype not in _DT:
+            raise ValueError("weights must be float32 or bfloat16")
+        if w1.dtype != w2.dtype:
+            raise ValueError("w1 and w2 must share a dtype")
+        self.vocab_size, self.markov_rank = int(w1.shape[0]), int(w1.shape[1])
+        if self.markov_rank <= 0:
+            raise ValueError(f"VanillaMarkov requires markov_rank > 0, got {self.markov_rank}")
+        _check_cuda(w1, "w1", w1.device)
+        _check_cuda(w2, "w2", w1.device)
+        self.device = w1.device
+        self.markov_w1 = w1
+        self.markov_w2 = w2
+        self._lib = N.load()
+
+    @property
+    def weight_dtype(self) -> torch.dtype:
+        return self.markov_w1.dtype
+
+    # ------------------------------------------------------------------ apply
+    def apply_block_logits(self, base_logits: torch.Tensor, *, token_ids: torch.Tensor,
+                           hidden_states: Optional[torch.Tensor] = None,
+                           out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Teacher-forced corrected logits, shape-agnostic over leading dims:
+        ``base_logits`` (..., M, V), ``token_ids`` (..., M). Returns
+        ``base_logits`` itself when it is empty or M == 0. ``hidden_states``
+        is accepted and ignored (the vanilla head is a function of the
+        previous token only). ``out`` may be ``base_logits`` (in place)."""
+        del hidden_states
+        if base_logits.numel() == 0 or base_logits.shape[-2] == 0:
+            return base_logits
+        vocab = base_logits.shape[-1]
+        if vocab != self.vocab_size:
+            raise ValueError(f"vocab mismatch: logits {vocab} vs head {self.vocab_size}")
+        if tuple(token_ids.shape) != tuple(base_logits.shape[:-1]):
+            raise ValueError("token_ids must match base_logits without its last dim")
+        if base_logits.dtype not in _DT:
+            raise ValueError("logits must be float32 or bfloat16")
+        _check_cuda(base_logits, "base_logits", self.device)
+        ids = token_ids if token_ids.dtype == torch.int64 else token_ids.long()
+        ids = ids.contiguous()
+        _check_cuda(ids, "token_ids", self.device)
+        if out is None:
+            out = torch.empty_like(base_logits)
+        else:
+            if out.shape != base_logits.shape or out.dtype != base_logits.dtype:
+                raise ValueError("out must match base_logits in shape and dtype")
+            _check_cuda(out, "out", self.device)
+        rows = base_logits.numel() // vocab
+        code = self._lib.dspark_markov_apply_block_logits(
+            base_logits.data_ptr(), out.data_ptr(), ids.data_ptr(), rows, vocab, self.markov_w1.data_ptr(),
+            self.markov_w2.data_ptr(), self.markov_rank, _DT[base_logits.dtype], _DT[self.weight_dtype],
+            _stream_ptr(self.device))
+        N.check(code, "dspark_markov_apply_block_logits")
+        return out
+
+    def apply_step_logits(self, logits: torch.Tensor, *, token_ids: torch.Tensor,
+                          hidden_states: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """One position (B, V) with its (B,) previous tokens."""
+        return self.apply_block_logits(logits.unsqueeze(-2), token_ids=token_ids.unsqueeze(-1),
+                                       hidden_states=hidden_states).squeeze(-2)
+
+    # ----------------------------------------------------------------- sample
+    def sample_block_tokens(self, base_logits: torch.Tensor, *, first_prev_token_ids: torch.Tensor,
+                            hidden_states: Optional[torch.Tensor] = None, temperature: Optional[float] = 0.0,
+                            seed: int = 0, out_tokens: Optional[torch.Tensor] = None,
+                            out_logits: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+        """Left-to-right sampling of ``base_logits`` (B, M, V). Returns
+        (sampled_tokens (B, M) int64, corrected_logits (B, M, V)). With M == 0
+        returns an empty (B, 0) token tensor and ``base_logits`` itself.
+        ``temperature`` None or below 1e-5 is greedy; otherwise each token is
+        a Gumbel-max draw from softmax(c / T) with Philox noise keyed by
+        ``seed``. ``hidden_states`` is accepted and ignored."""
+        del hidden_states
+        if base_logits.dim() != 3:
+            raise ValueError("base_logits must be (B, M, V)")
+        batch, m, vocab = base_logits.shape
+        if m == 0:
+            return torch.empty(batch, 0, dtype=torch.long, device=base_logits.device), base_logits
+        if vocab != self.vocab_size:
+            raise ValueError(f"vocab mismatch: logits {vocab} vs head {self.vocab_size}")
+        if base_logits.dtype not in _DT:
+            raise ValueError("logits must be float32 or bfloat16")
+        _check_cuda(base_logits, "base_logits", self.device)
+        prev = first_prev_token_ids if first_prev_token_ids.dtype == torch.int64 else first_prev_token_ids.long()
+        prev = prev.contiguous()
+        if tuple(prev.shape) != (batch,):
+            raise ValueError("first_prev_token_ids must be (B,)")
+        _check_cuda(prev, "first_prev_token_ids", self.device)
+        t = 0.0 if temperature is None else float(temperature)
+        if math.isnan(t):
+            raise ValueError("temperature is NaN")
+        tokens = out_tokens if out_tokens is not None else torch.empty(batch, m, dtype=torch.long, device=self.device)
+        corrected = out_logits if out_logits is not None else torch.empty_like(base_logits)
+        code = self._lib.dspark_markov_sample_block(
+            base_logits.data_ptr(), prev.data_ptr(), batch, m, vocab, self.markov_w1.data_ptr(),
+            self.markov_w2.data_ptr(), self.markov_rank, t, seed & 0xFFFFFFFFFFFFFFFF, tokens.data_ptr(),
+            corrected.data_ptr(), _DT[base_logits.dtype], _DT[self.weight_dtype], _stream_ptr(self.device))
+        N.check(code, "dspark_markov_sample_block")
+        return tokens, corrected
+
+
+def build_markov_head(w1: Optional[torch.Tensor], w2: Optional[torch.Tensor], markov_rank: int,
+                      head_type: str = "vanilla") -> Optional[VanillaMarkov]:
+    """``build_markov_head``: None when ``markov_rank == 0`` (head disabled);
+    a negative rank is an error; only the vanilla head is built here."""
+    markov_rank = int(markov_rank)
+    if markov_rank < 0:
+        raise ValueError(f"markov_rank must be >= 0, got {markov_rank}")
+    if markov_rank == 0:
+        return None
+    if str(head_type).lower() != "vanilla":
+        raise ValueError(f"Unsupported markov_head_type={head_type!r}; only 'vanilla' is built")
+    return VanillaMarkov(w1, w2)
+
+
+def device_status(device: Optional[torch.device] = None) -> int:
+    """Synchronise the current stream, then read and clear the device status
+    word (DSPARK_STATUS_* bits)."""
+    import ctypes
+    dev = device or torch.device("cuda", torch.cuda.current_device())
+    out = ctypes.c_int32(0)
+    with torch.cuda.device(dev):
+        N.check(N.load().dspark_markov_get_status(_stream_ptr(dev), ctypes.byref(out)), "dspark_markov_get_status")
+    return int(out.value)
+
+
+def set_algo(algo: int) -> int:
+    return int(N.load().dspark_markov_set_algo(int(algo)))
+
+
+def launch_count() -> int:
+    return int(N.load().dspark_markov_launch_count())
+
+
+def last_algo() -> int:
+    return int(N.load().dspark_markov_last_algo())
+
+
+def set_debug(flags: int, wait_limit_ns: int = 0) -> None:
+    N.check(N.load().dspark_markov_set_debug(int(flags), int(wait_limit_ns)), "dspark_markov_set_debug")

@@ -1,0 +1,219 @@
+"""Parity of the CUDA left-to-right sampler against the fp64 oracle (B200).
+
+Tokens are checked with the oracle teacher-forced on the sampled tokens
+(``oracle.checks.check_sampled_block``): exact where the oracle's top-1/top-2
+margin exceeds 1e-2, top-2 otherwise, exact everywhere for fp32.
+"""
+import numpy as np
+import pytest
+import torch
+from scipy import stats
+from scipy.special import softmax
+
+import oracle
+from oracle.checks import check_logits, check_sampled_block
+from rank_markov_draft_vanillamarkov_b200 import VanillaMarkov, device_status, last_algo, set_algo, set_debug
+from rank_markov_draft_vanillamarkov_b200 import _native as N
+from rank_markov_draft_vanillamarkov_b200 import workloads as W
+from rank_markov_draft_vanillamarkov_b200.build import build
+
+from _helpers import f64
+
+pytestmark = pytest.mark.gpu
+
+TC, GEN, AUTO = N.DSPARK_ALGO_TENSOR_CORE, N.DSPARK_ALGO_GENERIC, N.DSPARK_ALGO_AUTO
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build()
+    N.load()
+    yield
+    set_algo(AUTO)
+    set_debug(0, 0)
+
+
+def _sample(d, algo, temperature, seed=0, base=None, first=None):
+    set_algo(algo)
+    head = VanillaMarkov(d["w1"].cuda(), d["w2"].cuda())
+    base = (d["base"] if base is None else base).cuda()
+    first = (d["first_prev"] if first is None else first).cuda()
+    toks, corr = head.sample_block_tokens(base, first_prev_token_ids=first, temperature=temperature, seed=seed)
+    torch.cuda.synchronize()
+    return toks, corr, last_algo(), device_status()
+
+
+def _check(d, toks, corr, temperature, seed, dtype="bf16", rows=None):
+    rep = check_sampled_block(toks.cpu().numpy(), f64(corr), f64(d["base"]), f64(d["w1"]), f64(d["w2"]),
+                              d["first_prev"].numpy(), dtype, temperature, seed, rows=rows)
+    assert rep.logits.ok, (rep.logits.bad, rep.logits.first_bad, rep.logits.max_abs)
+    assert rep.bad == 0, (rep.bad, rep.exact_required, rep.near_ties)
+    return rep
+
+
+def _small(batch, vocab=1000, rank=64, m=5, wstd=0.3, seed=21, spike=6.0):
+    return W.GREEDY.with_(name=f"greedy_small_b{batch}_v{vocab}_k{rank}", batch=batch, vocab=vocab, rank=rank,
+                          proposal_len=m, weight_std=wstd, spike=spike, data_seed=seed)
+
+
+@pytest.mark.parametrize("algo", [TC, GEN], ids=["tc", "generic"])
+@pytest.mark.parametrize("batch,vocab,rank", [(1, 1000, 64), (5, 2056, 128), (33, 1000, 192), (70, 4096, 256)])
+def test_greedy_small(batch, vocab, rank, algo):
+    wl = _small(batch, vocab, rank)
+    d = W.make_inputs(wl)
+    toks, corr, used, st = _sample(d, algo, 0.0)
+    assert used == (2 if algo == TC else 1) and st == 0
+    # invariant: each token is the first argmax of its own corrected row
+    assert torch.equal(toks, corr.float().argmax(-1))
+    _check(d, toks, corr, 0.0, 0)
+
+
+@pytest.mark.parametrize("batch", W.GREEDY_BATCHES)
+def test_greedy_full_size(batch):
+    """M = 5, V = 129280, rank 128, peaked logits, every (b, k)."""
+    wl = W.greedy(batch)
+    d = W.make_inputs(wl)
+    toks, corr, used, st = _sample(d, AUTO, 0.0)
+    assert used == 2 and st == 0
+    assert torch.equal(toks, corr.float().argmax(-1))
+    _check(d, toks, corr, 0.0, 0)
+
+
+def test_greedy_strong_bias_changes_tokens():
+    """Weights ~N(0, 0.3) make the bias decide tokens; the chain must follow
+    its own choices (a teacher-forced or bias-free chain would differ)."""
+    wl = W.greedy(32).with_(weight_std=0.3, spike=0.0, data_seed=3)
+    d = W.make_inputs(wl)
+    toks, corr, used, st = _sample(d, AUTO, 0.0)
+    assert used == 2 and st == 0
+    _check(d, toks, corr, 0.0, 0)
+    unbiased = d["base"].float().argmax(-1)
+    assert (toks.cpu() != unbiased).float().mean() > 0.2
+
+
+def test_temperature_full_size():
+    """B = 32, M = 8, V = 151936, rank 64, T = 0.7, Philox seed 1234."""
+    wl = W.TEMPERATURE
+    d = W.make_inputs(wl)
+    toks, corr, used, st = _sample(d, AUTO, wl.temperature, seed=wl.philox_seed)
+    assert used == 2 and st == 0
+    rep = _check(d, toks, corr, wl.temperature, wl.philox_seed)
+    assert rep.exact_required > 0.9 * wl.batch * wl.proposal_len
+
+
+@pytest.mark.parametrize("algo", [TC, GEN], ids=["tc", "generic"])
+def test_temperature_small(algo):
+    wl = _small(40, 2056, 128, m=6, wstd=0.3).with_(temperature=1.3)
+    d = W.make_inputs(wl)
+    toks, corr, used, st = _sample(d, algo, 1.3, seed=99)
+    assert st == 0
+    _check(d, toks, corr, 1.3, 99)
+
+
+def test_tiny_fp32_greedy_exact():
+    wl = W.TINY_FP32
+    g = torch.Generator().manual_seed(0)
+    w1, w2 = W.make_weights(wl, g)
+    base = (torch.randn(2, 5, wl.vocab, generator=g) * wl.logit_std).float()
+    d = {"w1": w1, "w2": w2, "base": base, "first_prev": W.uniform_ids(g, 2, wl.vocab)}
+    toks, corr, used, st = _sample(d, AUTO, 0.0)
+    assert used == 1 and st == 0
+    _check(d, toks, corr, 0.0, 0, dtype="fp32")
+    t_or, _ = oracle.sample_block_tokens(f64(base), f64(w1), f64(w2), d["first_prev"].numpy(), "fp32", 0.0)
+    np.testing.assert_array_equal(toks.cpu().numpy(), t_or)
+
+
+@pytest.mark.parametrize("temperature", [0.0, 0.9])
+def test_sample_matches_apply_on_its_own_tokens(temperature):
+    """The sampler's corrected logits equal the teacher-forced apply computed
+    with prev = [first_prev, tok_0, ..., tok_{M-2}] (both tensor-core paths)."""
+    wl = W.greedy(16).with_(weight_std=0.3, data_seed=8)
+    d = W.make_inputs(wl)
+    toks, corr, used, _ = _sample(d, TC, temperature, seed=5)
+    prev = torch.cat([d["first_prev"].cuda()[:, None], toks[:, :-1]], dim=1)
+    head = VanillaMarkov(d["w1"].cuda(), d["w2"].cuda())
+    ref = head.apply_block_logits(d["base"].cuda(), token_ids=prev)
+    diff = (ref.float() - corr.float()).abs()
+    ulp = torch.from_numpy(oracle.ulp_bfloat16(f64(ref))).cuda().view_as(diff).float()
+    assert (diff <= ulp).all()
+
+
+def test_gpu_sampling_follows_softmax():
+    """V = 64, M = 1, 128 identical rows per call, 128 seeds: counts must fit
+    softmax(c / T) by chi-square."""
+    v, rows, temp = 64, 128, 0.8
+    rng = np.random.default_rng(4)
+    logits = torch.from_numpy(rng.standard_normal(v) * 1.2).to(torch.bfloat16)
+    base = logits.view(1, 1, v).expand(rows, 1, v).contiguous()
+    d = {"w1": torch.zeros(v, 64, dtype=torch.bfloat16), "w2": torch.zeros(v, 64, dtype=torch.bfloat16),
+         "base": base, "first_prev": torch.zeros(rows, dtype=torch.long)}
+    counts = np.zeros(v)
+    for seed in range(128):
+        toks, _, used, st = _sample(d, TC, temp, seed=seed)
+        assert used == 2 and st == 0
+        counts += np.bincount(toks.cpu().numpy()[:, 0], minlength=v)
+    p = softmax(f64(logits) / temp)
+    keep = p * counts.sum() >= 5
+    obs = np.append(counts[keep], counts[~keep].sum())
+    exp = np.append(p[keep], p[~keep].sum()) * counts.sum()
+    assert stats.chisquare(obs, exp).pvalue > 1e-3
+
+
+def test_philox_draws_match_the_oracle_bit_for_bit():
+    """Zero weights and all-equal logits: the token is the argmax of the
+    Gumbel noise alone, so the GPU's Philox must reproduce the oracle's draw."""
+    v, rows = 512, 64
+    base = torch.zeros(rows, 3, v, dtype=torch.bfloat16)
+    d = {"w1": torch.zeros(v, 64, dtype=torch.bfloat16), "w2": torch.zeros(v, 64, dtype=torch.bfloat16),
+         "base": base, "first_prev": torch.zeros(rows, dtype=torch.long)}
+    seed = (3 << 32) | 12345
+    toks, _, _, st = _sample(d, TC, 1.0, seed=seed)
+    want = np.array([[int(np.argmax(oracle.gumbel_noise(seed, b, k, v))) for k in range(3)] for b in range(rows)])
+    np.testing.assert_array_equal(toks.cpu().numpy(), want)
+    toks_g, _, _, _ = _sample(d, GEN, 1.0, seed=seed)
+    np.testing.assert_array_equal(toks_g.cpu().numpy(), want)
+
+
+def test_same_seed_same_draws_other_seed_differs():
+    wl = _small(16, 2056, 64, wstd=0.05, spike=0.0)
+    d = W.make_inputs(wl)
+    a, ca, _, _ = _sample(d, TC, 1.0, seed=7)
+    b, cb, _, _ = _sample(d, TC, 1.0, seed=7)
+    c, _, _, _ = _sample(d, TC, 1.0, seed=8)
+    assert torch.equal(a, b) and torch.equal(ca, cb)
+    assert not torch.equal(a, c)
+
+
+def test_zero_length_block():
+    d = W.make_inputs(_small(4))
+    head = VanillaMarkov(d["w1"].cuda(), d["w2"].cuda())
+    e = torch.zeros(4, 0, 1000, dtype=torch.bfloat16, device="cuda")
+    toks, corr = head.sample_block_tokens(e, first_prev_token_ids=torch.zeros(4, dtype=torch.long, device="cuda"))
+    assert corr is e and toks.shape == (4, 0) and toks.dtype == torch.long
+
+
+@pytest.mark.parametrize("algo", [TC, GEN], ids=["tc", "generic"])
+def test_out_of_range_first_prev_reports_status(algo):
+    d = W.make_inputs(_small(8))
+    first = d["first_prev"].clone()
+    first[2] = 10 ** 9
+    _, _, _, st = _sample(d, algo, 0.0, first=first)
+    assert st & N.DSPARK_STATUS_TOKEN_RANGE
+
+
+def test_barrier_timeout_is_reported_not_hung():
+    """One CTA withholds its grid-barrier arrival (a host-set test flag):
+    the other CTAs' bounded waits run out after 20 ms, the TIMEOUT bit is
+    set, the kernel returns, and the next call is correct again."""
+    wl = W.greedy(8)
+    d = W.make_inputs(wl)
+    set_debug(N.DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL, 20_000_000)
+    try:
+        _, _, used, st = _sample(d, TC, 0.0)
+    finally:
+        set_debug(0, 0)
+    assert used == 2
+    assert st & N.DSPARK_STATUS_TIMEOUT
+    toks, corr, used, st = _sample(d, TC, 0.0)
+    assert st == 0
+    _check(d, toks, corr, 0.0, 0)
