@@ -23,4 +23,4 @@ from .markov import (  # noqa: F401
 )
 from .philox import gumbel_noise, noise_words, philox4x32, uniform_from_word  # noqa: F401
 from .rounding import round_to, round_to_bfloat16, round_to_float32, ulp_bfloat16  # noqa: F401
-from .checks import check_logits, check_sampled_block, check_tokens  # noqa: F401
+from .checks import accumulation_bound, check_logits, check_sampled_block, check_tokens  # noqa: F401

@@ -19,7 +19,7 @@
 //   - merges its maxima into a per-(k, b) 64-bit key with atomicMax, then
 //     passes a grid barrier (bounded wait) after which every CTA decodes x_k.
 //
-// Warp roles (288 threads): 0 W2 producer, 1 MMA issuer + TMEM owner, 2 U
+// Warp roles (256 threads): 0 W2 producer, 1 MMA issuer + TMEM owner, 2 U
 // producer, 3 W1 gather + grid barrier, 4-7 epilogue (thread = vocab id).
 #include "common.cuh"
 #include "kernels.h"
@@ -31,7 +31,7 @@ namespace {
 constexpr int kBV = 128;               // vocabulary ids per tile (MMA M)
 constexpr int kAtomK = 64;             // bf16 elements per 128-byte swizzle row
 constexpr int kW2AtomBytes = 128 * 128;
-constexpr int kThreads = 288;
+constexpr int kThreads = 256;  // 8 warps: one per role below, four for the epilogue
 constexpr int kMaxStages = 12;
 constexpr int kMaxBatch = 256;
 constexpr size_t kSmemLimit = 232448;  // dynamic shared memory per block on sm_100
@@ -65,7 +65,7 @@ struct SampleParams {
 struct SampleTail {
   uint64_t w2_full[kMaxStages], w2_empty[kMaxStages];
   uint64_t u_full[kMaxStages], u_empty[kMaxStages];
-  uint64_t x_full[2], x_empty[2];
+  uint64_t x_full, x_empty;
   uint64_t acc_full[2], acc_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
@@ -130,8 +130,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* w2_smem = smem;                                            // w2_slots x KA atoms
-  uint8_t* x_smem = w2_smem + (size_t)p.w2_slots * KA * kW2AtomBytes;  // 2 x x_bytes
-  uint8_t* u_smem = x_smem + 2 * (size_t)p.x_bytes;                   // u_slots x u_slot_bytes
+  uint8_t* x_smem = w2_smem + (size_t)p.w2_slots * KA * kW2AtomBytes;  // one step's X
+  uint8_t* u_smem = x_smem + (size_t)p.x_bytes;                       // u_slots x u_slot_bytes
   unsigned long long* red = reinterpret_cast<unsigned long long*>(u_smem + (size_t)p.u_slots * p.u_slot_bytes);
   SampleTail* sh = reinterpret_cast<SampleTail*>(red + 4 * p.batch_pad);
 
@@ -156,9 +156,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sh->u_full[i], 1);
       mbar_init(&sh->u_empty[i], 1);
     }
+    mbar_init(&sh->x_full, 32);
+    mbar_init(&sh->x_empty, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&sh->x_full[i], 32);
-      mbar_init(&sh->x_empty[i], 1);
       mbar_init(&sh->acc_full[i], 1);
       mbar_init(&sh->acc_empty[i], 4);
     }
@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int t = t_begin + (int)(i % nt);
         const int s = (int)(i % p.u_slots);
         if (!mbar_wait(&sh->u_empty[s], ((uint32_t)(i / p.u_slots) & 1u) ^ 1u, ctl)) break;
-        mbar_arrive_expect_tx(&sh->u_full[s], p.u_slot_bytes);
+        mbar_arrive_expect_tx(&sh->u_full[s], (uint32_t)B * kBV * 2u);  // the box, not the padded slot
         tma_load_3d(u_smem + (size_t)s * p.u_slot_bytes, &maps.u, &sh->u_full[s], t * kBV, k, 0, pol_stream);
       }
       for (int64_t j = (i > p.u_slots ? i - p.u_slots : 0); j < i; ++j)
@@ -219,15 +219,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 3) {
     // ------------------------------------ W1 gather + grid barrier ----
+    // One X buffer suffices: step k+1's rows are gathered only after the grid
+    // barrier, i.e. after every MMA of step k has completed.
     for (int k = 0; k < M; ++k) {
-      const int xb = k & 1;
-      const uint32_t xe_par = ((uint32_t)(k >> 1) & 1u) ^ 1u;
+      const uint32_t xe_par = ((uint32_t)k & 1u) ^ 1u;
       // Lane 0 decides and the warp follows, so the lanes never split around
       // the warp-wide shuffles below.
-      bool xe_ok = lane == 0 ? mbar_wait(&sh->x_empty[xb], xe_par, ctl) : true;
+      bool xe_ok = lane == 0 ? mbar_wait(&sh->x_empty, xe_par, ctl) : true;
       xe_ok = __shfl_sync(0xffffffffu, xe_ok ? 1 : 0, 0) != 0;
       if (!xe_ok) break;
-      if (lane != 0) mbar_wait(&sh->x_empty[xb], xe_par, ctl);  // already complete
+      if (lane != 0) mbar_wait(&sh->x_empty, xe_par, ctl);  // already complete
       if (k > 0) {
         // Every CTA has merged its step k-1 maxima once the counter reaches k * G.
         bool ok = true;
@@ -252,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (!ok) break;
       }
-      uint8_t* xdst = x_smem + (size_t)xb * p.x_bytes;
+      uint8_t* xdst = x_smem;
       bool bad = false;
       for (int b0 = 0; b0 < BB; b0 += 32) {
         int64_t id = -1;
@@ -281,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (bad) report_status(p.status, DSPARK_STATUS_TOKEN_RANGE);
       fence_proxy_async_smem();
-      mbar_arrive(&sh->x_full[xb]);
+      mbar_arrive(&sh->x_full);
     }
   } else if (warp == 1) {
     // ------------------------------------------------- MMA issuer ----
@@ -291,8 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t x_addr = smem_u32(x_smem);
       bool ok = true;
       for (int k = 0; k < M && ok; ++k) {
-        const int xb = k & 1;
-        if (!mbar_wait(&sh->x_full[xb], (uint32_t)(k >> 1) & 1u, ctl)) break;
+        if (!mbar_wait(&sh->x_full, (uint32_t)k & 1u, ctl)) break;
         for (int tt = 0; tt < nt; ++tt) {
           const int64_t i = (int64_t)k * nt + tt;
           const int w = (int)(i % p.w2_slots);
@@ -309,14 +309,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < kAtomK / 16; ++kk) {
               const uint64_t ad = sw128_kmajor_desc(w2_addr + (uint32_t)(w * KA + ka) * kW2AtomBytes + kk * 32);
-              const uint64_t bd = sw128_kmajor_desc(x_addr + (uint32_t)xb * p.x_bytes + ka * atom_x + kk * 32);
+              const uint64_t bd = sw128_kmajor_desc(x_addr + ka * atom_x + kk * 32);
               umma_bf16_ss(d_tmem, ad, bd, idesc, (ka | kk) != 0);
             }
           }
           umma_commit(&sh->w2_empty[w]);
           umma_commit(&sh->acc_full[abuf]);
         }
-        if (ok) umma_commit(&sh->x_empty[xb]);
+        if (ok) umma_commit(&sh->x_empty);
       }
       umma_commit(&sh->drain);
       mbar_wait(&sh->drain, 0, drain_ctl);
@@ -396,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Merge the four warps' maxima, then this CTA's into the global keys.
 #pragma unroll
       for (int g = 0; g < kMaxBatch / 32; ++g)
-        if (g < groups) red[q * BB + 32 * g + lane] = best[g];
+        if (g < groups && 32 * g + lane < BB) red[q * BB + 32 * g + lane] = best[g];  // BB may be 16
       named_barrier_sync(1, 128);
       for (int b = et; b < B; b += 128) {
         const unsigned long long m = umax64(umax64(red[b], red[BB + b]), umax64(red[2 * BB + b], red[3 * BB + b]));
@@ -445,9 +445,9 @@ SampleConfig plan(int ka, int batch, int batch_pad) {
   SampleConfig c{};
   c.u_slot_bytes = (uint32_t)align1024((size_t)batch * kBV * 2);
   c.x_bytes = (uint32_t)((size_t)ka * batch_pad * 128);
-  const size_t fixed = 1024 + 2 * (size_t)c.x_bytes + 4 * (size_t)batch_pad * 8 + sizeof(SampleTail) + 64;
+  const size_t fixed = 1024 + (size_t)c.x_bytes + 4 * (size_t)batch_pad * 8 + sizeof(SampleTail) + 64;
   const size_t w2_slot = (size_t)ka * kW2AtomBytes;
-  for (int w = 4; w >= 2; --w) {
+  for (int w = 4; w >= 1; --w) {
     for (int u = 8; u >= 2; --u) {
       const size_t total = fixed + w * w2_slot + u * (size_t)c.u_slot_bytes;
       if (total <= kSmemLimit) {
