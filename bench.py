@@ -375,6 +375,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=[n for n, _ in PARTS + EXTRA], default=None,
+                    help="time a single part (for profiling); implies --no-e2e and --no-cpu-baseline")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extra", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -400,8 +404,20 @@ def main():
         torch.distributed.barrier()
     N.load()
 
+    if args.only:
+        wl = dict(PARTS + EXTRA)[args.only]
+        p = Part(args.only, wl, device, seed_offset=1000 * rank)
+        region, per = time_region([p], args.steps, args.warmup, world)
+        if rank == 0:
+            print(json.dumps({"only": args.only, "workload": wl.name, "us": per[args.only] * 1e6,
+                              "gbps": wl.bytes_moved() / per[args.only] / 1e9, "steps": args.steps}), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return 0
+
     parts = [Part(name, wl, device, seed_offset=1000 * rank) for name, wl in PARTS]
-    extra = [Part(name, wl, device, seed_offset=1000 * rank, min_bytes=2 * L2_BYTES) for name, wl in EXTRA]
+    extra = [] if args.no_extra else \
+        [Part(name, wl, device, seed_offset=1000 * rank, min_bytes=2 * L2_BYTES) for name, wl in EXTRA]
 
     clocks = ClockSampler(local)
     clocks.start()
@@ -409,9 +425,13 @@ def main():
     region, per = time_region(parts, args.steps, args.warmup, world)
     launches = launch_count() - n0
     clk = clocks.stop()
-    extra_region, extra_per = time_region(extra, max(20, args.steps // 20), 3, world)
+    extra_per = time_region(extra, max(20, args.steps // 20), 3, world)[1] if extra else {}
 
-    e2e_sec, h2d, d2h = time_e2e(parts, args.e2e_steps, world)
+    e2e = None
+    if not args.no_e2e:
+        e2e_sec, h2d, d2h = time_e2e(parts, args.e2e_steps, world)
+        e2e = {"value": sum(p.rows for p in parts) * world * args.e2e_steps / e2e_sec, "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
 
     rows_step = sum(p.rows for p in parts)
     value = rows_step * world * args.steps / region
@@ -441,8 +461,7 @@ def main():
                      "traffic": profile_traffic(tag), "algorithmic_bytes": dom.wl.bytes_moved()},
         "gpu_launches": launches,
         "clocks": clk,
-        "e2e": {"value": rows_step * world * args.e2e_steps / e2e_sec, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps},
+        "e2e": e2e,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         inputs = [W.make_inputs(wl) for _, wl in PARTS]

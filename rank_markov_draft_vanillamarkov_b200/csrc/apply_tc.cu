@@ -3,23 +3,31 @@
 //
 //     out[i, v] = round_bf16( U[i, v] + sum_j W1[prev_i, j] * W2[v, j] )
 //
-// One persistent CTA per SM walks a contiguous run of 128 x 128 output tiles,
-// ordered vocab-tile major (all row tiles of one vocab tile, then the next), so
-// the W2 tile [128 ids x rank] is loaded once per vocab tile and stays in
-// shared memory while the CTA walks the row tiles.
+// One persistent CTA per SM walks a contiguous run of 128-row x 128-id output
+// tiles ("units"), vocab-tile major: all row tiles of one vocab tile, then the
+// next. The W2 tile [128 ids x rank] is loaded by TMA once per vocab tile and
+// stays in shared memory while the CTA walks that tile's rows.
 //
-// Warp roles (256 threads):
-//   warp 0      TMA producer: W2 tiles and U tiles (two 64-column boxes of
-//               128 rows, 128-byte swizzle) into a ring of stages.
-//   warp 1      owns tensor memory; lane 0 issues tcgen05.mma
-//               (M = 128 rows, N = 128 ids, K = 16 per instruction) into one
-//               of two TMEM accumulators.
-//   warps 2-3   gather W1[prev] rows (the A operand) into shared memory in the
-//               128-byte swizzle layout. When all row tiles fit, they are
-//               gathered once and stay resident.
-//   warps 4-7   epilogue: tcgen05.ld the fp32 accumulator (thread = row),
-//               add the U tile in place in shared memory, round to bf16, and
-//               TMA-store the tile to `out`.
+// The gathered rows W1[prev] (the MMA's A operand, [128 rows x rank]) live in
+// tensor memory, loaded with tcgen05.st by four gather warps: resident for
+// the whole launch when every row tile fits (at rank 128 up to 512 rows),
+// otherwise double-buffered per unit. Shared memory then holds only W2 and a
+// deep ring of U tiles, which is what keeps enough HBM reads in flight.
+//
+// Warp roles (512 threads):
+//   warp 0       TMA producer: W2 tiles and U tiles (two 64-id boxes of 128
+//                rows each, 128-byte swizzle) into rings.
+//   warp 1       owns tensor memory (512 columns); lane 0 issues
+//                tcgen05.mma.kind::f16 with A in TMEM and B = the W2 tile in
+//                shared memory (M = 128, N = 128, K = 16 per instruction).
+//   warps 4-7    gather W1[prev] rows into TMEM (warp w owns lanes 32*(w%4)).
+//   warps 8-11   epilogue group 0 (even units, accumulator 0);
+//   warps 12-15  epilogue group 1 (odd units, accumulator 1): tcgen05.ld of
+//                the fp32 accumulator (thread = row), add the U tile in place
+//                in shared memory, round to bf16, TMA-store the tile.
+//
+// Tensor memory: columns [0,128) and [128,256) are the two accumulators,
+// [256,512) holds A (rank/2 columns per 128-row tile; two bf16 per column).
 //
 // Every wait is bounded (WaitCtl); a wait that runs out sets the TIMEOUT bit
 // of the status word and the CTA winds down without faulting.
@@ -30,15 +38,17 @@
 namespace dspark {
 namespace {
 
-constexpr int kBM = 128;              // rows per tile (MMA M)
-constexpr int kBN = 128;              // vocabulary ids per tile (MMA N)
+constexpr int kBM = 128;              // rows per unit (MMA M)
+constexpr int kBN = 128;              // vocabulary ids per unit (MMA N)
 constexpr int kAtomK = 64;            // bf16 elements in one 128-byte swizzle row
-constexpr int kAtomBytes = 128 * 128; // one 128-row x 64-element operand atom
+constexpr int kAtomBytes = 128 * 128; // one 128-row x 64-element W2 atom / one U box
 constexpr int kUStageBytes = 2 * kAtomBytes;  // 128 rows x 128 ids of bf16
-constexpr int kThreads = 256;
-constexpr int kSlotBudget = 14;       // 16 KB slots that fit next to the barriers
-constexpr int kTmemCols = 2 * kBN;    // two accumulators
-constexpr int kMaxStages = 16;
+constexpr int kThreads = 512;
+constexpr int kTmemCols = 512;
+constexpr int kAccCols = 2 * kBN;     // accumulators occupy [0, 256)
+constexpr int kMaxStages = 8;
+constexpr int kMaxResidentTiles = 8;
+constexpr size_t kSmemLimit = 232448;
 
 struct __align__(64) ApplyMaps {
   CUtensorMap u;    // [rows, vocab] bf16, box 64 x 128, 128B swizzle
@@ -52,17 +62,18 @@ struct ApplyParams {
   int64_t rows, vocab;
   int32_t rank;
   int32_t row_tiles, vocab_tiles;
-  int32_t a_slots, u_stages;
-  int32_t resident;  // all row tiles of A stay in shared memory
+  int32_t w2_slots, u_stages;
+  int32_t resident;  // all row tiles of A stay in tensor memory
   uint32_t* status;
   uint64_t wait_limit_ns;
 };
 
 struct SharedTail {
-  uint64_t w2_full, w2_empty, drain;
-  uint64_t a_full[kMaxStages], a_empty[kMaxStages];
+  uint64_t w2_full[2], w2_empty[2];
+  uint64_t a_full[kMaxResidentTiles], a_empty[2];
   uint64_t u_full[kMaxStages], u_empty[kMaxStages];
   uint64_t acc_full[2], acc_empty[2];
+  uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -79,9 +90,7 @@ __device__ __forceinline__ bool barrier_and(bool v, uint32_t id, uint32_t n) {
 
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
   return r;
 }
 
@@ -92,16 +101,56 @@ __device__ __forceinline__ uint32_t add_round_pair(uint32_t u2, uint32_t acc_lo,
   return *reinterpret_cast<uint32_t*>(&o);
 }
 
+// A warp-uniform bounded wait: lane 0 waits, the warp follows its verdict, and
+// the other lanes then observe the (already completed) phase themselves.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl, int lane) {
+  bool ok = lane == 0 ? mbar_wait(bar, parity, ctl) : true;
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  if (ok && lane != 0) mbar_wait(bar, parity, ctl);
+  return ok;
+}
+
+// One 128-row tile of A into tensor memory: thread `row` loads W1[prev] (rank
+// bf16 = rank/2 32-bit words) and stores it to its own TMEM lane, columns
+// [col, col + rank/2), eight words per 16-byte load.
+template <int KA>
+__device__ __forceinline__ void gather_tile_to_tmem(const ApplyParams& p, int m, int row, uint32_t taddr) {
+  const int64_t grow = (int64_t)m * kBM + row;
+  int64_t id = -1;
+  if (grow < p.rows) {
+    id = p.ids[grow];
+    if (id < 0 || id >= p.vocab) {
+      report_status(p.status, DSPARK_STATUS_TOKEN_RANGE);
+      id = -1;
+    }
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(p.w1 + (id < 0 ? 0 : id) * p.rank);
+#pragma unroll
+  for (int c = 0; c < KA; ++c) {  // 64 bf16 = 32 words = 8 loads per chunk
+    uint32_t w[32];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint4 x = id >= 0 ? ld_nc_v4(src + c * 8 + i) : make_uint4(0u, 0u, 0u, 0u);
+      w[4 * i + 0] = x.x;
+      w[4 * i + 1] = x.y;
+      w[4 * i + 2] = x.z;
+      w[4 * i + 3] = x.w;
+    }
+    tmem_st_32x32b_x32(taddr + c * 32, w);
+  }
+  tmem_st_wait();
+}
+
 template <int KA>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_apply_kernel(const __grid_constant__ ApplyMaps maps, const ApplyParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* w2_smem = smem;
-  uint8_t* a_smem = w2_smem + KA * kAtomBytes;
-  uint8_t* u_smem = a_smem + p.a_slots * kAtomBytes;
-  SharedTail* sh = reinterpret_cast<SharedTail*>(u_smem + p.u_stages * kUStageBytes);
+  uint8_t* w2_smem = smem;                                     // w2_slots x KA atoms
+  uint8_t* u_smem = w2_smem + (size_t)p.w2_slots * KA * kAtomBytes;  // u_stages x 32 KB
+  SharedTail* sh = reinterpret_cast<SharedTail*>(u_smem + (size_t)p.u_stages * kUStageBytes);
 
+  constexpr int kACols = KA * 32;  // TMEM columns of one A tile
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t units = (int64_t)p.row_tiles * p.vocab_tiles;
@@ -110,21 +159,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int MT = p.row_tiles;
 
   if (threadIdx.x == 0) {
-    mbar_init(&sh->w2_full, 1);
-    mbar_init(&sh->w2_empty, 1);
-    mbar_init(&sh->drain, 1);
-    for (int i = 0; i < p.a_slots; ++i) {
-      mbar_init(&sh->a_full[i], 64);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh->w2_full[i], 1);
+      mbar_init(&sh->w2_empty[i], 1);
       mbar_init(&sh->a_empty[i], 1);
+      mbar_init(&sh->acc_full[i], 1);
+      mbar_init(&sh->acc_empty[i], 4);
     }
+    for (int i = 0; i < kMaxResidentTiles; ++i) mbar_init(&sh->a_full[i], 128);
     for (int i = 0; i < p.u_stages; ++i) {
       mbar_init(&sh->u_full[i], 1);
       mbar_init(&sh->u_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sh->acc_full[i], 1);
-      mbar_init(&sh->acc_empty[i], 4);
-    }
+    mbar_init(&sh->drain, 1);
     sh->abort_flag = 0;
     fence_barrier_init();
   }
@@ -137,6 +184,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem_base = sh->tmem_base;
   const WaitCtl ctl{&sh->abort_flag, p.status, p.wait_limit_ns};
+  volatile int never = 0;
+  const WaitCtl drain_ctl{&never, p.status, p.wait_limit_ns};
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer ----
@@ -153,6 +202,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       int64_t it = 0;
       for (int64_t u = u_begin; u < u_end; ++u, ++it) {
         const int32_t n = (int32_t)(u / MT), m = (int32_t)(u % MT);
+        if (n != cur_n) {
+          const int ws = (int)(w2_loads % p.w2_slots);
+          if (!mbar_wait(&sh->w2_empty[ws], ((w2_loads / p.w2_slots) & 1u) ^ 1u, ctl)) break;
+          mbar_arrive_expect_tx(&sh->w2_full[ws], KA * kAtomBytes);
+#pragma unroll
+          for (int ka = 0; ka < KA; ++ka)
+            tma_load_2d(w2_smem + (ws * KA + ka) * kAtomBytes, &maps.w2, &sh->w2_full[ws], ka * kAtomK, n * kBN,
+                        pol_keep);
+          ++w2_loads;
+          cur_n = n;
+        }
         const int s = (int)(it % p.u_stages);
         if (!mbar_wait(&sh->u_empty[s], ((uint32_t)(it / p.u_stages) & 1u) ^ 1u, ctl)) break;
         mbar_arrive_expect_tx(&sh->u_full[s], kUStageBytes);
@@ -160,189 +220,127 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(st, &maps.u, &sh->u_full[s], n * kBN, m * kBM, pol_stream);
         tma_load_2d(st + kAtomBytes, &maps.u, &sh->u_full[s], n * kBN + 64, m * kBM, pol_stream);
         ++fills[s];
-        if (n != cur_n) {
-          if (w2_loads > 0 && !mbar_wait(&sh->w2_empty, (w2_loads - 1) & 1u, ctl)) break;
-          mbar_arrive_expect_tx(&sh->w2_full, KA * kAtomBytes);
-#pragma unroll
-          for (int ka = 0; ka < KA; ++ka)
-            tma_load_2d(w2_smem + ka * kAtomBytes, &maps.w2, &sh->w2_full, ka * kAtomK, n * kBN, pol_keep);
-          ++w2_loads;
-          cur_n = n;
-        }
       }
       // Wait (bounded, even after an abort) for every copy this thread
       // started before the CTA may exit.
-      volatile int never = 0;
-      const WaitCtl drain_ctl{&never, p.status, p.wait_limit_ns};
       for (int s = 0; s < p.u_stages; ++s)
         if (fills[s]) mbar_wait(&sh->u_full[s], (fills[s] - 1) & 1u, drain_ctl);
-      if (w2_loads) mbar_wait(&sh->w2_full, (w2_loads - 1) & 1u, drain_ctl);
+      for (uint32_t j = (w2_loads > (uint32_t)p.w2_slots ? w2_loads - p.w2_slots : 0); j < w2_loads; ++j)
+        mbar_wait(&sh->w2_full[j % p.w2_slots], (j / p.w2_slots) & 1u, drain_ctl);
     }
   } else if (warp == 1) {
     // ------------------------------------------------- MMA issuer -----
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(kBM, kBN);
       const uint32_t w2_addr = smem_u32(w2_smem);
-      const uint32_t a_addr = smem_u32(a_smem);
       int64_t cur_n = -1;
-      uint32_t w2_waits = 0;
-      int64_t a_it = 0;
+      uint32_t w2_uses = 0;
+      int ws = 0;
       int64_t it = 0;
-      bool ok = true;
-      for (int64_t u = u_begin; u < u_end && ok; ++u, ++it) {
+      for (int64_t u = u_begin; u < u_end; ++u, ++it) {
         const int32_t n = (int32_t)(u / MT), m = (int32_t)(u % MT);
         if (n != cur_n) {
-          if (!mbar_wait(&sh->w2_full, w2_waits & 1u, ctl)) break;
-          ++w2_waits;
+          ws = (int)(w2_uses % p.w2_slots);
+          if (!mbar_wait(&sh->w2_full[ws], (w2_uses / p.w2_slots) & 1u, ctl)) break;
+          ++w2_uses;
           cur_n = n;
         }
         const int abuf = (int)(it & 1);
         if (!mbar_wait(&sh->acc_empty[abuf], ((uint32_t)(it >> 1) & 1u) ^ 1u, ctl)) break;
+        const int aslot = p.resident ? m : (int)(it & 1);
+        const uint32_t apar = p.resident ? 0u : (uint32_t)(it >> 1) & 1u;
+        if (!mbar_wait(&sh->a_full[aslot], apar, ctl)) break;
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + (uint32_t)(abuf * kBN);
+        const uint32_t a_tmem = tmem_base + (uint32_t)(kAccCols + aslot * kACols);
 #pragma unroll
-        for (int ka = 0; ka < KA; ++ka) {
-          int slot;
-          uint32_t parity;
-          if (p.resident) {
-            slot = m * KA + ka;
-            parity = 0;
-          } else {
-            slot = (int)(a_it % p.a_slots);
-            parity = (uint32_t)(a_it / p.a_slots) & 1u;
-          }
-          if (!mbar_wait(&sh->a_full[slot], parity, ctl)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after_sync();
-#pragma unroll
-          for (int kk = 0; kk < kAtomK / 16; ++kk) {
-            const uint64_t ad = sw128_kmajor_desc(a_addr + slot * kAtomBytes + kk * 32);
-            const uint64_t bd = sw128_kmajor_desc(w2_addr + ka * kAtomBytes + kk * 32);
-            umma_bf16_ss(d_tmem, ad, bd, idesc, (ka | kk) != 0);
-          }
-          if (!p.resident) {
-            umma_commit(&sh->a_empty[slot]);
-            ++a_it;
-          }
+        for (int kk = 0; kk < KA * kAtomK / 16; ++kk) {
+          const uint64_t bd = sw128_kmajor_desc(w2_addr + (ws * KA + (kk >> 2)) * kAtomBytes + (kk & 3) * 32);
+          umma_bf16_ts(d_tmem, a_tmem + kk * 8, bd, idesc, kk != 0);
         }
-        if (!ok) break;
         umma_commit(&sh->acc_full[abuf]);
+        if (!p.resident) umma_commit(&sh->a_empty[aslot]);
         const int64_t next_n = (u + 1 < u_end) ? (u + 1) / MT : -1;
-        if (next_n != n) umma_commit(&sh->w2_empty);
+        if (next_n != n) umma_commit(&sh->w2_empty[ws]);
       }
       // All MMAs issued by this thread are complete once `drain` flips.
       umma_commit(&sh->drain);
-      volatile int never = 0;
-      const WaitCtl drain_ctl{&never, p.status, p.wait_limit_ns};
       mbar_wait(&sh->drain, 0, drain_ctl);
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------ W1 gather -------
-    const int gt = threadIdx.x - 64;  // 0..63
-    const int rank = p.rank;
-    auto gather = [&](int m, int ka, int slot) {
-      uint8_t* dst = a_smem + slot * kAtomBytes;
-      uint4 vals[16];
-      bool bad = false;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int q = gt + 64 * i;
-        const int row = q >> 3, j = q & 7;
-        const int64_t grow = (int64_t)m * kBM + row;
-        vals[i] = make_uint4(0u, 0u, 0u, 0u);
-        if (grow < p.rows) {
-          const int64_t id = p.ids[grow];
-          if (id >= 0 && id < p.vocab)
-            vals[i] = ld_nc_v4(p.w1 + id * rank + ka * kAtomK + j * 8);
-          else
-            bad = true;
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int q = gt + 64 * i;
-        const int row = q >> 3, j = q & 7;
-        *reinterpret_cast<uint4*>(dst + row * 128 + ((j ^ (row & 7)) << 4)) = vals[i];
-      }
-      if (bad) report_status(p.status, DSPARK_STATUS_TOKEN_RANGE);
-      fence_proxy_async_smem();
-      mbar_arrive(&sh->a_full[slot]);
-    };
+  } else if (warp >= 4 && warp < 8) {
+    // --------------------------------------- W1 gather into TMEM -------
+    const int q = warp & 3;
+    const int row = 32 * q + lane;
+    const uint32_t lane_base = tmem_base + ((uint32_t)(32 * q) << 16);
     if (p.resident) {
-      for (int m = 0; m < MT; ++m)
-        for (int ka = 0; ka < KA; ++ka) gather(m, ka, m * KA + ka);
+      for (int m = 0; m < MT; ++m) {
+        gather_tile_to_tmem<KA>(p, m, row, lane_base + kAccCols + m * kACols);
+        tc_fence_before_sync();
+        mbar_arrive(&sh->a_full[m]);
+      }
     } else {
-      int64_t a_it = 0;
-      bool ok = true;
-      for (int64_t u = u_begin; u < u_end && ok; ++u) {
-        const int m = (int)(u % MT);
-        for (int ka = 0; ka < KA; ++ka, ++a_it) {
-          const int slot = (int)(a_it % p.a_slots);
-          if (!mbar_wait(&sh->a_empty[slot], ((uint32_t)(a_it / p.a_slots) & 1u) ^ 1u, ctl)) {
-            ok = false;
-            break;
-          }
-          gather(m, ka, slot);
-        }
+      int64_t it = 0;
+      for (int64_t u = u_begin; u < u_end; ++u, ++it) {
+        const int aslot = (int)(it & 1);
+        if (!warp_wait(&sh->a_empty[aslot], ((uint32_t)(it >> 1) & 1u) ^ 1u, ctl, lane)) break;
+        tc_fence_after_sync();
+        gather_tile_to_tmem<KA>(p, (int)(u % MT), row, lane_base + kAccCols + aslot * kACols);
+        tc_fence_before_sync();
+        mbar_arrive(&sh->a_full[aslot]);
       }
     }
-  } else {
+  } else if (warp >= 8) {
     // ------------------------------------------------- epilogue -------
-    const int et = threadIdx.x - 128;  // = TMEM lane = row within the tile
-    const int q = warp & 3;            // TMEM lane quarter this warp may access
-    const int row = et;
-    int64_t it = 0;
-    int prev_s = -1;
-    for (int64_t u = u_begin; u < u_end; ++u, ++it) {
+    const int g = (warp - 8) >> 2;        // group: even or odd units
+    const int et = threadIdx.x - 256 - 128 * g;  // 0..127 within the group
+    const int q = warp & 3;               // TMEM lane quarter this warp may access
+    const int row = 32 * q + lane;
+    const uint32_t bar_id = 1 + g;
+    int64_t it = g;
+    for (int64_t u = u_begin + g; u < u_end; u += 2, it += 2) {
       const int32_t n = (int32_t)(u / MT), m = (int32_t)(u % MT);
       const int s = (int)(it % p.u_stages);
-      const int abuf = (int)(it & 1);
       const uint32_t acc_par = (uint32_t)(it >> 1) & 1u;
       const uint32_t u_par = (uint32_t)(it / p.u_stages) & 1u;
       bool ok = true;
-      if (et == 0) ok = mbar_wait(&sh->acc_full[abuf], acc_par, ctl) && mbar_wait(&sh->u_full[s], u_par, ctl);
-      if (!barrier_and(ok, 1, 128)) break;
+      if (et == 0) ok = mbar_wait(&sh->acc_full[g], acc_par, ctl) && mbar_wait(&sh->u_full[s], u_par, ctl);
+      if (!barrier_and(ok, bar_id, 128)) break;
       if (et != 0) {
-        mbar_wait(&sh->acc_full[abuf], acc_par, ctl);
+        mbar_wait(&sh->acc_full[g], acc_par, ctl);
         mbar_wait(&sh->u_full[s], u_par, ctl);
       }
       tc_fence_after_sync();
       uint8_t* st = u_smem + s * kUStageBytes;
-      const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(abuf * kBN);
-#pragma unroll 2
-      for (int c = 0; c < kBN / 16; ++c) {
-        uint32_t acc[16];
-        tmem_ld_32x32b_x16(tbase + c * 16, acc);
-        tmem_ld_wait();
-        const int box = c >> 2;
-        const int j0 = (c & 3) * 2;
+      const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(g * kBN);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint4* ptr = reinterpret_cast<uint4*>(st + box * kAtomBytes + row * 128 + (((j0 + h) ^ (row & 7)) << 4));
+      for (int h = 0; h < 2; ++h) {  // the two 64-id boxes of the tile
+        uint32_t acc[64];
+        tmem_ld_32x32b_x32(tbase + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&acc[0]));
+        tmem_ld_32x32b_x32(tbase + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&acc[32]));
+        tmem_ld_wait();
+        uint8_t* box = st + h * kAtomBytes + row * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4* ptr = reinterpret_cast<uint4*>(box + ((c ^ (row & 7)) << 4));
           uint4 x = *ptr;
-          x.x = add_round_pair(x.x, acc[h * 8 + 0], acc[h * 8 + 1]);
-          x.y = add_round_pair(x.y, acc[h * 8 + 2], acc[h * 8 + 3]);
-          x.z = add_round_pair(x.z, acc[h * 8 + 4], acc[h * 8 + 5]);
-          x.w = add_round_pair(x.w, acc[h * 8 + 6], acc[h * 8 + 7]);
+          x.x = add_round_pair(x.x, acc[c * 8 + 0], acc[c * 8 + 1]);
+          x.y = add_round_pair(x.y, acc[c * 8 + 2], acc[c * 8 + 3]);
+          x.z = add_round_pair(x.z, acc[c * 8 + 4], acc[c * 8 + 5]);
+          x.w = add_round_pair(x.w, acc[c * 8 + 6], acc[c * 8 + 7]);
           *ptr = x;
         }
       }
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->acc_empty[abuf]);
+      if (lane == 0) mbar_arrive(&sh->acc_empty[g]);
       fence_proxy_async_smem();
-      named_barrier_sync(1, 128);
+      named_barrier_sync(bar_id, 128);
       if (et == 0) {
         tma_store_2d(&maps.out, st, n * kBN, m * kBM);
         tma_store_2d(&maps.out, st + kAtomBytes, n * kBN + 64, m * kBM);
         bulk_commit_group();
-        if (prev_s >= 0) {
-          bulk_wait_group_read<1>();
-          mbar_arrive(&sh->u_empty[prev_s]);
-        }
-        prev_s = s;
+        bulk_wait_group_read<0>();  // the stage may be refilled once the store has read it
+        mbar_arrive(&sh->u_empty[s]);
       }
     }
     if (et == 0) bulk_wait_group<0>();
@@ -355,25 +353,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 struct ApplyConfig {
-  int a_slots, u_stages, resident;
+  int w2_slots, u_stages, resident;
   size_t smem_bytes;
 };
 
 ApplyConfig plan(int ka, int row_tiles) {
   ApplyConfig c{};
-  const int free_slots = kSlotBudget - ka;
-  if (row_tiles * ka + 2 * 3 <= free_slots) {
-    c.resident = 1;
-    c.a_slots = row_tiles * ka;
-    c.u_stages = (free_slots - c.a_slots) / 2;
-    if (c.u_stages > 4) c.u_stages = 4;
-  } else {
-    c.resident = 0;
-    c.u_stages = 3;
-    c.a_slots = free_slots - 2 * c.u_stages;
-    if (c.a_slots > kMaxStages) c.a_slots = kMaxStages;
+  c.resident = (row_tiles <= kMaxResidentTiles && row_tiles * ka * 32 <= kTmemCols - kAccCols) ? 1 : 0;
+  const size_t fixed = 1024 + sizeof(SharedTail) + 64;
+  // Two W2 slots hide the reload at a vocab-tile change, which comes every
+  // row_tiles units; with many row tiles one slot leaves room for more U.
+  c.w2_slots = row_tiles < 8 ? 2 : 1;
+  for (;;) {
+    const size_t w2 = (size_t)c.w2_slots * ka * kAtomBytes;
+    int stages = (int)((kSmemLimit - fixed - w2) / kUStageBytes);
+    if (stages > kMaxStages) stages = kMaxStages;
+    if (stages >= 3 || c.w2_slots == 1) {
+      c.u_stages = stages;
+      break;
+    }
+    c.w2_slots = 1;
   }
-  c.smem_bytes = 1024 + (size_t)(ka + c.a_slots) * kAtomBytes + (size_t)c.u_stages * kUStageBytes + sizeof(SharedTail);
+  c.smem_bytes = fixed + (size_t)c.w2_slots * ka * kAtomBytes + (size_t)c.u_stages * kUStageBytes;
   return c;
 }
 
@@ -403,7 +404,7 @@ cudaError_t launch_ka(const TcApplyArgs& a, int num_sms, cudaStream_t stream) {
   p.row_tiles = (int32_t)((a.rows + kBM - 1) / kBM);
   p.vocab_tiles = (int32_t)((a.vocab + kBN - 1) / kBN);
   const ApplyConfig c = plan(KA, p.row_tiles);
-  p.a_slots = c.a_slots;
+  p.w2_slots = c.w2_slots;
   p.u_stages = c.u_stages;
   p.resident = c.resident;
   p.status = a.status;

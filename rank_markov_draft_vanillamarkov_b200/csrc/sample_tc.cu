@@ -68,6 +68,7 @@ struct SampleTail {
   uint64_t x_full, x_empty;
   uint64_t acc_full[2], acc_empty[2];
   uint64_t drain;
+  int64_t xid[kMaxBatch];
   uint32_t tmem_base;
   int abort_flag;
   int is_last;
@@ -255,9 +256,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       uint8_t* xdst = x_smem;
       bool bad = false;
-      for (int b0 = 0; b0 < BB; b0 += 32) {
+      // Ids of this step's rows into shared memory (-1: padding or invalid).
+      for (int b = lane; b < BB; b += 32) {
         int64_t id = -1;
-        const int b = b0 + lane;
         if (b < B) {
           id = k == 0 ? p.first_prev[b] : (int64_t)key_token(ld_relaxed_gpu(&p.keys[(size_t)(k - 1) * B + b]));
           if (k > 0 && blockIdx.x == 0) p.tokens[(size_t)b * M + (k - 1)] = id;
@@ -266,17 +267,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             id = -1;
           }
         }
-        // lane j of this pass holds the id of row b0 + j; rows are gathered
-        // 4 at a time per warp pass (8 chunks each).
-        for (int r = 0; r < 32 && b0 + r < BB; r += 4) {
-          const int row = b0 + r + (lane >> 3);
-          const int j = lane & 7;
-          const int64_t rid = __shfl_sync(0xffffffffu, id, r + (lane >> 3));
+        sh->xid[b] = id;
+      }
+      __syncwarp();
+      // Then every 16-byte chunk of the BB x rank operand: consecutive lanes
+      // take consecutive chunks of one row (coalesced), and each lane issues
+      // all the loads of a batch before its first store.
+      const int chunks_per_row = KA * 8;
+      const int total = BB * chunks_per_row;
+      constexpr int kBatch = 16;
+      for (int q0 = 0; q0 < total; q0 += 32 * kBatch) {
+        uint4 val[kBatch];
 #pragma unroll
-          for (int ka = 0; ka < KA; ++ka) {
-            uint4 val = make_uint4(0u, 0u, 0u, 0u);
-            if (rid >= 0) val = ld_nc_v4(p.w1 + rid * p.rank + ka * kAtomK + j * 8);
-            *reinterpret_cast<uint4*>(xdst + ka * atom_x + row * 128 + ((j ^ (row & 7)) << 4)) = val;
+        for (int i = 0; i < kBatch; ++i) {
+          const int q = q0 + lane + 32 * i;
+          val[i] = make_uint4(0u, 0u, 0u, 0u);
+          if (q < total) {
+            const int64_t rid = sh->xid[q / chunks_per_row];
+            if (rid >= 0) val[i] = ld_nc_v4(p.w1 + rid * p.rank + (q % chunks_per_row) * 8);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+          const int q = q0 + lane + 32 * i;
+          if (q < total) {
+            const int row = q / chunks_per_row, rem = q % chunks_per_row;
+            const int ka = rem >> 3, j = rem & 7;
+            *reinterpret_cast<uint4*>(xdst + ka * atom_x + row * 128 + ((j ^ (row & 7)) << 4)) = val[i];
           }
         }
       }
