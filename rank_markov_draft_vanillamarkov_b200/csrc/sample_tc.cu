@@ -19,8 +19,9 @@
 //   - merges its maxima into a per-(k, b) 64-bit key with atomicMax, then
 //     passes a grid barrier (bounded wait) after which every CTA decodes x_k.
 //
-// Warp roles (256 threads): 0 W2 producer, 1 MMA issuer + TMEM owner, 2 U
-// producer, 3 W1 gather + grid barrier, 4-7 epilogue (thread = vocab id).
+// Warp roles (384 threads): 0 W2 producer, 1 MMA issuer + TMEM owner, 2 U
+// producer, 3 W1 gather + grid barrier, 4-7 and 8-11 two epilogue groups that
+// take alternate tiles (one TMEM accumulator each; thread = vocab id).
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
@@ -31,7 +32,7 @@ namespace {
 constexpr int kBV = 128;               // vocabulary ids per tile (MMA M)
 constexpr int kAtomK = 64;             // bf16 elements per 128-byte swizzle row
 constexpr int kW2AtomBytes = 128 * 128;
-constexpr int kThreads = 256;  // 8 warps: one per role below, four for the epilogue
+constexpr int kThreads = 384;  // 12 warps: four single roles, two epilogue groups of four
 constexpr int kMaxStages = 12;
 constexpr int kMaxBatch = 256;
 constexpr size_t kSmemLimit = 232448;  // dynamic shared memory per block on sm_100
@@ -134,7 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* x_smem = w2_smem + (size_t)p.w2_slots * KA * kW2AtomBytes;  // one step's X
   uint8_t* u_smem = x_smem + (size_t)p.x_bytes;                       // u_slots x u_slot_bytes
   unsigned long long* red = reinterpret_cast<unsigned long long*>(u_smem + (size_t)p.u_slots * p.u_slot_bytes);
-  SampleTail* sh = reinterpret_cast<SampleTail*>(red + 4 * p.batch_pad);
+  SampleTail* sh = reinterpret_cast<SampleTail*>(red + 8 * p.batch_pad);  // [group][quarter][b]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -340,88 +341,96 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // -------------------------------------------------- epilogue ----
-    const int et = threadIdx.x - 128;  // vocabulary id within the tile = TMEM lane
+    // Group g takes the tiles whose item index k * nt + tt has parity g, and
+    // uses TMEM accumulator g. Thread (quarter q, lane) owns vocabulary id
+    // 32q + lane of the tile (its TMEM lane) and every batch column b.
+    const int g = (warp - 4) >> 2;
+    const int et = threadIdx.x - 128 - 128 * g;  // 0..127 within the group
+    const int t256 = threadIdx.x - 128;          // 0..255 across both groups
     const int q = warp & 3;
+    const int row = 32 * q + lane;
+    const uint32_t gbar = 1 + g, allbar = 3;
     const int groups = (B + 31) >> 5;
-    int prev_s = -1;
+    unsigned long long* my_red = red + (size_t)(g * 4 + q) * BB;
     bool ok = true;
-    for (int k = 0; k < M && ok; ++k) {
-      unsigned long long best[kMaxBatch / 32];
-#pragma unroll
-      for (int g = 0; g < kMaxBatch / 32; ++g) best[g] = 0ull;
-      for (int tt = 0; tt < nt; ++tt) {
+    for (int k = 0; k < M; ++k) {
+      for (int gg = 0; gg < groups; ++gg)
+        if (32 * gg + lane < BB) my_red[32 * gg + lane] = 0ull;
+      for (int tt = ((k * nt) & 1) == g ? 0 : 1; tt < nt && ok; tt += 2) {
         const int64_t i = (int64_t)k * nt + tt;
         const int s = (int)(i % p.u_slots);
-        const int abuf = (int)(i & 1);
         const uint32_t acc_par = (uint32_t)(i >> 1) & 1u;
         const uint32_t u_par = (uint32_t)(i / p.u_slots) & 1u;
         bool w_ok = true;
-        if (et == 0) w_ok = mbar_wait(&sh->acc_full[abuf], acc_par, ctl) && mbar_wait(&sh->u_full[s], u_par, ctl);
-        if (!barrier_and(w_ok, 1, 128)) {
+        if (et == 0) w_ok = mbar_wait(&sh->acc_full[g], acc_par, ctl) && mbar_wait(&sh->u_full[s], u_par, ctl);
+        if (!barrier_and(w_ok, gbar, 128)) {
           ok = false;
           break;
         }
         if (et != 0) {
-          mbar_wait(&sh->acc_full[abuf], acc_par, ctl);
+          mbar_wait(&sh->acc_full[g], acc_par, ctl);
           mbar_wait(&sh->u_full[s], u_par, ctl);
         }
         tc_fence_after_sync();
         const int t = t_begin + tt;
-        const uint32_t v = (uint32_t)(t * kBV + et);
+        const uint32_t v = (uint32_t)(t * kBV + row);
         const bool valid = (int64_t)v < p.vocab;
-        __nv_bfloat16* slot = reinterpret_cast<__nv_bfloat16*>(u_smem + (size_t)s * p.u_slot_bytes);
-        const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(abuf * BB);
-#pragma unroll
-        for (int g = 0; g < kMaxBatch / 32; ++g) {
-          if (g >= groups) break;
+        __nv_bfloat16* slot = reinterpret_cast<__nv_bfloat16*>(u_smem + (size_t)s * p.u_slot_bytes) + row;
+        const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(g * BB);
+#pragma unroll 1
+        for (int gg = 0; gg < groups; ++gg) {
           uint32_t d[32];
-          tmem_ld_32x32b_x16(tb + 32 * g, *reinterpret_cast<uint32_t(*)[16]>(&d[0]));
-          if (32 * g + 16 < BB) tmem_ld_32x32b_x16(tb + 32 * g + 16, *reinterpret_cast<uint32_t(*)[16]>(&d[16]));
+          tmem_ld_32x32b_x16(tb + 32 * gg, *reinterpret_cast<uint32_t(*)[16]>(&d[0]));
+          if (32 * gg + 16 < BB) tmem_ld_32x32b_x16(tb + 32 * gg + 16, *reinterpret_cast<uint32_t(*)[16]>(&d[16]));
           tmem_ld_wait();
+          const int nb = B - 32 * gg < 32 ? B - 32 * gg : 32;  // batch columns of this group
+          __nv_bfloat16* col = slot + (size_t)(32 * gg) * kBV;
+          // All loads first, then the arithmetic, then all stores: the loads
+          // of one thread are independent, so they overlap instead of each
+          // waiting out the shared-memory latency of the previous element.
+          __nv_bfloat16 c[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) c[j] = j < nb ? col[j * kBV] : __float2bfloat16_rn(0.0f);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) c[j] = __float2bfloat16_rn(__bfloat162float(c[j]) + __uint_as_float(d[j]));
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < nb) col[j * kBV] = c[j];
           unsigned long long key[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const int b = 32 * g + j;
-            key[j] = 0ull;
-            if (b < B) {
-              __nv_bfloat16* e = slot + (size_t)b * kBV + et;
-              const __nv_bfloat16 c = __float2bfloat16_rn(__bfloat162float(*e) + __uint_as_float(d[j]));
-              *e = c;
-              float score = __bfloat162float(c);
-              if (!p.greedy) score = score / p.temperature + noise_for(p.seed, (uint32_t)b, (uint32_t)k, v);
-              if (valid) key[j] = pack_key(score, v);
-            }
+            float score = __bfloat162float(c[j]);
+            if (!p.greedy) score = score / p.temperature + noise_for(p.seed, (uint32_t)(32 * gg + j), (uint32_t)k, v);
+            key[j] = (j < nb && valid) ? pack_key(score, v) : 0ull;
           }
-          best[g] = umax64(best[g], transpose_max32(key, lane));
+          const unsigned long long best = transpose_max32(key, lane);
+          if (32 * gg + lane < BB) my_red[32 * gg + lane] = umax64(my_red[32 * gg + lane], best);
         }
         tc_fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sh->acc_empty[abuf]);
+        if (lane == 0) mbar_arrive(&sh->acc_empty[g]);
         fence_proxy_async_smem();
-        named_barrier_sync(1, 128);
+        named_barrier_sync(gbar, 128);
         if (et == 0) {
-          tma_store_3d(&maps.out, slot, t * kBV, k, 0);
+          tma_store_3d(&maps.out, slot - row, t * kBV, k, 0);
           bulk_commit_group();
-          if (prev_s >= 0) {
-            bulk_wait_group_read<1>();
-            mbar_arrive(&sh->u_empty[prev_s]);
-          }
-          prev_s = s;
+          bulk_wait_group_read<0>();  // the slot may be refilled once the store has read it
+          mbar_arrive(&sh->u_empty[s]);
         }
       }
-      if (!ok) break;
-      // Merge the four warps' maxima, then this CTA's into the global keys.
+      // Both groups agree to go on (an abort anywhere ends every step here).
+      if (!barrier_and(ok, allbar, 256)) break;
+      // Merge the eight partial maxima of each b, then this CTA's into the
+      // global keys.
+      for (int b = t256; b < B; b += 256) {
+        unsigned long long m = 0ull;
 #pragma unroll
-      for (int g = 0; g < kMaxBatch / 32; ++g)
-        if (g < groups && 32 * g + lane < BB) red[q * BB + 32 * g + lane] = best[g];  // BB may be 16
-      named_barrier_sync(1, 128);
-      for (int b = et; b < B; b += 128) {
-        const unsigned long long m = umax64(umax64(red[b], red[BB + b]), umax64(red[2 * BB + b], red[3 * BB + b]));
+        for (int r = 0; r < 8; ++r) m = umax64(m, red[(size_t)r * BB + b]);
         atomicMax(&p.keys[(size_t)k * B + b], m);
       }
       __threadfence();
-      named_barrier_sync(1, 128);
-      if (et == 0) {
+      named_barrier_sync(allbar, 256);
+      if (t256 == 0) {
         const bool skip = (p.debug_flags & DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL) && blockIdx.x == 0 && k == 0;
         int last = 0;
         if (!skip) {
@@ -431,13 +440,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         sh->is_last = last;
       }
-      if (k == M - 1) {
-        named_barrier_sync(1, 128);
-        if (sh->is_last) {
-          __threadfence();
-          for (int b = et; b < B; b += 128)
-            p.tokens[(size_t)b * M + (M - 1)] = (int64_t)key_token(ld_relaxed_gpu(&p.keys[(size_t)(M - 1) * B + b]));
-        }
+      named_barrier_sync(allbar, 256);
+      if (k == M - 1 && sh->is_last) {
+        __threadfence();
+        for (int b = t256; b < B; b += 256)
+          p.tokens[(size_t)b * M + (M - 1)] = (int64_t)key_token(ld_relaxed_gpu(&p.keys[(size_t)(M - 1) * B + b]));
       }
     }
     if (et == 0) bulk_wait_group<0>();
@@ -462,7 +469,7 @@ SampleConfig plan(int ka, int batch, int batch_pad) {
   SampleConfig c{};
   c.u_slot_bytes = (uint32_t)align1024((size_t)batch * kBV * 2);
   c.x_bytes = (uint32_t)((size_t)ka * batch_pad * 128);
-  const size_t fixed = 1024 + (size_t)c.x_bytes + 4 * (size_t)batch_pad * 8 + sizeof(SampleTail) + 64;
+  const size_t fixed = 1024 + (size_t)c.x_bytes + 8 * (size_t)batch_pad * 8 + sizeof(SampleTail) + 64;
   const size_t w2_slot = (size_t)ka * kW2AtomBytes;
   for (int w = 4; w >= 1; --w) {
     for (int u = 8; u >= 2; --u) {
