@@ -124,6 +124,7 @@ __device__ __forceinline__ void gather_tile_to_tmem(const ApplyParams& p, int m,
       id = -1;
     }
   }
+  __syncwarp();  // tcgen05.st below is warp-aligned
   const uint4* src = reinterpret_cast<const uint4*>(p.w1 + (id < 0 ? 0 : id) * p.rank);
 #pragma unroll
   for (int c = 0; c < KA; ++c) {  // 64 bf16 = 32 words = 8 loads per chunk
@@ -166,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sh->acc_full[i], 1);
       mbar_init(&sh->acc_empty[i], 4);
     }
-    for (int i = 0; i < kMaxResidentTiles; ++i) mbar_init(&sh->a_full[i], 128);
+    for (int i = 0; i < kMaxResidentTiles; ++i) mbar_init(&sh->a_full[i], 4);  // one arrival per gather warp
     for (int i = 0; i < p.u_stages; ++i) {
       mbar_init(&sh->u_full[i], 1);
       mbar_init(&sh->u_empty[i], 1);
@@ -179,6 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&sh->tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  __syncwarp();  // warp 0 diverged around the barrier set-up
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -276,7 +278,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int m = 0; m < MT; ++m) {
         gather_tile_to_tmem<KA>(p, m, row, lane_base + kAccCols + m * kACols);
         tc_fence_before_sync();
-        mbar_arrive(&sh->a_full[m]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->a_full[m]);
       }
     } else {
       int64_t it = 0;
@@ -286,7 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after_sync();
         gather_tile_to_tmem<KA>(p, (int)(u % MT), row, lane_base + kAccCols + aslot * kACols);
         tc_fence_before_sync();
-        mbar_arrive(&sh->a_full[aslot]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->a_full[aslot]);
       }
     }
   } else if (warp >= 8) {
@@ -304,11 +308,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t u_par = (uint32_t)(it / p.u_stages) & 1u;
       bool ok = true;
       if (et == 0) ok = mbar_wait(&sh->acc_full[g], acc_par, ctl) && mbar_wait(&sh->u_full[s], u_par, ctl);
+      __syncwarp();
       if (!barrier_and(ok, bar_id, 128)) break;
       if (et != 0) {
         mbar_wait(&sh->acc_full[g], acc_par, ctl);
         mbar_wait(&sh->u_full[s], u_par, ctl);
       }
+      __syncwarp();  // tcgen05.ld below is warp-aligned
       tc_fence_after_sync();
       uint8_t* st = u_smem + s * kUStageBytes;
       const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(g * kBN);
@@ -333,6 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->acc_empty[g]);
+      __syncwarp();
       fence_proxy_async_smem();
       named_barrier_sync(bar_id, 128);
       if (et == 0) {
@@ -342,10 +349,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_wait_group_read<0>();  // the stage may be refilled once the store has read it
         mbar_arrive(&sh->u_empty[s]);
       }
+      __syncwarp();
     }
     if (et == 0) bulk_wait_group<0>();
   }
 
+  // Single-lane roles and lane-0 branches leave warps diverged; bar.sync is
+  // warp-aligned, so every warp reconverges first.
+  __syncwarp();
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();

@@ -39,6 +39,7 @@ constexpr size_t kSmemLimit = 232448;  // dynamic shared memory per block on sm_
 
 struct __align__(64) SampleMaps {
   CUtensorMap w2;   // [vocab, rank] bf16, box 64 x 128, 128B swizzle
+  CUtensorMap w1;   // [vocab, rank] bf16, box 64 x 1 (row gathers), 128B swizzle
   CUtensorMap u;    // [batch, steps, vocab] bf16, box 128 x 1 x batch
   CUtensorMap out;  // same geometry as u
 };
@@ -69,7 +70,7 @@ struct SampleTail {
   uint64_t x_full, x_empty;
   uint64_t acc_full[2], acc_empty[2];
   uint64_t drain;
-  int64_t xid[kMaxBatch];
+  int32_t xid[kMaxBatch];
   uint32_t tmem_base;
   int abort_flag;
   int is_last;
@@ -126,7 +127,8 @@ __device__ __forceinline__ unsigned long long transpose_max32(unsigned long long
   return k[0];
 }
 
-template <int KA>
+// GREEDY selects at compile time: the greedy instance carries no noise code.
+template <int KA, bool GREEDY>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_sample_kernel(const __grid_constant__ SampleMaps maps, const SampleParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -158,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sh->u_full[i], 1);
       mbar_init(&sh->u_empty[i], 1);
     }
-    mbar_init(&sh->x_full, 32);
+    mbar_init(&sh->x_full, 1);
     mbar_init(&sh->x_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sh->acc_full[i], 1);
@@ -173,6 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&sh->tmem_base, p.tmem_cols);
     tmem_relinquish();
   }
+  __syncwarp();  // warp 0 diverged around the barrier set-up
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -221,6 +224,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 3) {
     // ------------------------------------ W1 gather + grid barrier ----
+    const uint64_t pol_w1 = policy_evict_last();
+    if (lane == 0) prefetch_tensormap(&maps.w1);
     // One X buffer suffices: step k+1's rows are gathered only after the grid
     // barrier, i.e. after every MMA of step k has completed.
     for (int k = 0; k < M; ++k) {
@@ -255,52 +260,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (!ok) break;
       }
-      uint8_t* xdst = x_smem;
       bool bad = false;
-      // Ids of this step's rows into shared memory (-1: padding or invalid).
+      // Row of W1 for each batch column; padding columns and invalid ids use
+      // row `vocab`, outside the tensor, which the gather reads as zeros.
       for (int b = lane; b < BB; b += 32) {
-        int64_t id = -1;
+        int32_t row = (int32_t)p.vocab;
         if (b < B) {
-          id = k == 0 ? p.first_prev[b] : (int64_t)key_token(ld_relaxed_gpu(&p.keys[(size_t)(k - 1) * B + b]));
+          const int64_t id =
+              k == 0 ? p.first_prev[b] : (int64_t)key_token(ld_relaxed_gpu(&p.keys[(size_t)(k - 1) * B + b]));
           if (k > 0 && blockIdx.x == 0) p.tokens[(size_t)b * M + (k - 1)] = id;
-          if (id < 0 || id >= p.vocab) {
+          if (id < 0 || id >= p.vocab)
             bad = true;
-            id = -1;
-          }
+          else
+            row = (int32_t)id;
         }
-        sh->xid[b] = id;
-      }
-      __syncwarp();
-      // Then every 16-byte chunk of the BB x rank operand: consecutive lanes
-      // take consecutive chunks of one row (coalesced), and each lane issues
-      // all the loads of a batch before its first store.
-      const int chunks_per_row = KA * 8;
-      const int total = BB * chunks_per_row;
-      constexpr int kBatch = 16;
-      for (int q0 = 0; q0 < total; q0 += 32 * kBatch) {
-        uint4 val[kBatch];
-#pragma unroll
-        for (int i = 0; i < kBatch; ++i) {
-          const int q = q0 + lane + 32 * i;
-          val[i] = make_uint4(0u, 0u, 0u, 0u);
-          if (q < total) {
-            const int64_t rid = sh->xid[q / chunks_per_row];
-            if (rid >= 0) val[i] = ld_nc_v4(p.w1 + rid * p.rank + (q % chunks_per_row) * 8);
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < kBatch; ++i) {
-          const int q = q0 + lane + 32 * i;
-          if (q < total) {
-            const int row = q / chunks_per_row, rem = q % chunks_per_row;
-            const int ka = rem >> 3, j = rem & 7;
-            *reinterpret_cast<uint4*>(xdst + ka * atom_x + row * 128 + ((j ^ (row & 7)) << 4)) = val[i];
-          }
-        }
+        sh->xid[b] = row;
       }
       if (bad) report_status(p.status, DSPARK_STATUS_TOKEN_RANGE);
-      fence_proxy_async_smem();
-      mbar_arrive(&sh->x_full);
+      __syncwarp();
+      // The operand arrives through the async proxy (TMA row gathers into the
+      // 128-byte-swizzle K-major layout), so no proxy fence is needed before
+      // the MMA reads it: x_full completes on the transferred byte count.
+      if (lane == 0) mbar_arrive_expect_tx(&sh->x_full, p.x_bytes);
+      __syncwarp();
+      const int quads = BB / 4;
+      for (int i = lane; i < quads * KA; i += 32) {
+        const int j = i % quads, ka = i / quads;
+        tma_gather4(x_smem + ka * atom_x + j * 4 * 128, &maps.w1, &sh->x_full, ka * kAtomK, sh->xid[4 * j],
+                    sh->xid[4 * j + 1], sh->xid[4 * j + 2], sh->xid[4 * j + 3], pol_w1);
+      }
+      __syncwarp();
     }
   } else if (warp == 1) {
     // ------------------------------------------------- MMA issuer ----
@@ -363,6 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t u_par = (uint32_t)(i / p.u_slots) & 1u;
         bool w_ok = true;
         if (et == 0) w_ok = mbar_wait(&sh->acc_full[g], acc_par, ctl) && mbar_wait(&sh->u_full[s], u_par, ctl);
+        __syncwarp();
         if (!barrier_and(w_ok, gbar, 128)) {
           ok = false;
           break;
@@ -371,6 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(&sh->acc_full[g], acc_par, ctl);
           mbar_wait(&sh->u_full[s], u_par, ctl);
         }
+        __syncwarp();  // tcgen05.ld below is warp-aligned
         tc_fence_after_sync();
         const int t = t_begin + tt;
         const uint32_t v = (uint32_t)(t * kBV + row);
@@ -400,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             float score = __bfloat162float(c[j]);
-            if (!p.greedy) score = score / p.temperature + noise_for(p.seed, (uint32_t)(32 * gg + j), (uint32_t)k, v);
+            if (!GREEDY) score = score / p.temperature + noise_for(p.seed, (uint32_t)(32 * gg + j), (uint32_t)k, v);
             key[j] = (j < nb && valid) ? pack_key(score, v) : 0ull;
           }
           const unsigned long long best = transpose_max32(key, lane);
@@ -409,6 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh->acc_empty[g]);
+        __syncwarp();
         fence_proxy_async_smem();
         named_barrier_sync(gbar, 128);
         if (et == 0) {
@@ -417,6 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_wait_group_read<0>();  // the slot may be refilled once the store has read it
           mbar_arrive(&sh->u_empty[s]);
         }
+        __syncwarp();
       }
       // Both groups agree to go on (an abort anywhere ends every step here).
       if (!barrier_and(ok, allbar, 256)) break;
@@ -440,6 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         sh->is_last = last;
       }
+      __syncwarp();
       named_barrier_sync(allbar, 256);
       if (k == M - 1 && sh->is_last) {
         __threadfence();
@@ -450,6 +444,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (et == 0) bulk_wait_group<0>();
   }
 
+  // Single-lane roles and lane-0 branches leave warps diverged; bar.sync is
+  // warp-aligned, so every warp reconverges first.
+  __syncwarp();
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -495,7 +492,7 @@ uint32_t tmem_cols_for(int batch_pad) {
   return cols;
 }
 
-template <int KA>
+template <int KA, bool GREEDY>
 cudaError_t launch_ka(const TcSampleArgs& a, int num_sms, cudaStream_t stream) {
   const int BB = batch_pad_of(a.batch);
   const SampleConfig c = plan(KA, (int)a.batch, BB);
@@ -505,6 +502,10 @@ cudaError_t launch_ka(const TcSampleArgs& a, int num_sms, cudaStream_t stream) {
   const uint64_t wdim[2] = {(uint64_t)a.rank, (uint64_t)a.vocab};
   const uint64_t wstr[1] = {(uint64_t)a.rank * 2};
   if (!encode_tensor_map(&maps.w2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.w2, wdim, wstr, wbox,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  const uint32_t rbox[2] = {64, 1};
+  if (!encode_tensor_map(&maps.w1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.w1, wdim, wstr, rbox,
                          CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   const uint64_t udim[3] = {(uint64_t)a.vocab, (uint64_t)a.steps, (uint64_t)a.batch};
@@ -540,7 +541,7 @@ cudaError_t launch_ka(const TcSampleArgs& a, int num_sms, cudaStream_t stream) {
   p.debug_flags = a.debug_flags;
   p.tmem_cols = tmem_cols_for(BB);
 
-  cudaError_t e = cudaFuncSetAttribute(tc_sample_kernel<KA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(tc_sample_kernel<KA, GREEDY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)c.smem_bytes);
   if (e != cudaSuccess) return e;
   const int grid = p.vocab_tiles < num_sms ? p.vocab_tiles : num_sms;
@@ -554,9 +555,20 @@ cudaError_t launch_ka(const TcSampleArgs& a, int num_sms, cudaStream_t stream) {
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, tc_sample_kernel<KA>, maps, p);
+  e = cudaLaunchKernelEx(&cfg, tc_sample_kernel<KA, GREEDY>, maps, p);
   note_launch();
   return e;
+}
+
+template <bool GREEDY>
+cudaError_t launch_mode(const TcSampleArgs& a, int num_sms, cudaStream_t s) {
+  switch (a.rank / 64) {
+    case 1: return launch_ka<1, GREEDY>(a, num_sms, s);
+    case 2: return launch_ka<2, GREEDY>(a, num_sms, s);
+    case 3: return launch_ka<3, GREEDY>(a, num_sms, s);
+    case 4: return launch_ka<4, GREEDY>(a, num_sms, s);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace
@@ -570,13 +582,7 @@ bool tc_sample_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_
 }
 
 cudaError_t launch_tc_sample(const TcSampleArgs& a, int num_sms, cudaStream_t s) {
-  switch (a.rank / 64) {
-    case 1: return launch_ka<1>(a, num_sms, s);
-    case 2: return launch_ka<2>(a, num_sms, s);
-    case 3: return launch_ka<3>(a, num_sms, s);
-    case 4: return launch_ka<4>(a, num_sms, s);
-    default: return cudaErrorInvalidValue;
-  }
+  return a.greedy ? launch_mode<true>(a, num_sms, s) : launch_mode<false>(a, num_sms, s);
 }
 
 }  // namespace dspark
