@@ -169,7 +169,7 @@ int dspark_markov_sample_block(const void* base_logits, const int64_t* first_pre
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool greedy = !(temperature >= 1e-5f);
   const int32_t algo = g_algo.load();
-  const bool tc_ok = tc_sample_supported(batch, vocab, rank, logits_dtype, weight_dtype) &&
+  const bool tc_ok = tc_sample_supported(batch, vocab, rank, logits_dtype, weight_dtype, d->num_sms) &&
                      (reinterpret_cast<uintptr_t>(base_logits) % 16 == 0) &&
                      (reinterpret_cast<uintptr_t>(corrected_logits) % 16 == 0) &&
                      (reinterpret_cast<uintptr_t>(w2) % 16 == 0) && (reinterpret_cast<uintptr_t>(w1) % 16 == 0);

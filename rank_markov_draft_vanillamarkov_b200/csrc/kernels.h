@@ -56,7 +56,8 @@ bool tc_apply_supported(int64_t rows, int64_t vocab, int32_t rank, int logits_dt
 cudaError_t launch_tc_apply(const TcApplyArgs& a, int num_sms, cudaStream_t s);
 
 // Persistent left-to-right sampler on tcgen05: bf16 logits, bf16 weights,
-// vocab % 8 == 0, rank in {64, 128, 192, 256}, batch <= 256.
+// vocab % 8 == 0, rank in {64, 128, 192, 256}, batch <= 256 (and within the
+// shared-memory plan), at most 512 vocabulary tiles per CTA.
 struct TcSampleArgs {
   const void* base;
   const int64_t* first_prev;
@@ -75,7 +76,8 @@ struct TcSampleArgs {
   uint64_t wait_limit_ns;
   uint32_t debug_flags;
 };
-bool tc_sample_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype);
+bool tc_sample_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype,
+                         int num_sms);
 cudaError_t launch_tc_sample(const TcSampleArgs& a, int num_sms, cudaStream_t s);
 
 // Encodes a tiled TMA descriptor through the driver entry point.

@@ -8,20 +8,31 @@
 //
 // with x_{-1} = first_prev. One launch covers all M steps. The grid is one
 // CTA per SM (cooperative launch, so all CTAs are resident); CTA c owns a
-// contiguous run of 128-id vocabulary tiles. Per step each CTA
-//   - computes bias^T = W2_tile[128 x r] . X^T[r x B] on tcgen05 (swap-AB:
-//     M = 128 ids, N = B padded to 16, K = r), X = the gathered W1 rows of
-//     x_{k-1}; W2 tiles come from L2 (loaded with an evict-last policy, so
-//     the M steps re-read them from L2, not HBM);
+// contiguous run of 128-id vocabulary tiles.
+//
+// W2 stays on chip for the whole launch. Each CTA loads its slice of W2 once:
+// as many tiles as fit into shared memory (by TMA, 128-byte swizzle), the rest
+// into tensor memory (tcgen05.st), where they serve as the A operand of the
+// MMA directly. Across 148 SMs that holds a 33 MB W2, so the M steps read it
+// from HBM once and never again.
+//
+// Per step each CTA
+//   - gathers X = W1[x_{k-1}] ([B_pad x r], TMA tile::gather4 row gathers);
+//   - computes bias^T = W2_tile[128 x r] . X^T[r x B_pad] per vocabulary tile
+//     on tcgen05 (swap-AB: M = 128 ids, N = B padded to 16, K = r);
 //   - adds U (TMA-staged [B x 128] tiles, prefetched across step boundaries
 //     since U does not depend on the chain), rounds to bf16, stores c_k, and
-//     keeps the packed (score, -id) maximum per b;
+//     keeps the packed (score, id) maximum per b;
 //   - merges its maxima into a per-(k, b) 64-bit key with atomicMax, then
 //     passes a grid barrier (bounded wait) after which every CTA decodes x_k.
 //
-// Warp roles (384 threads): 0 W2 producer, 1 MMA issuer + TMEM owner, 2 U
-// producer, 3 W1 gather + grid barrier, 4-7 and 8-11 two epilogue groups that
-// take alternate tiles (one TMEM accumulator each; thread = vocab id).
+// Warp roles (640 threads): 0 W2 loader, 1 MMA issuer + TMEM owner, 2 U
+// producer, 3 W1 gather + grid barrier, 4-19 up to four epilogue groups of
+// four warps that take tiles round-robin (one TMEM accumulator each; thread =
+// vocab id). Several groups in flight hide the shared-memory and shuffle
+// latency of the per-element work and even out the tile counts per step.
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
@@ -29,13 +40,18 @@
 namespace dspark {
 namespace {
 
-constexpr int kBV = 128;               // vocabulary ids per tile (MMA M)
-constexpr int kAtomK = 64;             // bf16 elements per 128-byte swizzle row
-constexpr int kW2AtomBytes = 128 * 128;
-constexpr int kThreads = 384;  // 12 warps: four single roles, two epilogue groups of four
+constexpr int kBV = 128;                           // vocabulary ids per tile (MMA M)
+constexpr int kAtomK = 64;                         // bf16 elements per 128-byte swizzle row
+constexpr int kW2AtomBytes = 128 * 128;            // one 128-id x 64-element W2 atom
+constexpr int kMaxGroups = 4;                      // epilogue groups
+constexpr int kThreads = 128 + kMaxGroups * 128;   // four single-role warps + the groups
 constexpr int kMaxStages = 12;
 constexpr int kMaxBatch = 256;
-constexpr size_t kSmemLimit = 232448;  // dynamic shared memory per block on sm_100
+constexpr int kMaxTiles = 24;                      // vocabulary tiles per CTA
+constexpr uint32_t kTmemCols = 512;
+constexpr size_t kSmemLimit = 232448;              // dynamic shared memory per block on sm_100
+
+__host__ __device__ constexpr size_t align8(size_t x) { return (x + 7) & ~size_t(7); }
 
 struct __align__(64) SampleMaps {
   CUtensorMap w2;   // [vocab, rank] bf16, box 64 x 128, 128B swizzle
@@ -46,7 +62,7 @@ struct __align__(64) SampleMaps {
 
 struct SampleParams {
   const int64_t* first_prev;
-  const __nv_bfloat16* w1;
+  const __nv_bfloat16* w2;
   int64_t* tokens;
   unsigned long long* keys;
   uint32_t* barrier;
@@ -54,21 +70,21 @@ struct SampleParams {
   int32_t batch, batch_pad, steps, rank;
   int64_t vocab;
   int32_t vocab_tiles;
-  int32_t w2_slots, u_slots;
+  int32_t smem_tiles;  // W2 tiles a CTA keeps in shared memory; the rest go to TMEM
+  int32_t u_slots;
   uint32_t u_slot_bytes, x_bytes;  // x_bytes: one step's gathered operand
   float temperature;
-  int32_t greedy;
   uint64_t seed;
   uint64_t wait_limit_ns;
   uint32_t debug_flags;
-  uint32_t tmem_cols;
+  int32_t groups;  // epilogue groups in use (<= kMaxGroups)
 };
 
 struct SampleTail {
-  uint64_t w2_full[kMaxStages], w2_empty[kMaxStages];
+  uint64_t w2_full, w2t_full;
   uint64_t u_full[kMaxStages], u_empty[kMaxStages];
   uint64_t x_full, x_empty;
-  uint64_t acc_full[2], acc_empty[2];
+  uint64_t acc_full[kMaxGroups], acc_empty[kMaxGroups];
   uint64_t drain;
   int32_t xid[kMaxBatch];
   uint32_t tmem_base;
@@ -104,40 +120,55 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   return r;
 }
 
-__device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsigned long long b) {
-  return a > b ? a : b;
-}
-
-// Thirty-two keys per lane in; lane L leaves with the warp-wide maximum of key
-// index L. Each round halves the keys a lane holds: it keeps the half whose
-// index bit matches its own lane bit and trades the other half with the lane
-// across that bit.
-__device__ __forceinline__ unsigned long long transpose_max32(unsigned long long (&k)[32], int lane) {
+// Sixteen keys per lane in; lanes 2i and 2i+1 leave with the warp-wide
+// maximum of key index i. Each of the first four rounds halves the keys a lane
+// holds: it keeps the half whose index bit matches a lane bit and trades the
+// other half with the lane across that bit; the last round merges lane pairs.
+template <typename K>
+__device__ __forceinline__ K transpose_max16(K (&k)[16], int lane) {
 #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
+  for (int r = 0; r < 4; ++r) {
+    const int o = 16 >> r;    // lane bit of this round
+    const int half = 8 >> r;  // keys kept
     const bool upper = (lane & o) != 0;
 #pragma unroll
-    for (int j = 0; j < o; ++j) {
-      const unsigned long long send = upper ? k[j] : k[j + o];
-      const unsigned long long keep = upper ? k[j + o] : k[j];
-      const unsigned long long recv = __shfl_xor_sync(0xffffffffu, send, o);
-      k[j] = umax64(keep, recv);
+    for (int j = 0; j < half; ++j) {
+      const K send = upper ? k[j] : k[j + half];
+      const K keep = upper ? k[j + half] : k[j];
+      const K recv = __shfl_xor_sync(0xffffffffu, send, o);
+      k[j] = keep > recv ? keep : recv;
     }
   }
-  return k[0];
+  const K other = __shfl_xor_sync(0xffffffffu, k[0], 1);
+  return k[0] > other ? k[0] : other;
+}
+
+// Greedy key of a bf16 corrected logit: its bits mapped to an unsigned order
+// in the high half (NaN made +qNaN, above +inf; -0 made +0) and the
+// complement of the CTA-local vocabulary index in the low half, so that the
+// maximum is the largest value and, among equal values, the lowest id.
+__device__ __forceinline__ uint32_t greedy_key(uint32_t bits, uint32_t local_id) {
+  bits &= 0xFFFFu;
+  if ((bits & 0x7FFFu) > 0x7F80u) bits = 0x7FC0u;
+  if (bits == 0x8000u) bits = 0u;
+  const uint32_t ord = (bits & 0x8000u) ? (~bits & 0xFFFFu) : (bits | 0x8000u);
+  return (ord << 16) | (0xFFFFu - local_id);
 }
 
 // GREEDY selects at compile time: the greedy instance carries no noise code.
 template <int KA, bool GREEDY>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_sample_kernel(const __grid_constant__ SampleMaps maps, const SampleParams p) {
+  using Key = typename std::conditional<GREEDY, uint32_t, unsigned long long>::type;
+  constexpr int kTileCols = KA * 32;  // TMEM columns of one W2 tile (two bf16 per column)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* w2_smem = smem;                                            // w2_slots x KA atoms
-  uint8_t* x_smem = w2_smem + (size_t)p.w2_slots * KA * kW2AtomBytes;  // one step's X
-  uint8_t* u_smem = x_smem + (size_t)p.x_bytes;                       // u_slots x u_slot_bytes
-  unsigned long long* red = reinterpret_cast<unsigned long long*>(u_smem + (size_t)p.u_slots * p.u_slot_bytes);
-  SampleTail* sh = reinterpret_cast<SampleTail*>(red + 8 * p.batch_pad);  // [group][quarter][b]
+  uint8_t* w2_smem = smem;                                              // smem_tiles x KA atoms
+  uint8_t* x_smem = w2_smem + (size_t)p.smem_tiles * KA * kW2AtomBytes;  // one step's X
+  uint8_t* u_smem = x_smem + (size_t)p.x_bytes;                         // u_slots x u_slot_bytes
+  Key* red = reinterpret_cast<Key*>(u_smem + (size_t)p.u_slots * p.u_slot_bytes);  // [group][quarter][b]
+  SampleTail* sh = reinterpret_cast<SampleTail*>(
+      u_smem + (size_t)p.u_slots * p.u_slot_bytes + align8((size_t)kMaxGroups * 4 * p.batch_pad * sizeof(Key)));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -145,24 +176,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int t_begin = (int)((int64_t)p.vocab_tiles * blockIdx.x / G);
   const int t_end = (int)((int64_t)p.vocab_tiles * (blockIdx.x + 1) / G);
   const int nt = t_end - t_begin;
+  const int n_smem = nt < p.smem_tiles ? nt : p.smem_tiles;  // tiles [0, n_smem) in smem, the rest in TMEM
   const int M = p.steps;
   const int B = p.batch;
   const int BB = p.batch_pad;
+  const int NG = p.groups;
   const int64_t items = (int64_t)M * nt;
   const uint32_t atom_x = (uint32_t)BB * 128u;  // bytes of one X atom
+  const uint32_t acc_cols = (uint32_t)(NG * BB);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < p.w2_slots; ++i) {
-      mbar_init(&sh->w2_full[i], 1);
-      mbar_init(&sh->w2_empty[i], 1);
-    }
+    mbar_init(&sh->w2_full, 1);
+    mbar_init(&sh->w2t_full, 4);
     for (int i = 0; i < p.u_slots; ++i) {
       mbar_init(&sh->u_full[i], 1);
       mbar_init(&sh->u_empty[i], 1);
     }
     mbar_init(&sh->x_full, 1);
     mbar_init(&sh->x_empty, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kMaxGroups; ++i) {
       mbar_init(&sh->acc_full[i], 1);
       mbar_init(&sh->acc_empty[i], 4);
     }
@@ -172,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(&sh->tmem_base, p.tmem_cols);
+    tmem_alloc(&sh->tmem_base, kTmemCols);
     tmem_relinquish();
   }
   __syncwarp();  // warp 0 diverged around the barrier set-up
@@ -185,24 +217,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const WaitCtl drain_ctl{&never, p.status, p.wait_limit_ns};
 
   if (warp == 0) {
-    // ----------------------------------------------- W2 producer ----
-    if (lane == 0) {
+    // ---------------------------------------- W2 into shared memory ----
+    if (lane == 0 && n_smem > 0) {
       prefetch_tensormap(&maps.w2);
-      const uint64_t pol_keep = policy_evict_last();
-      int64_t i = 0;
-      for (; i < items; ++i) {
-        const int t = t_begin + (int)(i % nt);
-        const int w = (int)(i % p.w2_slots);
-        if (!mbar_wait(&sh->w2_empty[w], ((uint32_t)(i / p.w2_slots) & 1u) ^ 1u, ctl)) break;
-        mbar_arrive_expect_tx(&sh->w2_full[w], KA * kW2AtomBytes);
-        uint8_t* dst = w2_smem + (size_t)w * KA * kW2AtomBytes;
+      const uint64_t pol = policy_evict_first();
+      mbar_arrive_expect_tx(&sh->w2_full, (uint32_t)(n_smem * KA * kW2AtomBytes));
+      for (int tt = 0; tt < n_smem; ++tt)
 #pragma unroll
         for (int ka = 0; ka < KA; ++ka)
-          tma_load_2d(dst + ka * kW2AtomBytes, &maps.w2, &sh->w2_full[w], ka * kAtomK, t * kBV, pol_keep);
-      }
-      // Drain: wait for the last fill of every slot this thread started.
-      for (int64_t j = (i > p.w2_slots ? i - p.w2_slots : 0); j < i; ++j)
-        mbar_wait(&sh->w2_full[j % p.w2_slots], (uint32_t)(j / p.w2_slots) & 1u, drain_ctl);
+          tma_load_2d(w2_smem + (size_t)(tt * KA + ka) * kW2AtomBytes, &maps.w2, &sh->w2_full, ka * kAtomK,
+                      (t_begin + tt) * kBV, pol);
+      mbar_wait(&sh->w2_full, 0, drain_ctl);  // the copies are done before this thread may exit
     }
   } else if (warp == 2) {
     // ------------------------------------------------ U producer ----
@@ -253,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               ok = false;
               break;
             }
-            __nanosleep(64);
+            __nanosleep(32);
           }
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -297,30 +322,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc = idesc_bf16_f32(kBV, (uint32_t)BB);
       const uint32_t w2_addr = smem_u32(w2_smem);
       const uint32_t x_addr = smem_u32(x_smem);
-      bool ok = true;
+      bool ok = (n_smem == 0 || mbar_wait(&sh->w2_full, 0, ctl)) && (nt == n_smem || mbar_wait(&sh->w2t_full, 0, ctl));
       for (int k = 0; k < M && ok; ++k) {
         if (!mbar_wait(&sh->x_full, (uint32_t)k & 1u, ctl)) break;
         for (int tt = 0; tt < nt; ++tt) {
           const int64_t i = (int64_t)k * nt + tt;
-          const int w = (int)(i % p.w2_slots);
-          const int abuf = (int)(i & 1);
-          if (!mbar_wait(&sh->w2_full[w], (uint32_t)(i / p.w2_slots) & 1u, ctl) ||
-              !mbar_wait(&sh->acc_empty[abuf], ((uint32_t)(i >> 1) & 1u) ^ 1u, ctl)) {
+          const int abuf = (int)(i % NG);
+          if (!mbar_wait(&sh->acc_empty[abuf], ((uint32_t)(i / NG) & 1u) ^ 1u, ctl)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
           const uint32_t d_tmem = tmem_base + (uint32_t)(abuf * BB);
+          if (tt < n_smem) {
 #pragma unroll
-          for (int ka = 0; ka < KA; ++ka) {
+            for (int kk = 0; kk < KA * kAtomK / 16; ++kk) {
+              const uint64_t ad = sw128_kmajor_desc(w2_addr + (uint32_t)(tt * KA + (kk >> 2)) * kW2AtomBytes +
+                                                    (kk & 3) * 32);
+              const uint64_t bd = sw128_kmajor_desc(x_addr + (kk >> 2) * atom_x + (kk & 3) * 32);
+              umma_bf16_ss(d_tmem, ad, bd, idesc, kk != 0);
+            }
+          } else {
+            const uint32_t a_tmem = tmem_base + acc_cols + (uint32_t)((tt - n_smem) * kTileCols);
 #pragma unroll
-            for (int kk = 0; kk < kAtomK / 16; ++kk) {
-              const uint64_t ad = sw128_kmajor_desc(w2_addr + (uint32_t)(w * KA + ka) * kW2AtomBytes + kk * 32);
-              const uint64_t bd = sw128_kmajor_desc(x_addr + ka * atom_x + kk * 32);
-              umma_bf16_ss(d_tmem, ad, bd, idesc, (ka | kk) != 0);
+            for (int kk = 0; kk < KA * kAtomK / 16; ++kk) {
+              const uint64_t bd = sw128_kmajor_desc(x_addr + (kk >> 2) * atom_x + (kk & 3) * 32);
+              umma_bf16_ts(d_tmem, a_tmem + kk * 8, bd, idesc, kk != 0);
             }
           }
-          umma_commit(&sh->w2_empty[w]);
           umma_commit(&sh->acc_full[abuf]);
         }
         if (ok) umma_commit(&sh->x_empty);
@@ -328,27 +357,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(&sh->drain);
       mbar_wait(&sh->drain, 0, drain_ctl);
     }
-  } else {
+  } else if ((warp - 4) / 4 < NG) {
     // -------------------------------------------------- epilogue ----
-    // Group g takes the tiles whose item index k * nt + tt has parity g, and
-    // uses TMEM accumulator g. Thread (quarter q, lane) owns vocabulary id
-    // 32q + lane of the tile (its TMEM lane) and every batch column b.
+    // Group g takes the tiles whose item index k * nt + tt is g modulo the
+    // group count, with TMEM accumulator g. Thread (quarter q, lane) owns
+    // vocabulary id 32q + lane of the tile (its TMEM lane) and every batch
+    // column b.
     const int g = (warp - 4) >> 2;
     const int et = threadIdx.x - 128 - 128 * g;  // 0..127 within the group
-    const int t256 = threadIdx.x - 128;          // 0..255 across both groups
+    const int te = threadIdx.x - 128;            // 0..NG*128-1 across the groups
     const int q = warp & 3;
     const int row = 32 * q + lane;
-    const uint32_t gbar = 1 + g, allbar = 3;
-    const int groups = (B + 31) >> 5;
-    unsigned long long* my_red = red + (size_t)(g * 4 + q) * BB;
+    const uint32_t gbar = 1 + g, allbar = 1 + kMaxGroups;
+    const uint32_t all_n = (uint32_t)NG * 128u;
+    const int chunks = (B + 15) >> 4;  // 16 batch columns per chunk
+    Key* my_red = red + (size_t)(g * 4 + q) * BB;
+    const uint32_t vbase = (uint32_t)t_begin * kBV;
+
+    if (g == 0 && nt > n_smem) {
+      // W2 tiles beyond the shared-memory share go to TMEM once: thread `row`
+      // writes W2[v] (rank bf16, two per column) into its own lane.
+      const uint32_t lane_base = tmem_base + ((uint32_t)(32 * q) << 16) + acc_cols;
+      for (int j = 0; j < nt - n_smem; ++j) {
+        const int64_t v = (int64_t)(t_begin + n_smem + j) * kBV + row;
+        const uint4* src = reinterpret_cast<const uint4*>(p.w2 + (v < p.vocab ? v : 0) * p.rank);
+#pragma unroll
+        for (int c = 0; c < KA; ++c) {
+          uint32_t w[32];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint4 x = v < p.vocab ? ld_nc_v4(src + c * 8 + i) : make_uint4(0u, 0u, 0u, 0u);
+            w[4 * i + 0] = x.x;
+            w[4 * i + 1] = x.y;
+            w[4 * i + 2] = x.z;
+            w[4 * i + 3] = x.w;
+          }
+          __syncwarp();
+          tmem_st_32x32b_x32(lane_base + (uint32_t)(j * kTileCols + c * 32), w);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->w2t_full);
+      __syncwarp();
+    }
+
     bool ok = true;
     for (int k = 0; k < M; ++k) {
-      for (int gg = 0; gg < groups; ++gg)
-        if (32 * gg + lane < BB) my_red[32 * gg + lane] = 0ull;
-      for (int tt = ((k * nt) & 1) == g ? 0 : 1; tt < nt && ok; tt += 2) {
+      for (int b = lane; b < BB; b += 32) my_red[b] = 0;
+      const int first = (g - (int)(((int64_t)k * nt) % NG) + NG) % NG;
+      for (int tt = first; tt < nt && ok; tt += NG) {
         const int64_t i = (int64_t)k * nt + tt;
         const int s = (int)(i % p.u_slots);
-        const uint32_t acc_par = (uint32_t)(i >> 1) & 1u;
+        const uint32_t acc_par = (uint32_t)(i / NG) & 1u;
         const uint32_t u_par = (uint32_t)(i / p.u_slots) & 1u;
         bool w_ok = true;
         if (et == 0) w_ok = mbar_wait(&sh->acc_full[g], acc_par, ctl) && mbar_wait(&sh->u_full[s], u_par, ctl);
@@ -369,33 +431,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         __nv_bfloat16* slot = reinterpret_cast<__nv_bfloat16*>(u_smem + (size_t)s * p.u_slot_bytes) + row;
         const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(g * BB);
 #pragma unroll 1
-        for (int gg = 0; gg < groups; ++gg) {
-          uint32_t d[32];
-          tmem_ld_32x32b_x16(tb + 32 * gg, *reinterpret_cast<uint32_t(*)[16]>(&d[0]));
-          if (32 * gg + 16 < BB) tmem_ld_32x32b_x16(tb + 32 * gg + 16, *reinterpret_cast<uint32_t(*)[16]>(&d[16]));
+        for (int ch = 0; ch < chunks; ++ch) {
+          uint32_t d[16];
+          tmem_ld_32x32b_x16(tb + 16 * ch, d);
           tmem_ld_wait();
-          const int nb = B - 32 * gg < 32 ? B - 32 * gg : 32;  // batch columns of this group
-          __nv_bfloat16* col = slot + (size_t)(32 * gg) * kBV;
+          const int nb = B - 16 * ch < 16 ? B - 16 * ch : 16;  // batch columns of this chunk
+          __nv_bfloat16* col = slot + (size_t)(16 * ch) * kBV;
           // All loads first, then the arithmetic, then all stores: the loads
           // of one thread are independent, so they overlap instead of each
           // waiting out the shared-memory latency of the previous element.
-          __nv_bfloat16 c[32];
+          __nv_bfloat16 c[16];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) c[j] = j < nb ? col[j * kBV] : __float2bfloat16_rn(0.0f);
+          for (int j = 0; j < 16; ++j) c[j] = j < nb ? col[j * kBV] : __float2bfloat16_rn(0.0f);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) c[j] = __float2bfloat16_rn(__bfloat162float(c[j]) + __uint_as_float(d[j]));
+          for (int j = 0; j < 16; ++j) c[j] = __float2bfloat16_rn(__bfloat162float(c[j]) + __uint_as_float(d[j]));
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
+          for (int j = 0; j < 16; ++j)
             if (j < nb) col[j * kBV] = c[j];
-          unsigned long long key[32];
+          Key key[16];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            float score = __bfloat162float(c[j]);
-            if (!GREEDY) score = score / p.temperature + noise_for(p.seed, (uint32_t)(32 * gg + j), (uint32_t)k, v);
-            key[j] = (j < nb && valid) ? pack_key(score, v) : 0ull;
+          for (int j = 0; j < 16; ++j) {
+            if constexpr (GREEDY) {
+              key[j] = (j < nb && valid) ? greedy_key(__bfloat16_as_ushort(c[j]), v - vbase) : 0u;
+            } else {
+              const float score =
+                  __bfloat162float(c[j]) / p.temperature + noise_for(p.seed, (uint32_t)(16 * ch + j), (uint32_t)k, v);
+              key[j] = (j < nb && valid) ? pack_key(score, v) : 0ull;
+            }
           }
-          const unsigned long long best = transpose_max32(key, lane);
-          if (32 * gg + lane < BB) my_red[32 * gg + lane] = umax64(my_red[32 * gg + lane], best);
+          const Key best = transpose_max16(key, lane);
+          const int b = 16 * ch + (lane >> 1);
+          if ((lane & 1) == 0 && b < BB && best > my_red[b]) my_red[b] = best;
         }
         tc_fence_before_sync();
         __syncwarp();
@@ -411,19 +477,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       }
-      // Both groups agree to go on (an abort anywhere ends every step here).
-      if (!barrier_and(ok, allbar, 256)) break;
-      // Merge the eight partial maxima of each b, then this CTA's into the
-      // global keys.
-      for (int b = t256; b < B; b += 256) {
-        unsigned long long m = 0ull;
-#pragma unroll
-        for (int r = 0; r < 8; ++r) m = umax64(m, red[(size_t)r * BB + b]);
-        atomicMax(&p.keys[(size_t)k * B + b], m);
+      // The groups agree to go on (an abort anywhere ends every step here).
+      if (!barrier_and(ok, allbar, all_n)) break;
+      // Merge the partial maxima of each b, then this CTA's into the global
+      // keys (64-bit: orderable score, complement of the global id).
+      for (int b = te; b < B; b += (int)all_n) {
+        Key m = 0;
+        for (int r = 0; r < NG * 4; ++r) m = red[(size_t)r * BB + b] > m ? red[(size_t)r * BB + b] : m;
+        unsigned long long gk;
+        if constexpr (GREEDY) {
+          const uint32_t vid = vbase + (0xFFFFu - (m & 0xFFFFu));
+          gk = m ? ((unsigned long long)(m >> 16) << 32) | (unsigned long long)(0xFFFFFFFFu - vid) : 0ull;
+        } else {
+          gk = m;
+        }
+        atomicMax(&p.keys[(size_t)k * B + b], gk);
       }
       __threadfence();
-      named_barrier_sync(allbar, 256);
-      if (t256 == 0) {
+      named_barrier_sync(allbar, all_n);
+      if (te == 0) {
         const bool skip = (p.debug_flags & DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL) && blockIdx.x == 0 && k == 0;
         int last = 0;
         if (!skip) {
@@ -434,10 +506,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         sh->is_last = last;
       }
       __syncwarp();
-      named_barrier_sync(allbar, 256);
+      named_barrier_sync(allbar, all_n);
       if (k == M - 1 && sh->is_last) {
         __threadfence();
-        for (int b = t256; b < B; b += 256)
+        for (int b = te; b < B; b += (int)all_n)
           p.tokens[(size_t)b * M + (M - 1)] = (int64_t)key_token(ld_relaxed_gpu(&p.keys[(size_t)(M - 1) * B + b]));
       }
     }
@@ -450,11 +522,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  if (warp == 1) tmem_dealloc(tmem_base, p.tmem_cols);
+  if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
 }
 
 struct SampleConfig {
-  int w2_slots, u_slots;
+  int smem_tiles, u_slots, groups;
   uint32_t u_slot_bytes, x_bytes;
   size_t smem_bytes;
   bool ok;
@@ -462,40 +534,45 @@ struct SampleConfig {
 
 size_t align1024(size_t x) { return (x + 1023) & ~size_t(1023); }
 
-SampleConfig plan(int ka, int batch, int batch_pad) {
+int batch_pad_of(int64_t batch) { return (int)(((batch + 15) / 16) * 16); }
+
+// Shared memory: [W2 tiles][X][U ring][partial maxima][tail]; tensor memory:
+// [accumulators: groups x batch_pad][W2 tiles that did not fit in smem].
+// Prefer four epilogue groups, then more U slots, and give the rest of shared
+// memory to W2; the remaining tiles must fit in tensor memory.
+SampleConfig plan(int ka, int batch, int batch_pad, int tiles_per_cta) {
   SampleConfig c{};
   c.u_slot_bytes = (uint32_t)align1024((size_t)batch * kBV * 2);
   c.x_bytes = (uint32_t)((size_t)ka * batch_pad * 128);
-  const size_t fixed = 1024 + (size_t)c.x_bytes + 8 * (size_t)batch_pad * 8 + sizeof(SampleTail) + 64;
-  const size_t w2_slot = (size_t)ka * kW2AtomBytes;
-  for (int w = 4; w >= 1; --w) {
+  const size_t tile_bytes = (size_t)ka * kW2AtomBytes;
+  const size_t fixed =
+      1024 + (size_t)c.x_bytes + align8((size_t)kMaxGroups * 4 * batch_pad * 8) + sizeof(SampleTail) + 64;
+  if (tiles_per_cta > kMaxTiles || fixed > kSmemLimit) return c;
+  for (int groups = kMaxGroups; groups >= 1; groups >>= 1) {
     for (int u = 8; u >= 2; --u) {
-      const size_t total = fixed + w * w2_slot + u * (size_t)c.u_slot_bytes;
-      if (total <= kSmemLimit) {
-        c.w2_slots = w;
-        c.u_slots = u;
-        c.smem_bytes = total;
-        c.ok = true;
-        return c;
-      }
+      const size_t used = fixed + (size_t)u * c.u_slot_bytes;
+      if (used > kSmemLimit) continue;
+      int smem_tiles = (int)((kSmemLimit - used) / tile_bytes);
+      if (smem_tiles > tiles_per_cta) smem_tiles = tiles_per_cta;
+      const int tmem_tiles = tiles_per_cta - smem_tiles;
+      if ((uint32_t)(groups * batch_pad + tmem_tiles * ka * 32) > kTmemCols) continue;
+      c.smem_tiles = smem_tiles;
+      c.u_slots = u;
+      c.groups = groups;
+      c.smem_bytes = used + (size_t)smem_tiles * tile_bytes;
+      c.ok = true;
+      return c;
     }
   }
-  c.ok = false;
   return c;
-}
-
-int batch_pad_of(int64_t batch) { return (int)(((batch + 15) / 16) * 16); }
-
-uint32_t tmem_cols_for(int batch_pad) {
-  uint32_t need = 2u * (uint32_t)batch_pad, cols = 32;
-  while (cols < need) cols <<= 1;
-  return cols;
 }
 
 template <int KA, bool GREEDY>
 cudaError_t launch_ka(const TcSampleArgs& a, int num_sms, cudaStream_t stream) {
   const int BB = batch_pad_of(a.batch);
-  const SampleConfig c = plan(KA, (int)a.batch, BB);
+  const int tiles = (int)((a.vocab + kBV - 1) / kBV);
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  const SampleConfig c = plan(KA, (int)a.batch, BB, (tiles + grid - 1) / grid);
   if (!c.ok) return cudaErrorInvalidValue;
   SampleMaps maps;
   const uint32_t wbox[2] = {64, 128};
@@ -519,7 +596,7 @@ cudaError_t launch_ka(const TcSampleArgs& a, int num_sms, cudaStream_t stream) {
 
   SampleParams p{};
   p.first_prev = a.first_prev;
-  p.w1 = static_cast<const __nv_bfloat16*>(a.w1);
+  p.w2 = static_cast<const __nv_bfloat16*>(a.w2);
   p.tokens = a.tokens;
   p.keys = a.keys;
   p.barrier = a.barrier;
@@ -529,22 +606,20 @@ cudaError_t launch_ka(const TcSampleArgs& a, int num_sms, cudaStream_t stream) {
   p.steps = (int32_t)a.steps;
   p.rank = a.rank;
   p.vocab = a.vocab;
-  p.vocab_tiles = (int32_t)((a.vocab + kBV - 1) / kBV);
-  p.w2_slots = c.w2_slots;
+  p.vocab_tiles = tiles;
+  p.smem_tiles = c.smem_tiles;
   p.u_slots = c.u_slots;
   p.u_slot_bytes = c.u_slot_bytes;
   p.x_bytes = c.x_bytes;
   p.temperature = a.temperature;
-  p.greedy = a.greedy;
   p.seed = a.seed;
   p.wait_limit_ns = a.wait_limit_ns;
   p.debug_flags = a.debug_flags;
-  p.tmem_cols = tmem_cols_for(BB);
+  p.groups = c.groups;
 
   cudaError_t e = cudaFuncSetAttribute(tc_sample_kernel<KA, GREEDY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)c.smem_bytes);
   if (e != cudaSuccess) return e;
-  const int grid = p.vocab_tiles < num_sms ? p.vocab_tiles : num_sms;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(kThreads);
@@ -573,12 +648,19 @@ cudaError_t launch_mode(const TcSampleArgs& a, int num_sms, cudaStream_t s) {
 
 }  // namespace
 
-bool tc_sample_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype) {
+bool tc_sample_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype,
+                         int num_sms) {
   if (logits_dtype != DSPARK_DTYPE_BF16 || weight_dtype != DSPARK_DTYPE_BF16) return false;
   if (vocab % 8 != 0 || rank % 64 != 0 || rank < 64 || rank > 256) return false;
   if (batch < 1 || batch > kMaxBatch) return false;
-  if (vocab >= (1ll << 31) - kBV) return false;
-  return plan(rank / 64, (int)batch, batch_pad_of(batch)).ok;
+  if (vocab >= (1ll << 31) - kBV || num_sms < 1) return false;
+  const int64_t tiles = (vocab + kBV - 1) / kBV;
+  const int64_t grid = tiles < num_sms ? tiles : num_sms;
+  const int64_t per_cta = (tiles + grid - 1) / grid;
+  // The greedy key keeps a CTA-local vocabulary index in 16 bits, and W2 must
+  // fit on chip (shared plus tensor memory) for the whole launch.
+  if (per_cta * kBV > 65536) return false;
+  return plan(rank / 64, (int)batch, batch_pad_of(batch), (int)per_cta).ok;
 }
 
 cudaError_t launch_tc_sample(const TcSampleArgs& a, int num_sms, cudaStream_t s) {
