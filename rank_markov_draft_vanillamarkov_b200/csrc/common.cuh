@@ -78,10 +78,14 @@ __device__ __forceinline__ uint32_t philox_word(const Philox4& p, uint32_t i) {
 }
 
 // u = (2 * (w >> 9) + 1) * 2^-24 lies strictly inside (0, 1) and is exact in
-// binary32. The Gumbel variate is g = -log(-log u).
+// binary32. The Gumbel variate is g = -log(e) with e = -log u. e must be
+// accurate relative to itself (for u near 1 it is as small as 6e-8, and those
+// draws are the likely winners), so it uses the full-accuracy logf; the outer
+// log only needs a small absolute error (e lies in [6e-8, 16.7]), for which
+// the hardware approximation suffices.
 __device__ __forceinline__ float gumbel_from_word(uint32_t w) {
   const float u = (float)(2u * (w >> 9) + 1u) * 5.9604644775390625e-08f;  // 2^-24
-  return -logf(-logf(u));
+  return -__logf(-logf(u));
 }
 
 __device__ __forceinline__ float noise_for(uint64_t seed, uint32_t b, uint32_t k, uint32_t v) {

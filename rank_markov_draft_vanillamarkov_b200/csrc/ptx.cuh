@@ -229,6 +229,11 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
          ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
 }
 
+// The descriptor of an operand `bytes` further on: the start-address field
+// holds address >> 4 in its low bits, so stepping is one 64-bit add (valid
+// while the address stays inside shared memory, which it always does).
+__device__ __forceinline__ uint64_t desc_advance(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
+
 // Instruction descriptor of kind::f16 with bf16 A and B (both K-major) and an
 // fp32 accumulator: D format (bits 4-5) = 1, A format (7-9) = 1, B format
 // (10-12) = 1, N >> 3 (17-22), M >> 4 (24-28).

@@ -26,7 +26,8 @@
 //   - merges its maxima into a per-(k, b) 64-bit key with atomicMax, then
 //     passes a grid barrier (bounded wait) after which every CTA decodes x_k.
 //
-// Warp roles (640 threads): 0 W2 loader, 1 MMA issuer + TMEM owner, 2 U
+// Warp roles (640 threads): 0 W2 loader then tile store warp, 1 MMA issuer +
+// TMEM owner, 2 U
 // producer, 3 W1 gather + grid barrier, 4-19 up to four epilogue groups of
 // four warps that take tiles round-robin (one TMEM accumulator each; thread =
 // vocab id). Several groups in flight hide the shared-memory and shuffle
@@ -62,6 +63,7 @@ struct __align__(64) SampleMaps {
 
 struct SampleParams {
   const int64_t* first_prev;
+  const __nv_bfloat16* w1;
   const __nv_bfloat16* w2;
   int64_t* tokens;
   unsigned long long* keys;
@@ -82,14 +84,13 @@ struct SampleParams {
 
 struct SampleTail {
   uint64_t w2_full, w2t_full;
-  uint64_t u_full[kMaxStages], u_empty[kMaxStages];
+  uint64_t u_full[kMaxStages], u_empty[kMaxStages], tile_ready[kMaxStages];
   uint64_t x_full, x_empty;
   uint64_t acc_full[kMaxGroups], acc_empty[kMaxGroups];
   uint64_t drain;
   int32_t xid[kMaxBatch];
   uint32_t tmem_base;
   int abort_flag;
-  int is_last;
 };
 
 __device__ __forceinline__ bool barrier_and(bool v, uint32_t id, uint32_t n) {
@@ -108,6 +109,18 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   return v;
 }
 
+__device__ __forceinline__ void red_max_gpu(unsigned long long* p, unsigned long long v) {
+  asm volatile("red.relaxed.gpu.global.max.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ void red_add_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p) : "memory");
+}
+
 __device__ __forceinline__ unsigned long long ld_relaxed_gpu(const unsigned long long* p) {
   unsigned long long v;
   asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
@@ -120,27 +133,24 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   return r;
 }
 
-// Sixteen keys per lane in; lanes 2i and 2i+1 leave with the warp-wide
-// maximum of key index i. Each of the first four rounds halves the keys a lane
-// holds: it keeps the half whose index bit matches a lane bit and trades the
-// other half with the lane across that bit; the last round merges lane pairs.
-template <typename K>
-__device__ __forceinline__ K transpose_max16(K (&k)[16], int lane) {
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int o = 16 >> r;    // lane bit of this round
-    const int half = 8 >> r;  // keys kept
-    const bool upper = (lane & o) != 0;
-#pragma unroll
-    for (int j = 0; j < half; ++j) {
-      const K send = upper ? k[j] : k[j + half];
-      const K keep = upper ? k[j + half] : k[j];
-      const K recv = __shfl_xor_sync(0xffffffffu, send, o);
-      k[j] = keep > recv ? keep : recv;
-    }
-  }
-  const K other = __shfl_xor_sync(0xffffffffu, k[0], 1);
-  return k[0] > other ? k[0] : other;
+// A warp-uniform bounded wait: lane 0 waits, the warp follows its verdict, and
+// the other lanes then observe the (already completed) phase themselves.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl, int lane) {
+  bool ok = lane == 0 ? mbar_wait(bar, parity, ctl) : true;
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  if (ok && lane != 0) mbar_wait(bar, parity, ctl);
+  return ok;
+}
+
+// Warp-wide maximum of a key: one redux for 32-bit keys; for 64-bit keys the
+// maximum high word first, then the maximum low word among the lanes that
+// hold it (the same result as a 64-bit maximum).
+__device__ __forceinline__ uint32_t warp_max_key(uint32_t k) { return __reduce_max_sync(0xffffffffu, k); }
+__device__ __forceinline__ unsigned long long warp_max_key(unsigned long long k) {
+  const uint32_t hi = (uint32_t)(k >> 32);
+  const uint32_t hmax = __reduce_max_sync(0xffffffffu, hi);
+  const uint32_t lmax = __reduce_max_sync(0xffffffffu, hi == hmax ? (uint32_t)k : 0u);
+  return ((unsigned long long)hmax << 32) | lmax;
 }
 
 // Greedy key of a bf16 corrected logit: its bits mapped to an unsigned order
@@ -151,8 +161,33 @@ __device__ __forceinline__ uint32_t greedy_key(uint32_t bits, uint32_t local_id)
   bits &= 0xFFFFu;
   if ((bits & 0x7FFFu) > 0x7F80u) bits = 0x7FC0u;
   if (bits == 0x8000u) bits = 0u;
-  const uint32_t ord = (bits & 0x8000u) ? (~bits & 0xFFFFu) : (bits | 0x8000u);
+  const uint32_t ord = bits ^ (0x8000u | ((bits >> 15) * 0x7FFFu));  // negative: all bits flipped
   return (ord << 16) | (0xFFFFu - local_id);
+}
+
+// Lane 0 waits (bounded) until the grid-barrier counter reaches `target`; the
+// warp follows its verdict.
+__device__ __forceinline__ bool grid_wait(const uint32_t* counter, uint32_t target, const WaitCtl& ctl, int lane) {
+  bool ok = true;
+  if (lane == 0) {
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_gpu(counter) < target) {
+      if (*ctl.abort_flag) {
+        ok = false;
+        break;
+      }
+      if (globaltimer_ns() - t0 > ctl.limit_ns) {
+        *ctl.abort_flag = 1;
+        atomicOr(ctl.status, DSPARK_STATUS_TIMEOUT);
+        ok = false;
+        break;
+      }
+      __nanosleep(32);
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  __syncwarp();
+  return ok;
 }
 
 // GREEDY selects at compile time: the greedy instance carries no noise code.
@@ -191,6 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < p.u_slots; ++i) {
       mbar_init(&sh->u_full[i], 1);
       mbar_init(&sh->u_empty[i], 1);
+      mbar_init(&sh->tile_ready[i], 4);  // the four warps of the tile's epilogue group
     }
     mbar_init(&sh->x_full, 1);
     mbar_init(&sh->x_empty, 1);
@@ -200,7 +236,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&sh->drain, 1);
     sh->abort_flag = 0;
-    sh->is_last = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -217,17 +252,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   const WaitCtl drain_ctl{&never, p.status, p.wait_limit_ns};
 
   if (warp == 0) {
-    // ---------------------------------------- W2 into shared memory ----
-    if (lane == 0 && n_smem > 0) {
-      prefetch_tensormap(&maps.w2);
-      const uint64_t pol = policy_evict_first();
-      mbar_arrive_expect_tx(&sh->w2_full, (uint32_t)(n_smem * KA * kW2AtomBytes));
-      for (int tt = 0; tt < n_smem; ++tt)
+    // ------------------------- W2 into shared memory, then store warp ----
+    if (lane == 0) {
+      if (n_smem > 0) {
+        prefetch_tensormap(&maps.w2);
+        const uint64_t pol = policy_evict_first();
+        mbar_arrive_expect_tx(&sh->w2_full, (uint32_t)(n_smem * KA * kW2AtomBytes));
+        for (int tt = 0; tt < n_smem; ++tt)
 #pragma unroll
-        for (int ka = 0; ka < KA; ++ka)
-          tma_load_2d(w2_smem + (size_t)(tt * KA + ka) * kW2AtomBytes, &maps.w2, &sh->w2_full, ka * kAtomK,
-                      (t_begin + tt) * kBV, pol);
-      mbar_wait(&sh->w2_full, 0, drain_ctl);  // the copies are done before this thread may exit
+          for (int ka = 0; ka < KA; ++ka)
+            tma_load_2d(w2_smem + (size_t)(tt * KA + ka) * kW2AtomBytes, &maps.w2, &sh->w2_full, ka * kAtomK,
+                        (t_begin + tt) * kBV, pol);
+      }
+      // TMA-store each finished tile of corrected logits and hand its U slot
+      // back to the producer once the store has read it; one store in flight.
+      int prev_s = -1;
+      for (int64_t i = 0; i < items; ++i) {
+        const int k = (int)(i / nt);
+        const int t = t_begin + (int)(i % nt);
+        const int s = (int)(i % p.u_slots);
+        if (!mbar_wait(&sh->tile_ready[s], (uint32_t)(i / p.u_slots) & 1u, ctl)) break;
+        tma_store_3d(&maps.out, u_smem + (size_t)s * p.u_slot_bytes, t * kBV, k, 0);
+        bulk_commit_group();
+        if (prev_s >= 0) {
+          bulk_wait_group_read<1>();
+          mbar_arrive(&sh->u_empty[prev_s]);
+        }
+        prev_s = s;
+      }
+      bulk_wait_group<0>();
+      if (n_smem > 0) mbar_wait(&sh->w2_full, 0, drain_ctl);  // the W2 copies are done before exit
     }
   } else if (warp == 2) {
     // ------------------------------------------------ U producer ----
@@ -261,30 +315,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       xe_ok = __shfl_sync(0xffffffffu, xe_ok ? 1 : 0, 0) != 0;
       if (!xe_ok) break;
       if (lane != 0) mbar_wait(&sh->x_empty, xe_par, ctl);  // already complete
-      if (k > 0) {
-        // Every CTA has merged its step k-1 maxima once the counter reaches k * G.
-        bool ok = true;
-        if (lane == 0) {
-          const uint32_t target = (uint32_t)k * (uint32_t)G;
-          const uint64_t t0 = globaltimer_ns();
-          while (ld_acquire_gpu(p.barrier) < target) {
-            if (*ctl.abort_flag) {
-              ok = false;
-              break;
-            }
-            if (globaltimer_ns() - t0 > p.wait_limit_ns) {
-              *ctl.abort_flag = 1;
-              atomicOr(p.status, DSPARK_STATUS_TIMEOUT);
-              ok = false;
-              break;
-            }
-            __nanosleep(32);
-          }
-        }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        __syncwarp();
-        if (!ok) break;
-      }
+      // Every CTA has merged its step k-1 maxima once the counter reaches k * G.
+      if (k > 0 && !grid_wait(p.barrier, (uint32_t)k * (uint32_t)G, ctl, lane)) break;
       bool bad = false;
       // Row of W1 for each batch column; padding columns and invalid ids use
       // row `vocab`, outside the tensor, which the gather reads as zeros.
@@ -315,13 +347,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     sh->xid[4 * j + 1], sh->xid[4 * j + 2], sh->xid[4 * j + 3], pol_w1);
       }
       __syncwarp();
+      if (k == M - 1 && blockIdx.x == 0) {
+        // The last step's tokens, once every CTA has merged its maxima.
+        if (grid_wait(p.barrier, (uint32_t)M * (uint32_t)G, ctl, lane))
+          for (int b = lane; b < B; b += 32)
+            p.tokens[(size_t)b * M + (M - 1)] = (int64_t)key_token(ld_relaxed_gpu(&p.keys[(size_t)(M - 1) * B + b]));
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------- MMA issuer ----
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(kBV, (uint32_t)BB);
-      const uint32_t w2_addr = smem_u32(w2_smem);
-      const uint32_t x_addr = smem_u32(x_smem);
+      // Descriptors are built once; each K-step only advances the start address.
+      const uint64_t w2_desc = sw128_kmajor_desc(smem_u32(w2_smem));
+      const uint64_t x_desc = sw128_kmajor_desc(smem_u32(x_smem));
       bool ok = (n_smem == 0 || mbar_wait(&sh->w2_full, 0, ctl)) && (nt == n_smem || mbar_wait(&sh->w2t_full, 0, ctl));
       for (int k = 0; k < M && ok; ++k) {
         if (!mbar_wait(&sh->x_full, (uint32_t)k & 1u, ctl)) break;
@@ -335,20 +374,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after_sync();
           const uint32_t d_tmem = tmem_base + (uint32_t)(abuf * BB);
           if (tt < n_smem) {
+            const uint64_t a0 = desc_advance(w2_desc, (uint32_t)(tt * KA) * kW2AtomBytes);
 #pragma unroll
-            for (int kk = 0; kk < KA * kAtomK / 16; ++kk) {
-              const uint64_t ad = sw128_kmajor_desc(w2_addr + (uint32_t)(tt * KA + (kk >> 2)) * kW2AtomBytes +
-                                                    (kk & 3) * 32);
-              const uint64_t bd = sw128_kmajor_desc(x_addr + (kk >> 2) * atom_x + (kk & 3) * 32);
-              umma_bf16_ss(d_tmem, ad, bd, idesc, kk != 0);
-            }
+            for (int kk = 0; kk < KA * kAtomK / 16; ++kk)
+              umma_bf16_ss(d_tmem, desc_advance(a0, (kk >> 2) * kW2AtomBytes + (kk & 3) * 32),
+                           desc_advance(x_desc, (kk >> 2) * atom_x + (kk & 3) * 32), idesc, kk != 0);
           } else {
             const uint32_t a_tmem = tmem_base + acc_cols + (uint32_t)((tt - n_smem) * kTileCols);
 #pragma unroll
-            for (int kk = 0; kk < KA * kAtomK / 16; ++kk) {
-              const uint64_t bd = sw128_kmajor_desc(x_addr + (kk >> 2) * atom_x + (kk & 3) * 32);
-              umma_bf16_ts(d_tmem, a_tmem + kk * 8, bd, idesc, kk != 0);
-            }
+            for (int kk = 0; kk < KA * kAtomK / 16; ++kk)
+              umma_bf16_ts(d_tmem, a_tmem + kk * 8, desc_advance(x_desc, (kk >> 2) * atom_x + (kk & 3) * 32), idesc,
+                           kk != 0);
           }
           umma_commit(&sh->acc_full[abuf]);
         }
@@ -364,15 +400,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // vocabulary id 32q + lane of the tile (its TMEM lane) and every batch
     // column b.
     const int g = (warp - 4) >> 2;
-    const int et = threadIdx.x - 128 - 128 * g;  // 0..127 within the group
     const int te = threadIdx.x - 128;            // 0..NG*128-1 across the groups
     const int q = warp & 3;
     const int row = 32 * q + lane;
-    const uint32_t gbar = 1 + g, allbar = 1 + kMaxGroups;
+    const uint32_t allbar = 1;  // all epilogue warps (named barrier 0 is __syncthreads)
     const uint32_t all_n = (uint32_t)NG * 128u;
     const int chunks = (B + 15) >> 4;  // 16 batch columns per chunk
     Key* my_red = red + (size_t)(g * 4 + q) * BB;
     const uint32_t vbase = (uint32_t)t_begin * kBV;
+    const float inv_t = GREEDY ? 0.0f : 1.0f / p.temperature;
 
     if (g == 0 && nt > n_smem) {
       // W2 tiles beyond the shared-memory share go to TMEM once: thread `row`
@@ -412,18 +448,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = (int)(i % p.u_slots);
         const uint32_t acc_par = (uint32_t)(i / NG) & 1u;
         const uint32_t u_par = (uint32_t)(i / p.u_slots) & 1u;
-        bool w_ok = true;
-        if (et == 0) w_ok = mbar_wait(&sh->acc_full[g], acc_par, ctl) && mbar_wait(&sh->u_full[s], u_par, ctl);
-        __syncwarp();
-        if (!barrier_and(w_ok, gbar, 128)) {
+        if (!warp_wait(&sh->acc_full[g], acc_par, ctl, lane) || !warp_wait(&sh->u_full[s], u_par, ctl, lane)) {
           ok = false;
           break;
         }
-        if (et != 0) {
-          mbar_wait(&sh->acc_full[g], acc_par, ctl);
-          mbar_wait(&sh->u_full[s], u_par, ctl);
-        }
-        __syncwarp();  // tcgen05.ld below is warp-aligned
         tc_fence_after_sync();
         const int t = t_begin + tt;
         const uint32_t v = (uint32_t)(t * kBV + row);
@@ -449,38 +477,66 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 16; ++j)
             if (j < nb) col[j * kBV] = c[j];
           Key key[16];
+          if constexpr (GREEDY) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if constexpr (GREEDY) {
+            for (int j = 0; j < 16; ++j)
               key[j] = (j < nb && valid) ? greedy_key(__bfloat16_as_ushort(c[j]), v - vbase) : 0u;
-            } else {
-              const float score =
-                  __bfloat162float(c[j]) / p.temperature + noise_for(p.seed, (uint32_t)(16 * ch + j), (uint32_t)k, v);
-              key[j] = (j < nb && valid) ? pack_key(score, v) : 0ull;
+          } else {
+            // One Philox call (counter v>>2, k, b, 0) serves the four ids of a
+            // lane quad. Lane i of the quad computes the calls of columns
+            // 4jj + i; a 4 x 4 transpose inside the quad then hands each lane
+            // the word of its own id (v & 3) for all four columns.
+            const uint32_t qi = (uint32_t)lane & 3u;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              const Philox4 r = philox4x32_10(v >> 2, (uint32_t)k, (uint32_t)(16 * ch + 4 * jj) + qi, 0u,
+                                              (uint32_t)p.seed, (uint32_t)(p.seed >> 32));
+              uint32_t a0 = r.x, a1 = r.y, a2 = r.z, a3 = r.w;
+              {  // exchange across lane bit 0
+                const bool odd = (qi & 1u) != 0;
+                const uint32_t s0 = odd ? a0 : a1, s1 = odd ? a2 : a3;
+                const uint32_t r0 = __shfl_xor_sync(0xffffffffu, s0, 1), r1 = __shfl_xor_sync(0xffffffffu, s1, 1);
+                if (odd) { a0 = r0; a2 = r1; } else { a1 = r0; a3 = r1; }
+              }
+              {  // exchange across lane bit 1
+                const bool hi = (qi & 2u) != 0;
+                const uint32_t s0 = hi ? a0 : a2, s1 = hi ? a1 : a3;
+                const uint32_t r0 = __shfl_xor_sync(0xffffffffu, s0, 2), r1 = __shfl_xor_sync(0xffffffffu, s1, 2);
+                if (hi) { a0 = r0; a1 = r1; } else { a2 = r0; a3 = r1; }
+              }
+              const uint32_t wv[4] = {a0, a1, a2, a3};  // words of columns 4jj + 0..3 for this lane's id
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int j = 4 * jj + i;
+                const float score = __bfloat162float(c[j]) * inv_t + gumbel_from_word(wv[i]);
+                key[j] = (j < nb && valid) ? pack_key(score, v) : 0ull;
+              }
             }
           }
-          const Key best = transpose_max16(key, lane);
-          const int b = 16 * ch + (lane >> 1);
-          if ((lane & 1) == 0 && b < BB && best > my_red[b]) my_red[b] = best;
+          // Column j's warp-wide maximum ends up in lane j.
+          Key mine = 0;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const Key m = warp_max_key(key[j]);
+            mine = lane == j ? m : mine;
+          }
+          if (lane < nb && mine > my_red[16 * ch + lane]) my_red[16 * ch + lane] = mine;
         }
         tc_fence_before_sync();
+        fence_proxy_async_smem();  // this thread's stores become visible to the TMA store
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sh->acc_empty[g]);
-        __syncwarp();
-        fence_proxy_async_smem();
-        named_barrier_sync(gbar, 128);
-        if (et == 0) {
-          tma_store_3d(&maps.out, slot - row, t * kBV, k, 0);
-          bulk_commit_group();
-          bulk_wait_group_read<0>();  // the slot may be refilled once the store has read it
-          mbar_arrive(&sh->u_empty[s]);
+        if (lane == 0) {
+          mbar_arrive(&sh->acc_empty[g]);
+          mbar_arrive(&sh->tile_ready[s]);
         }
         __syncwarp();
       }
       // The groups agree to go on (an abort anywhere ends every step here).
       if (!barrier_and(ok, allbar, all_n)) break;
       // Merge the partial maxima of each b, then this CTA's into the global
-      // keys (64-bit: orderable score, complement of the global id).
+      // keys (64-bit: orderable score, complement of the global id). The W1
+      // row of this CTA's candidate is prefetched into L2: if it wins, the
+      // next step's gather finds it there.
       for (int b = te; b < B; b += (int)all_n) {
         Key m = 0;
         for (int r = 0; r < NG * 4; ++r) m = red[(size_t)r * BB + b] > m ? red[(size_t)r * BB + b] : m;
@@ -491,29 +547,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           gk = m;
         }
-        atomicMax(&p.keys[(size_t)k * B + b], gk);
+        if (gk) {
+          red_max_gpu(&p.keys[(size_t)k * B + b], gk);
+          if (k + 1 < M) prefetch_l2(p.w1 + (size_t)key_token(gk) * p.rank);
+        }
+        __threadfence();  // the merge is performed before this CTA's arrival below
       }
-      __threadfence();
       named_barrier_sync(allbar, all_n);
       if (te == 0) {
         const bool skip = (p.debug_flags & DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL) && blockIdx.x == 0 && k == 0;
-        int last = 0;
-        if (!skip) {
-          __threadfence();
-          const uint32_t ticket = atomicAdd(p.barrier, 1u);
-          last = (k == M - 1) && ticket == (uint32_t)M * (uint32_t)G - 1u;
-        }
-        sh->is_last = last;
-      }
-      __syncwarp();
-      named_barrier_sync(allbar, all_n);
-      if (k == M - 1 && sh->is_last) {
-        __threadfence();
-        for (int b = te; b < B; b += (int)all_n)
-          p.tokens[(size_t)b * M + (M - 1)] = (int64_t)key_token(ld_relaxed_gpu(&p.keys[(size_t)(M - 1) * B + b]));
+        if (!skip) red_add_release_gpu(p.barrier, 1u);
       }
     }
-    if (et == 0) bulk_wait_group<0>();
   }
 
   // Single-lane roles and lane-0 branches leave warps diverged; bar.sync is
@@ -596,6 +641,7 @@ cudaError_t launch_ka(const TcSampleArgs& a, int num_sms, cudaStream_t stream) {
 
   SampleParams p{};
   p.first_prev = a.first_prev;
+  p.w1 = static_cast<const __nv_bfloat16*>(a.w1);
   p.w2 = static_cast<const __nv_bfloat16*>(a.w2);
   p.tokens = a.tokens;
   p.keys = a.keys;
