@@ -106,6 +106,42 @@ int dspark_markov_sample_block(const void* base_logits, const int64_t* first_pre
                                int32_t logits_dtype, int32_t weight_dtype, void* stream);
 
 /*
+ * dspark_markov_sample_block without any device allocation. The pages define
+ * no counterpart: this is a library entry for callers that must not allocate
+ * device memory during the call -- a serving loop whose memory is fully
+ * reserved up front, a caller holding its own allocator's lock, or code on a
+ * path where an allocation (or the implicit synchronisation cudaFree does)
+ * would stall other streams. dspark_markov_sample_block keeps its reduction
+ * keys and barrier counter in a workspace that it allocates on first use and
+ * regrows for larger calls; this entry uses a fixed scratch in the library's
+ * static device memory instead.
+ *
+ *   Arguments, layouts, ownership and results are those of
+ *   dspark_markov_sample_block; the tensor-core sampler is always used (the
+ *   process-wide DSPARK_ALGO_* choice does not apply).
+ *   batch * proposal_len must not exceed DSPARK_NOALLOC_MAX_KEYS (8192, for
+ *   64 KiB of scratch); larger calls return DSPARK_ERR_UNSUPPORTED, as do the
+ *   shapes, dtypes and alignments the tensor-core sampler does not take
+ *   (bf16 logits and weights, rank a multiple of 64 in [64, 256], vocab a
+ *   multiple of 8, batch <= 256, 16-byte aligned buffers).
+ *   The first call on each device looks up the scratch's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture. Every call clears the scratch's counter and
+ *   keys with an asynchronous memset on `stream` and then launches one kernel.
+ *   Device-side errors go to a status word in the scratch, which
+ *   dspark_markov_get_status folds into the value it returns.
+ *   There is one scratch per device: calls that overlap on one device (other
+ *   streams or threads without ordering between them) race on it and give
+ *   wrong results. Issue them on one stream or order them with events.
+ */
+#define DSPARK_NOALLOC_MAX_KEYS 8192
+int dspark_markov_sample_block_noalloc(const void* base_logits, const int64_t* first_prev_token_ids, int64_t batch,
+                                       int64_t proposal_len, int64_t vocab, const void* w1, const void* w2,
+                                       int32_t rank, float temperature, uint64_t seed, int64_t* sampled_tokens,
+                                       void* corrected_logits, int32_t logits_dtype, int32_t weight_dtype,
+                                       void* stream);
+
+/*
  * Synchronise `stream`, then read and clear the current device's status word
  * (DSPARK_STATUS_* bits) into *status_out. Not part of the hot path.
  */

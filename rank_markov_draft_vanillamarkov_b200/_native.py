@@ -29,12 +29,16 @@ DSPARK_ALGO_TENSOR_CORE = 2
 
 DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL = 1
 
+DSPARK_NOALLOC_MAX_KEYS = 8192
+
 # Every symbol include/dspark_markov.h declares, with its ctypes signature.
 _vp, _i64, _i32, _u32, _u64, _f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_uint32, ctypes.c_uint64, ctypes.c_float
 SIGNATURES = {
     "dspark_markov_apply_block_logits": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i64, _vp, _vp, _i32, _i32, _i32, _vp]),
     "dspark_markov_sample_block": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _i32, _f32, _u64, _vp, _vp,
                                                   _i32, _i32, _vp]),
+    "dspark_markov_sample_block_noalloc": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _i32, _f32, _u64,
+                                                          _vp, _vp, _i32, _i32, _vp]),
     "dspark_markov_get_status": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_int32)]),
     "dspark_markov_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "dspark_markov_set_algo": (_i32, [_i32]),

@@ -90,6 +90,56 @@ unsigned char* workspace(DeviceState* d, size_t bytes) {
   return d->workspace;
 }
 
+// ---------------------------------------------------------------------------
+// Fixed scratch of dspark_markov_sample_block_noalloc, for callers that cannot
+// allocate device memory during the call. It lives in this module's static
+// device memory, so it exists from module load on and nothing is allocated.
+// Layout: status word at 0, grid-barrier counter at 256, then
+// DSPARK_NOALLOC_MAX_KEYS packed step maxima.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocStatusOff = 0;
+constexpr size_t kNoAllocCounterOff = 256;
+constexpr size_t kNoAllocKeysOff = 512;
+constexpr size_t kNoAllocBytes = kNoAllocKeysOff + (size_t)DSPARK_NOALLOC_MAX_KEYS * sizeof(unsigned long long);
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+struct NoAllocState {
+  bool ready = false;
+  int num_sms = 0;
+  unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch
+};
+
+NoAllocState g_noalloc[kMaxDevices];
+
+// Set-up of the current device, done once by its first call: the SM count and
+// the scratch's device address. Neither call allocates.
+int noalloc_state(NoAllocState** out, bool* fresh) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSPARK_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  NoAllocState& n = g_noalloc[dev];
+  if (!n.ready) {
+    void* ptr = nullptr;
+    if (cudaDeviceGetAttribute(&n.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return DSPARK_ERR_CUDA;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return DSPARK_ERR_CUDA;
+    n.scratch = static_cast<unsigned char*>(ptr);
+    n.ready = true;
+    *fresh = true;
+  }
+  *out = &n;
+  return DSPARK_OK;
+}
+
+// The scratch of the current device when its set-up has run, else null.
+unsigned char* noalloc_scratch_if_ready() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  return g_noalloc[dev].ready ? g_noalloc[dev].scratch : nullptr;
+}
+
 bool dtype_ok(int32_t t) { return t == DSPARK_DTYPE_FP32 || t == DSPARK_DTYPE_BF16; }
 
 int cuda_code(cudaError_t e) { return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA; }
@@ -236,6 +286,65 @@ int dspark_markov_sample_block(const void* base_logits, const int64_t* first_pre
   return DSPARK_OK;
 }
 
+int dspark_markov_sample_block_noalloc(const void* base_logits, const int64_t* first_prev_token_ids, int64_t batch,
+                                       int64_t proposal_len, int64_t vocab, const void* w1, const void* w2,
+                                       int32_t rank, float temperature, uint64_t seed, int64_t* sampled_tokens,
+                                       void* corrected_logits, int32_t logits_dtype, int32_t weight_dtype,
+                                       void* stream) {
+  t_last_algo = 0;
+  if (batch < 0 || proposal_len < 0 || vocab <= 0 || rank <= 0 || !dtype_ok(logits_dtype) ||
+      !dtype_ok(weight_dtype) || std::isnan(temperature))
+    return DSPARK_ERR_INVALID_ARG;
+  if (batch == 0 || proposal_len == 0) return DSPARK_OK;
+  if (!base_logits || !first_prev_token_ids || !w1 || !w2 || !sampled_tokens || !corrected_logits)
+    return DSPARK_ERR_INVALID_ARG;
+  if (batch * proposal_len > DSPARK_NOALLOC_MAX_KEYS) return DSPARK_ERR_UNSUPPORTED;
+  {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(base_logits), c0 = reinterpret_cast<uintptr_t>(corrected_logits);
+    const uintptr_t n = (uintptr_t)(batch * proposal_len * vocab) * (logits_dtype == DSPARK_DTYPE_BF16 ? 2 : 4);
+    if (a0 < c0 + n && c0 < a0 + n) return DSPARK_ERR_INVALID_ARG;
+  }
+  NoAllocState* st = nullptr;
+  bool fresh = false;
+  const int err = noalloc_state(&st, &fresh);
+  if (err != DSPARK_OK) return err;
+  const bool tc_ok = tc_sample_supported(batch, vocab, rank, logits_dtype, weight_dtype, st->num_sms) &&
+                     (reinterpret_cast<uintptr_t>(base_logits) % 16 == 0) &&
+                     (reinterpret_cast<uintptr_t>(corrected_logits) % 16 == 0) &&
+                     (reinterpret_cast<uintptr_t>(w2) % 16 == 0) && (reinterpret_cast<uintptr_t>(w1) % 16 == 0);
+  if (!tc_ok) return DSPARK_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (fresh && cudaMemsetAsync(st->scratch + kNoAllocStatusOff, 0, sizeof(uint32_t), s) != cudaSuccess)
+    return DSPARK_ERR_CUDA;
+  // The barrier counter and the step maxima start at zero; the status word
+  // keeps its bits until dspark_markov_get_status reads it.
+  const size_t keys_bytes = (size_t)batch * (size_t)proposal_len * sizeof(unsigned long long);
+  if (cudaMemsetAsync(st->scratch + kNoAllocCounterOff, 0, kNoAllocKeysOff - kNoAllocCounterOff + keys_bytes, s) !=
+      cudaSuccess)
+    return DSPARK_ERR_CUDA;
+  TcSampleArgs a{};
+  a.base = base_logits;
+  a.first_prev = first_prev_token_ids;
+  a.batch = batch;
+  a.steps = proposal_len;
+  a.vocab = vocab;
+  a.w1 = w1;
+  a.w2 = w2;
+  a.rank = rank;
+  a.temperature = temperature;
+  a.greedy = !(temperature >= 1e-5f) ? 1 : 0;
+  a.seed = seed;
+  a.tokens = sampled_tokens;
+  a.corrected = corrected_logits;
+  a.keys = reinterpret_cast<unsigned long long*>(st->scratch + kNoAllocKeysOff);
+  a.barrier = reinterpret_cast<uint32_t*>(st->scratch + kNoAllocCounterOff);
+  a.status = reinterpret_cast<uint32_t*>(st->scratch + kNoAllocStatusOff);
+  a.wait_limit_ns = g_wait_limit_ns.load();
+  a.debug_flags = g_debug_flags.load();
+  t_last_algo = 2;
+  return cuda_code(launch_tc_sample(a, st->num_sms, s));
+}
+
 int dspark_markov_get_status(void* stream, int32_t* status_out) {
   if (!status_out) return DSPARK_ERR_INVALID_ARG;
   int err = DSPARK_OK;
@@ -246,6 +355,14 @@ int dspark_markov_get_status(void* stream, int32_t* status_out) {
   uint32_t v = 0;
   if (cudaMemcpy(&v, d->status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return DSPARK_ERR_CUDA;
   if (cudaMemset(d->status, 0, sizeof(uint32_t)) != cudaSuccess) return DSPARK_ERR_CUDA;
+  if (unsigned char* sc = noalloc_scratch_if_ready()) {
+    // The no-allocation sampler reports into its own scratch's status word.
+    uint32_t w = 0;
+    if (cudaMemcpy(&w, sc + kNoAllocStatusOff, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemset(sc + kNoAllocStatusOff, 0, sizeof(uint32_t)) != cudaSuccess)
+      return DSPARK_ERR_CUDA;
+    v |= w;
+  }
   *status_out = (int32_t)v;
   return DSPARK_OK;
 }

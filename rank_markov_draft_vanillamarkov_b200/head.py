@@ -148,6 +148,44 @@ class VanillaMarkov:
         N.check(code, "dspark_markov_sample_block")
         return tokens, corrected
 
+    def sample_block_tokens_noalloc(self, base_logits: torch.Tensor, *, first_prev_token_ids: torch.Tensor,
+                                    out_tokens: torch.Tensor, out_logits: torch.Tensor,
+                                    temperature: Optional[float] = 0.0, seed: int = 0) -> None:
+        """``sample_block_tokens`` for callers that must not allocate device
+        memory during the call (memory reserved up front, an allocator lock
+        held): the outputs are caller-provided, ``first_prev_token_ids`` must
+        already be contiguous int64 on the head's device, and the library's
+        fixed static scratch replaces its growable workspace. Requires
+        B * M <= 8192 and a shape the tensor-core sampler takes. Calls that
+        overlap on one device race on the shared scratch; the first call on a
+        device should come before any stream capture."""
+        if base_logits.dim() != 3:
+            raise ValueError("base_logits must be (B, M, V)")
+        batch, m, vocab = base_logits.shape
+        if vocab != self.vocab_size:
+            raise ValueError(f"vocab mismatch: logits {vocab} vs head {self.vocab_size}")
+        if base_logits.dtype not in _DT:
+            raise ValueError("logits must be float32 or bfloat16")
+        prev = first_prev_token_ids
+        if prev.dtype != torch.int64 or not prev.is_contiguous() or tuple(prev.shape) != (batch,):
+            raise ValueError("first_prev_token_ids must be contiguous int64 (B,)")
+        if tuple(out_tokens.shape) != (batch, m) or out_tokens.dtype != torch.int64 or not out_tokens.is_contiguous():
+            raise ValueError("out_tokens must be contiguous int64 (B, M)")
+        if out_logits.shape != base_logits.shape or out_logits.dtype != base_logits.dtype or \
+                not out_logits.is_contiguous():
+            raise ValueError("out_logits must be contiguous with the shape and dtype of base_logits")
+        for t, name in ((base_logits, "base_logits"), (prev, "first_prev_token_ids"), (out_tokens, "out_tokens"),
+                        (out_logits, "out_logits")):
+            _check_cuda(t, name, self.device)
+        t = 0.0 if temperature is None else float(temperature)
+        if math.isnan(t):
+            raise ValueError("temperature is NaN")
+        code = self._lib.dspark_markov_sample_block_noalloc(
+            base_logits.data_ptr(), prev.data_ptr(), batch, m, vocab, self.markov_w1.data_ptr(),
+            self.markov_w2.data_ptr(), self.markov_rank, t, seed & 0xFFFFFFFFFFFFFFFF, out_tokens.data_ptr(),
+            out_logits.data_ptr(), _DT[base_logits.dtype], _DT[self.weight_dtype], _stream_ptr(self.device))
+        N.check(code, "dspark_markov_sample_block_noalloc")
+
 
 def build_markov_head(w1: Optional[torch.Tensor], w2: Optional[torch.Tensor], markov_rank: int,
                       head_type: str = "vanilla") -> Optional[VanillaMarkov]:

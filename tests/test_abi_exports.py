@@ -37,7 +37,7 @@ def test_header_constants_match_binding():
     for name in ["DSPARK_OK", "DSPARK_ERR_INVALID_ARG", "DSPARK_ERR_UNSUPPORTED", "DSPARK_ERR_CUDA",
                  "DSPARK_STATUS_TOKEN_RANGE", "DSPARK_STATUS_TIMEOUT", "DSPARK_DTYPE_FP32", "DSPARK_DTYPE_BF16",
                  "DSPARK_ALGO_AUTO", "DSPARK_ALGO_GENERIC", "DSPARK_ALGO_TENSOR_CORE",
-                 "DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL"]:
+                 "DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL", "DSPARK_NOALLOC_MAX_KEYS"]:
         m = re.search(rf"#define {name} (\d+)", text)
         assert m, name
         assert int(m.group(1)) == getattr(N, name), name
@@ -62,6 +62,13 @@ def test_argument_errors_are_caught_on_the_host(lib):
     # corrected logits overlapping the base logits are refused
     q = ctypes.c_void_p(4096)
     assert sp(q, p, 2, 5, 128, p, p, 16, 0.0, 0, p, q, 1, 1, None) == N.DSPARK_ERR_INVALID_ARG
+    # the no-allocation sampler: same argument checks, and its scratch bound
+    na = lib.dspark_markov_sample_block_noalloc
+    assert na(p, p, 2, 5, 128, p, p, 16, nan, 0, p, p, 1, 1, None) == N.DSPARK_ERR_INVALID_ARG
+    assert na(None, None, 2, 0, 128, None, None, 16, 0.0, 0, None, None, 1, 1, None) == N.DSPARK_OK
+    assert na(q, p, 2, 5, 128, p, p, 16, 0.0, 0, p, q, 1, 1, None) == N.DSPARK_ERR_INVALID_ARG
+    assert na(p, p, 256, 33, 128, p, p, 64, 0.0, 0, p, ctypes.c_void_p(1 << 40), 1, 1, None) == \
+        N.DSPARK_ERR_UNSUPPORTED
 
 
 def test_host_utilities(lib):
