@@ -78,15 +78,20 @@ __device__ __forceinline__ uint32_t philox_word(const Philox4& p, uint32_t i) {
 }
 
 // u = (2 * (w >> 9) + 1) * 2^-24 lies strictly inside (0, 1) and is exact in
-// binary32. The Gumbel variate is g = -log(e) with e = -log u. e must be
-// accurate relative to itself (for u near 1 it is as small as 6e-8, and those
-// draws are the likely winners), so it uses the full-accuracy logf; the outer
-// log only needs a small absolute error (e lies in [6e-8, 16.7]), for which
-// the hardware approximation suffices.
-__device__ __forceinline__ float gumbel_from_word(uint32_t w) {
-  const float u = (float)(2u * (w >> 9) + 1u) * 5.9604644775390625e-08f;  // 2^-24
-  return -__logf(-logf(u));
+// binary32. It is formed without an integer-to-float conversion: the top 23
+// bits of w as the mantissa of a number in [1, 2) give 1 + m 2^-23, and
+// subtracting 1 - 2^-24 leaves (2m + 1) 2^-24, which is representable, so the
+// subtraction is exact.
+__device__ __forceinline__ float uniform_from_word(uint32_t w) {
+  return __uint_as_float(0x3F800000u | (w >> 9)) - 0.999999940395355224609375f;
 }
+
+// The Gumbel variate is g = -log(e) with e = -log u. e must be accurate
+// relative to itself (for u near 1 it is as small as 6e-8, and those draws are
+// the likely winners), so it uses the full-accuracy logf; the outer log only
+// needs a small absolute error (e lies in [6e-8, 16.7]), for which the
+// hardware approximation suffices.
+__device__ __forceinline__ float gumbel_from_word(uint32_t w) { return -__logf(-logf(uniform_from_word(w))); }
 
 __device__ __forceinline__ float noise_for(uint64_t seed, uint32_t b, uint32_t k, uint32_t v) {
   const Philox4 p = philox4x32_10(v >> 2, k, b, 0u, (uint32_t)seed, (uint32_t)(seed >> 32));

@@ -142,16 +142,8 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return ok;
 }
 
-// Warp-wide maximum of a key: one redux for 32-bit keys; for 64-bit keys the
-// maximum high word first, then the maximum low word among the lanes that
-// hold it (the same result as a 64-bit maximum).
+// Warp-wide maximum of a 32-bit key.
 __device__ __forceinline__ uint32_t warp_max_key(uint32_t k) { return __reduce_max_sync(0xffffffffu, k); }
-__device__ __forceinline__ unsigned long long warp_max_key(unsigned long long k) {
-  const uint32_t hi = (uint32_t)(k >> 32);
-  const uint32_t hmax = __reduce_max_sync(0xffffffffu, hi);
-  const uint32_t lmax = __reduce_max_sync(0xffffffffu, hi == hmax ? (uint32_t)k : 0u);
-  return ((unsigned long long)hmax << 32) | lmax;
-}
 
 // Greedy key of a bf16 corrected logit: its bits mapped to an unsigned order
 // in the high half (NaN made +qNaN, above +inf; -0 made +0) and the
@@ -476,17 +468,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j)
             if (j < nb) col[j * kBV] = c[j];
-          Key key[16];
+          // Column j's warp-wide maximum ends up in lane j.
+          Key mine = 0;
           if constexpr (GREEDY) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              key[j] = (j < nb && valid) ? greedy_key(__bfloat16_as_ushort(c[j]), v - vbase) : 0u;
+            for (int j = 0; j < 16; ++j) {
+              const Key m = warp_max_key((j < nb && valid) ? greedy_key(__bfloat16_as_ushort(c[j]), v - vbase) : 0u);
+              mine = lane == j ? m : mine;
+            }
           } else {
             // One Philox call (counter v>>2, k, b, 0) serves the four ids of a
             // lane quad. Lane i of the quad computes the calls of columns
             // 4jj + i; a 4 x 4 transpose inside the quad then hands each lane
             // the word of its own id (v & 3) for all four columns.
             const uint32_t qi = (uint32_t)lane & 3u;
+            uint32_t o[16];  // order-preserving bits of each column's score (0: no candidate)
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
               const Philox4 r = philox4x32_10(v >> 2, (uint32_t)k, (uint32_t)(16 * ch + 4 * jj) + qi, 0u,
@@ -509,16 +505,21 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int i = 0; i < 4; ++i) {
                 const int j = 4 * jj + i;
                 const float score = __bfloat162float(c[j]) * inv_t + gumbel_from_word(wv[i]);
-                key[j] = (j < nb && valid) ? pack_key(score, v) : 0ull;
+                o[j] = (j < nb && valid) ? orderable_bits(score) : 0u;
               }
             }
-          }
-          // Column j's warp-wide maximum ends up in lane j.
-          Key mine = 0;
+            // Per column: the largest score bits, then the lowest lane (the
+            // lowest id) holding them; the 64-bit key is formed once, in lane j.
+            uint32_t mo = 0u, mw = 0u;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const Key m = warp_max_key(key[j]);
-            mine = lane == j ? m : mine;
+            for (int j = 0; j < 16; ++j) {
+              const uint32_t m = __reduce_max_sync(0xffffffffu, o[j]);
+              const uint32_t w = (uint32_t)(__ffs(__ballot_sync(0xffffffffu, o[j] == m)) - 1);
+              mo = lane == j ? m : mo;
+              mw = lane == j ? w : mw;
+            }
+            const uint32_t vw = (uint32_t)(t * kBV + 32 * q) + mw;
+            mine = mo ? ((Key)mo << 32) | (Key)(0xffffffffu - vw) : (Key)0;
           }
           if (lane < nb && mine > my_red[16 * ch + lane]) my_red[16 * ch + lane] = mine;
         }
