@@ -142,19 +142,24 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return ok;
 }
 
-// Warp-wide maximum of a 32-bit key.
-__device__ __forceinline__ uint32_t warp_max_key(uint32_t k) { return __reduce_max_sync(0xffffffffu, k); }
+// Order-preserving bits of an fp32 value computed by this kernel's own
+// arithmetic, as an unsigned integer: the sign bit is set for non-negative
+// values and every bit is flipped for negative ones. Adding +0 first makes -0
+// into +0 (the two compare equal), and turns any NaN into the canonical
+// positive NaN of the GPU's floating-point unit, which orders above +inf
+// (NaN counts as the largest value). Two ALU operations besides the add.
+__device__ __forceinline__ uint32_t ordered_bits(float x) {
+  const uint32_t b = __float_as_uint(x + 0.0f);
+  return b ^ ((uint32_t)((int32_t)b >> 31) | 0x80000000u);
+}
 
-// Greedy key of a bf16 corrected logit: its bits mapped to an unsigned order
-// in the high half (NaN made +qNaN, above +inf; -0 made +0) and the
-// complement of the CTA-local vocabulary index in the low half, so that the
-// maximum is the largest value and, among equal values, the lowest id.
-__device__ __forceinline__ uint32_t greedy_key(uint32_t bits, uint32_t local_id) {
-  bits &= 0xFFFFu;
-  if ((bits & 0x7FFFu) > 0x7F80u) bits = 0x7FC0u;
-  if (bits == 0x8000u) bits = 0u;
-  const uint32_t ord = bits ^ (0x8000u | ((bits >> 15) * 0x7FFFu));  // negative: all bits flipped
-  return (ord << 16) | (0xFFFFu - local_id);
+// Greedy key of a bf16 corrected logit: its order-preserving bits in the high
+// half and `low` = 0xFFFF - (CTA-local vocabulary index) in the low half, so
+// that the maximum is the largest value and, among equal values, the lowest
+// id. The low half of a bf16 value widened to fp32 is zero, except for the
+// canonical NaN, whose low half the mask clears (so equal NaNs tie too).
+__device__ __forceinline__ uint32_t greedy_key(uint32_t bf16_bits, uint32_t low) {
+  return (ordered_bits(__uint_as_float(bf16_bits << 16)) & 0xFFFF0000u) | low;
 }
 
 // Lane 0 waits (bounded) until the grid-barrier counter reaches `target`; the
@@ -450,31 +455,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool valid = (int64_t)v < p.vocab;
         __nv_bfloat16* slot = reinterpret_cast<__nv_bfloat16*>(u_smem + (size_t)s * p.u_slot_bytes) + row;
         const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(g * BB);
-#pragma unroll 1
-        for (int ch = 0; ch < chunks; ++ch) {
+        // A chunk is 16 batch columns. Full chunks of a tile whose ids are all
+        // in the vocabulary need no per-element validity selects.
+        const bool tile_valid = (int64_t)(t + 1) * kBV <= p.vocab;
+        const uint32_t low = 0xFFFFu - (v - vbase);      // greedy key's low half
+        const uint32_t vwarp = (uint32_t)(t * kBV + 32 * q);  // id of lane 0
+        auto chunk = [&](int ch, auto full_tag) {
+          constexpr bool FULL = decltype(full_tag)::value;
           uint32_t d[16];
           tmem_ld_32x32b_x16(tb + 16 * ch, d);
           tmem_ld_wait();
-          const int nb = B - 16 * ch < 16 ? B - 16 * ch : 16;  // batch columns of this chunk
+          const int nb = FULL ? 16 : (B - 16 * ch < 16 ? B - 16 * ch : 16);  // batch columns of this chunk
           __nv_bfloat16* col = slot + (size_t)(16 * ch) * kBV;
+          Key* red_ch = my_red + 16 * ch;
           // All loads first, then the arithmetic, then all stores: the loads
           // of one thread are independent, so they overlap instead of each
           // waiting out the shared-memory latency of the previous element.
           __nv_bfloat16 c[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) c[j] = j < nb ? col[j * kBV] : __float2bfloat16_rn(0.0f);
+          for (int j = 0; j < 16; ++j) c[j] = (FULL || j < nb) ? col[j * kBV] : __float2bfloat16_rn(0.0f);
 #pragma unroll
           for (int j = 0; j < 16; ++j) c[j] = __float2bfloat16_rn(__bfloat162float(c[j]) + __uint_as_float(d[j]));
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            if (j < nb) col[j * kBV] = c[j];
-          // Column j's warp-wide maximum ends up in lane j.
-          Key mine = 0;
+            if (FULL || j < nb) col[j * kBV] = c[j];
+          // Per column: the warp's maximum key (one redux), merged by lane 0
+          // into this warp's running maxima with a shared-memory atomic.
           if constexpr (GREEDY) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              const Key m = warp_max_key((j < nb && valid) ? greedy_key(__bfloat16_as_ushort(c[j]), v - vbase) : 0u);
-              mine = lane == j ? m : mine;
+              uint32_t kj = greedy_key(__bfloat16_as_ushort(c[j]), low);
+              if (!FULL) kj = (j < nb && valid) ? kj : 0u;
+              const uint32_t m = __reduce_max_sync(0xffffffffu, kj);
+              if (lane == 0 && (FULL || j < nb)) atomicMax(&red_ch[j], m);
             }
           } else {
             // One Philox call (counter v>>2, k, b, 0) serves the four ids of a
@@ -505,11 +518,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int i = 0; i < 4; ++i) {
                 const int j = 4 * jj + i;
                 const float score = __bfloat162float(c[j]) * inv_t + gumbel_from_word(wv[i]);
-                o[j] = (j < nb && valid) ? orderable_bits(score) : 0u;
+                o[j] = ordered_bits(score);
+                if (!FULL) o[j] = (j < nb && valid) ? o[j] : 0u;
               }
             }
-            // Per column: the largest score bits, then the lowest lane (the
-            // lowest id) holding them; the 64-bit key is formed once, in lane j.
+            // Per column: the largest score bits (one redux) and the lowest
+            // lane (lowest id) holding them (a ballot); lane j keeps column j's
+            // pair and forms one 64-bit key.
             uint32_t mo = 0u, mw = 0u;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
@@ -518,11 +533,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               mo = lane == j ? m : mo;
               mw = lane == j ? w : mw;
             }
-            const uint32_t vw = (uint32_t)(t * kBV + 32 * q) + mw;
-            mine = mo ? ((Key)mo << 32) | (Key)(0xffffffffu - vw) : (Key)0;
+            const Key mine = mo ? ((Key)mo << 32) | (Key)(0xffffffffu - (vwarp + mw)) : (Key)0;
+            if (lane < nb && mine > red_ch[lane]) red_ch[lane] = mine;
           }
-          if (lane < nb && mine > my_red[16 * ch + lane]) my_red[16 * ch + lane] = mine;
+        };
+#pragma unroll 1
+        for (int ch = 0; ch < chunks; ++ch) {
+          if (tile_valid && B - 16 * ch >= 16)
+            chunk(ch, std::true_type{});
+          else
+            chunk(ch, std::false_type{});
         }
+        __syncwarp();
         tc_fence_before_sync();
         fence_proxy_async_smem();  // this thread's stores become visible to the TMA store
         __syncwarp();

@@ -219,3 +219,88 @@ def test_barrier_timeout_is_reported_not_hung():
     toks, corr, used, st = _sample(d, TC, 0.0)
     assert st == 0
     _check(d, toks, corr, 0.0, 0)
+
+
+def _edge_rows(vocab: int, m: int):
+    """Base logits (B, M, V) of selection edge cases, with the first NaN, the
+    lowest tied id, etc. spread over lanes, warps, tiles and CTAs."""
+    rows = []
+    # ties at the maximum: far apart (other CTAs) and adjacent (one warp)
+    r = torch.full((vocab,), -1.0)
+    for v in (vocab - 1, 70001 % vocab, 41, 40, 3 + 128 * 5):
+        r[v] = 5.0
+    rows.append(r)
+    # NaN counts as the largest value whatever its sign bit; the first NaN
+    # wins, above +inf (the lowest one here has its sign bit set)
+    r = torch.zeros(vocab)
+    r[7] = float("inf")
+    for v in (100003 % vocab, vocab - 1):
+        r[v] = float("nan")
+    r[500 % vocab] = -torch.tensor(float("nan"))
+    rows.append(r)
+    # -0 and +0 are equal: the lower id wins whichever sign it has
+    r = torch.full((vocab,), -1.0)
+    r[1234 % vocab] = -0.0
+    r[1000 % vocab] = 0.0
+    rows.append(r)
+    r = torch.full((vocab,), -1.0)
+    r[2000 % vocab] = 0.0
+    r[1500 % vocab] = -0.0
+    rows.append(r)
+    # every value -inf: all equal, id 0 wins
+    rows.append(torch.full((vocab,), float("-inf")))
+    # the maximum in the ragged last tile
+    r = torch.full((vocab,), -3.0)
+    r[vocab - 1] = 2.0
+    rows.append(r)
+    # a unique maximum in a middle CTA, negative values elsewhere
+    r = -torch.rand(vocab, generator=torch.Generator().manual_seed(5)) - 0.5
+    r[vocab // 2 + 17] = -0.25
+    rows.append(r)
+    base = torch.stack(rows).unsqueeze(1).repeat(1, m, 1)
+    return base.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("algo", [TC, GEN], ids=["tc", "generic"])
+@pytest.mark.parametrize("vocab", [129280, 1000])
+def test_greedy_ties_nan_signed_zero_and_inf(algo, vocab):
+    """Greedy selection on exact ties, NaN, -0/+0 and all -inf: with W2 = 0
+    every corrected logit is its base logit, so each token is numpy's argmax
+    (first NaN, else the lowest id among equal maxima) of its base row."""
+    m, rank = 3, 64
+    base = _edge_rows(vocab, m)
+    g = torch.Generator().manual_seed(2)
+    w1 = (torch.randn(vocab, rank, generator=g) * 0.1).to(torch.bfloat16)
+    w2 = torch.zeros(vocab, rank, dtype=torch.bfloat16)
+    first = torch.arange(base.shape[0], dtype=torch.long) * 13
+    d = {"w1": w1, "w2": w2, "base": base, "first_prev": first}
+    toks, corr, used, st = _sample(d, algo, 0.0)
+    assert used == (2 if algo == TC else 1) and st == 0
+    want = oracle.select_greedy(f64(base))
+    np.testing.assert_array_equal(toks.cpu().numpy(), want)
+    # the corrected logits are the base logits (-0 + 0 = +0, NaN stays NaN)
+    c, b = f64(corr), f64(base)
+    assert np.array_equal(np.isnan(c), np.isnan(b))
+    ok = ~np.isnan(b)
+    assert np.array_equal(c[ok], b[ok] + 0.0)
+
+
+@pytest.mark.parametrize("algo", [TC, GEN], ids=["tc", "generic"])
+def test_temperature_nan_is_selected_first(algo):
+    """With temperature, a NaN logit gives a NaN score, which counts as the
+    largest: the first NaN id of each row is drawn whatever the noise."""
+    vocab, m, rank = 129280, 2, 64
+    g = torch.Generator().manual_seed(4)
+    base = (torch.randn(3, m, vocab, generator=g) * 2.0)
+    for b, ids in enumerate([(90000, 65), (5,), (129279, 64000)]):
+        for v in ids:
+            base[b, :, v] = float("nan")
+    base[0, :, 65] = -torch.tensor(float("nan"))  # sign bit set: still the largest
+    base = base.to(torch.bfloat16)
+    assert (base[0, 0, 65].view(torch.int16) < 0).item()
+    w1 = (torch.randn(vocab, rank, generator=g) * 0.1).to(torch.bfloat16)
+    w2 = torch.zeros(vocab, rank, dtype=torch.bfloat16)
+    d = {"w1": w1, "w2": w2, "base": base, "first_prev": torch.tensor([1, 2, 3])}
+    toks, corr, used, st = _sample(d, algo, 0.8, seed=7)
+    assert used == (2 if algo == TC else 1) and st == 0
+    np.testing.assert_array_equal(toks.cpu().numpy(), [[65, 65], [5, 5], [64000, 64000]])
