@@ -168,6 +168,15 @@ int dspark_markov_set_debug(uint32_t flags, uint64_t wait_limit_ns);
 /* Which kernel the last call on this thread selected: 0 none, 1 generic, 2 tensor core. */
 int32_t dspark_markov_last_algo(void);
 
+/*
+ * Test hook: out[i] = the Gumbel variate g = -log(-log u) that every sampler
+ * kernel draws for the Philox output word words[i] (u = (2 (w >> 9) + 1) 2^-24),
+ * computed by the same device function. words, out: n caller-owned device
+ * elements. |g - exact| is below about 5e-6 for every word. n == 0 enqueues
+ * nothing; n < 0 or a null buffer with n > 0 is DSPARK_ERR_INVALID_ARG.
+ */
+int dspark_markov_debug_gumbel(const uint32_t* words, float* out, int64_t n, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

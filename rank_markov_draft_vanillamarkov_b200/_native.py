@@ -45,6 +45,7 @@ SIGNATURES = {
     "dspark_markov_launch_count": (_i64, []),
     "dspark_markov_set_debug": (ctypes.c_int, [_u32, _u64]),
     "dspark_markov_last_algo": (_i32, []),
+    "dspark_markov_debug_gumbel": (ctypes.c_int, [_vp, _vp, _i64, _vp]),
 }
 
 _lib = None

@@ -392,4 +392,13 @@ int dspark_markov_set_debug(uint32_t flags, uint64_t wait_limit_ns) {
 
 int32_t dspark_markov_last_algo(void) { return t_last_algo; }
 
+int dspark_markov_debug_gumbel(const uint32_t* words, float* out, int64_t n, void* stream) {
+  if (n < 0 || (n > 0 && (!words || !out))) return DSPARK_ERR_INVALID_ARG;
+  if (n == 0) return DSPARK_OK;
+  int err = DSPARK_OK;
+  DeviceState* d = device_state(&err);
+  if (!d) return err;
+  return cuda_code(launch_gumbel_probe(words, out, n, d->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

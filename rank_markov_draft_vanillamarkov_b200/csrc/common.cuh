@@ -60,13 +60,14 @@ __device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint3
                                                  uint32_t k0, uint32_t k1) {
 #pragma unroll
   for (int i = 0; i < 10; ++i) {
-    const uint32_t lo0 = 0xD2511F53u * c0, hi0 = __umulhi(0xD2511F53u, c0);
-    const uint32_t lo1 = 0xCD9E8D57u * c2, hi1 = __umulhi(0xCD9E8D57u, c2);
-    const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+    // Each multiply is one 32 x 32 -> 64-bit product (high and low words together).
+    const uint64_t p0 = (uint64_t)c0 * 0xD2511F53u;
+    const uint64_t p1 = (uint64_t)c2 * 0xCD9E8D57u;
+    const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0, n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1;
     c0 = n0;
-    c1 = lo1;
+    c1 = (uint32_t)p1;
     c2 = n2;
-    c3 = lo0;
+    c3 = (uint32_t)p0;
     k0 += 0x9E3779B9u;
     k1 += 0xBB67AE85u;
   }
@@ -86,12 +87,27 @@ __device__ __forceinline__ float uniform_from_word(uint32_t w) {
   return __uint_as_float(0x3F800000u | (w >> 9)) - 0.999999940395355224609375f;
 }
 
-// The Gumbel variate is g = -log(e) with e = -log u. e must be accurate
-// relative to itself (for u near 1 it is as small as 6e-8, and those draws are
-// the likely winners), so it uses the full-accuracy logf; the outer log only
-// needs a small absolute error (e lies in [6e-8, 16.7]), for which the
-// hardware approximation suffices.
-__device__ __forceinline__ float gumbel_from_word(uint32_t w) { return -__logf(-logf(uniform_from_word(w))); }
+// e = -ln u for such a u, accurate relative to e itself (e is as small as
+// 6e-8 for u near 1, and those draws are the likely winners). With d = 1 - u,
+// which is exact (u is a multiple of 2^-24 in (0, 1)):
+//   d < 1/16:  the Taylor series -ln(1 - d) = d + d^2/2 + d^3/3 + d^4/4 + d^5/5
+//              + ..., whose remainder is below d^6 / (6 (1 - d)), i.e. under
+//              2e-7 of e;
+//   otherwise: -ln 2 * log2(u) with the hardware log2 approximation, whose
+//              absolute error (about 2^-22 in log2) is under 3e-6 of e >= 0.0645.
+__device__ __forceinline__ float neg_log_uniform(float u) {
+  const float d = 1.0f - u;
+  const float series = d * fmaf(d, fmaf(d, fmaf(d, fmaf(d, 0.2f, 0.25f), 0.333333343f), 0.5f), 1.0f);
+  const float via_log2 = __log2f(u) * -0.693147182f;
+  return d < 0.0625f ? series : via_log2;
+}
+
+// The Gumbel variate g = -ln(e), e = -ln u. The outer log needs only a small
+// absolute error (e lies in [6e-8, 16.7]), which the hardware log2 gives:
+// |g - exact| stays below about 5e-6 over all 2^23 possible u.
+__device__ __forceinline__ float gumbel_from_word(uint32_t w) {
+  return __log2f(neg_log_uniform(uniform_from_word(w))) * -0.693147182f;
+}
 
 __device__ __forceinline__ float noise_for(uint64_t seed, uint32_t b, uint32_t k, uint32_t v) {
   const Philox4 p = philox4x32_10(v >> 2, k, b, 0u, (uint32_t)seed, (uint32_t)(seed >> 32));

@@ -112,6 +112,23 @@ cudaError_t launch_generic_apply(const GenericApplyArgs& a, int logits_dtype, in
   return launch_apply_t<__nv_bfloat16, float>(a, s);
 }
 
+namespace {
+// Test hook: the Gumbel variate every sampler kernel draws for each word.
+__global__ void gumbel_probe_kernel(const uint32_t* __restrict__ words, float* __restrict__ out, int64_t n) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = gumbel_from_word(words[i]);
+}
+}  // namespace
+
+cudaError_t launch_gumbel_probe(const uint32_t* words, float* out, int64_t n, int num_sms, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t blocks = (n + 255) / 256;
+  const int grid = (int)(blocks < 8ll * num_sms ? blocks : 8ll * num_sms);
+  gumbel_probe_kernel<<<grid, 256, 0, s>>>(words, out, n);
+  note_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_generic_select(const GenericSelectArgs& a, int logits_dtype, cudaStream_t s) {
   if (a.batch == 0) return cudaSuccess;
   if (a.batch > 0x7fffffffll) return cudaErrorInvalidConfiguration;

@@ -37,6 +37,7 @@ struct GenericSelectArgs {
 
 cudaError_t launch_generic_apply(const GenericApplyArgs& a, int logits_dtype, int weight_dtype, cudaStream_t s);
 cudaError_t launch_generic_select(const GenericSelectArgs& a, int logits_dtype, cudaStream_t s);
+cudaError_t launch_gumbel_probe(const uint32_t* words, float* out, int64_t n, int num_sms, cudaStream_t s);
 
 // ----------------------------------------------------------- tensor core --
 // Teacher-forced apply on tcgen05: bf16 logits, bf16 weights,

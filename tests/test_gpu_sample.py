@@ -304,3 +304,26 @@ def test_temperature_nan_is_selected_first(algo):
     toks, corr, used, st = _sample(d, algo, 0.8, seed=7)
     assert used == (2 if algo == TC else 1) and st == 0
     np.testing.assert_array_equal(toks.cpu().numpy(), [[65, 65], [5, 5], [64000, 64000]])
+
+
+def test_gumbel_noise_every_word_within_bound():
+    """Every possible uniform (all 2^23 values of w >> 9) through the device's
+    Gumbel function, against g = -log(-log u) in fp64: the absolute error
+    stays below 1e-5, and the low 9 bits of the word are ignored."""
+    import ctypes
+    lib = N.load()
+    m = torch.arange(1 << 23, dtype=torch.int64)
+    low = torch.randint(0, 512, (1 << 23,), generator=torch.Generator().manual_seed(3))
+    words = ((m << 9) | low).to(torch.int64)
+    words32 = (words - ((words >> 31) << 32)).to(torch.int32).cuda()  # same bits as uint32
+    out = torch.empty(1 << 23, dtype=torch.float32, device="cuda")
+    code = lib.dspark_markov_debug_gumbel(words32.data_ptr(), out.data_ptr(), 1 << 23,
+                                          torch.cuda.current_stream().cuda_stream)
+    assert code == 0
+    torch.cuda.synchronize()
+    u = (2.0 * m.double().numpy() + 1.0) * 2.0 ** -24
+    exact = -np.log(-np.log(u))
+    err = np.abs(out.cpu().double().numpy() - exact)
+    assert err.max() < 1e-5, (err.max(), int(err.argmax()))
+    # u closest to 1 (the largest draws) and closest to 0
+    assert abs(out[-1].item() - exact[-1]) < 1e-5 and abs(out[0].item() - exact[0]) < 1e-5
