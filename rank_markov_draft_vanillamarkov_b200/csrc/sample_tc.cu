@@ -26,11 +26,10 @@
 //   - merges its maxima into a per-(k, b) 64-bit key with atomicMax, then
 //     passes a grid barrier (bounded wait) after which every CTA decodes x_k.
 //
-// Warp roles (640 threads): 0 W2 loader then tile store warp, 1 MMA issuer +
-// TMEM owner, 2 U
-// producer, 3 W1 gather + grid barrier, 4-19 up to four epilogue groups of
-// four warps that take tiles round-robin (one TMEM accumulator each; thread =
-// vocab id). Several groups in flight hide the shared-memory and shuffle
+// Warp roles (640 threads): 0 W2 loader, then the tile store warp; 1 MMA
+// issuer and TMEM owner; 2 U producer; 3 W1 gather and grid barrier; 4-19 up
+// to four epilogue groups of four warps that take tiles round-robin (one TMEM
+// accumulator each; thread = vocabulary id). Several groups in flight hide the
 // latency of the per-element work and even out the tile counts per step.
 #include <type_traits>
 
