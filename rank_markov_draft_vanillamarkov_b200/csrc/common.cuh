@@ -74,6 +74,41 @@ __device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint3
   return Philox4{c0, c1, c2, c3};
 }
 
+// The same generator with its ten round keys given: round_keys[2i] and
+// round_keys[2i+1] are (k0, k1) after i Weyl steps. Kernels whose key is fixed
+// for the launch receive them precomputed (round_keys_for below), as kernel
+// parameters, so the rounds need no key arithmetic.
+struct PhiloxRoundKeys {
+  uint32_t k[20];
+};
+
+__host__ __device__ inline PhiloxRoundKeys round_keys_for(uint64_t seed) {
+  PhiloxRoundKeys r;
+  uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+  for (int i = 0; i < 10; ++i) {
+    r.k[2 * i] = k0;
+    r.k[2 * i + 1] = k1;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return r;
+}
+
+__device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+                                                 const PhiloxRoundKeys& rk) {
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    const uint64_t p0 = (uint64_t)c0 * 0xD2511F53u;
+    const uint64_t p1 = (uint64_t)c2 * 0xCD9E8D57u;
+    const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ rk.k[2 * i], n2 = (uint32_t)(p0 >> 32) ^ c3 ^ rk.k[2 * i + 1];
+    c0 = n0;
+    c1 = (uint32_t)p1;
+    c2 = n2;
+    c3 = (uint32_t)p0;
+  }
+  return Philox4{c0, c1, c2, c3};
+}
+
 __device__ __forceinline__ uint32_t philox_word(const Philox4& p, uint32_t i) {
   return i == 0 ? p.x : i == 1 ? p.y : i == 2 ? p.z : p.w;
 }

@@ -75,7 +75,7 @@ struct SampleParams {
   int32_t u_slots;
   uint32_t u_slot_bytes, x_bytes;  // x_bytes: one step's gathered operand
   float temperature;
-  uint64_t seed;
+  PhiloxRoundKeys round_keys;  // of the launch's seed
   uint64_t wait_limit_ns;
   uint32_t debug_flags;
   int32_t groups;  // epilogue groups in use (<= kMaxGroups)
@@ -498,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
               const Philox4 r = philox4x32_10(v >> 2, (uint32_t)k, (uint32_t)(16 * ch + 4 * jj) + qi, 0u,
-                                              (uint32_t)p.seed, (uint32_t)(p.seed >> 32));
+                                              p.round_keys);
               uint32_t a0 = r.x, a1 = r.y, a2 = r.z, a3 = r.w;
               {  // exchange across lane bit 0
                 const bool odd = (qi & 1u) != 0;
@@ -680,7 +680,7 @@ cudaError_t launch_ka(const TcSampleArgs& a, int num_sms, cudaStream_t stream) {
   p.u_slot_bytes = c.u_slot_bytes;
   p.x_bytes = c.x_bytes;
   p.temperature = a.temperature;
-  p.seed = a.seed;
+  p.round_keys = round_keys_for(a.seed);
   p.wait_limit_ns = a.wait_limit_ns;
   p.debug_flags = a.debug_flags;
   p.groups = c.groups;
