@@ -478,16 +478,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j)
             if (FULL || j < nb) col[j * kBV] = c[j];
-          // Per column: the warp's maximum key (one redux), merged by lane 0
-          // into this warp's running maxima with a shared-memory atomic.
+          // Per column: the warp's maximum key (one redux each, with no
+          // branch between them); lane j keeps column j's, and each lane
+          // merges its column into this warp's running maxima with one
+          // shared-memory atomic.
           if constexpr (GREEDY) {
+            uint32_t mine = 0u;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
+              if (!FULL && j >= nb) break;  // uniform
               uint32_t kj = greedy_key(__bfloat16_as_ushort(c[j]), low);
-              if (!FULL) kj = (j < nb && valid) ? kj : 0u;
+              if (!FULL) kj = valid ? kj : 0u;
               const uint32_t m = __reduce_max_sync(0xffffffffu, kj);
-              if (lane == 0 && (FULL || j < nb)) atomicMax(&red_ch[j], m);
+              mine = lane == j ? m : mine;
             }
+            if (lane < nb) atomicMax(&red_ch[lane], mine);
           } else {
             // One Philox call (counter v>>2, k, b, 0) serves the four ids of a
             // lane quad. Lane i of the quad computes the calls of columns
@@ -496,7 +501,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t qi = (uint32_t)lane & 3u;
             uint32_t o[16];  // order-preserving bits of each column's score (0: no candidate)
 #pragma unroll
+            for (int j = 0; j < 16; ++j) o[j] = 0u;
+#pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
+              if (!FULL && 4 * jj >= nb) break;  // uniform: no batch column left in this chunk
               const Philox4 r = philox4x32_10(v >> 2, (uint32_t)k, (uint32_t)(16 * ch + 4 * jj) + qi, 0u,
                                               p.round_keys);
               uint32_t a0 = r.x, a1 = r.y, a2 = r.z, a3 = r.w;
@@ -527,6 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t mo = 0u, mw = 0u;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
+              if (!FULL && j >= nb) break;  // uniform
               const uint32_t m = __reduce_max_sync(0xffffffffu, o[j]);
               const uint32_t w = (uint32_t)(__ffs(__ballot_sync(0xffffffffu, o[j] == m)) - 1);
               mo = lane == j ? m : mo;
