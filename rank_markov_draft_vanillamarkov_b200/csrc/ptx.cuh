@@ -38,7 +38,7 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 // One try of the phase test. The thread may sleep inside the instruction until
 // the phase completes or about kTryWaitHintNs pass; the short hint bounds the
 // wake-up delay of a waiter on a latency-critical path.
-constexpr uint32_t kTryWaitHintNs = 128;
+constexpr uint32_t kTryWaitHintNs = 1000;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
