@@ -42,12 +42,12 @@ METRIC = "corrected-logit rows/s + achieved HBM GB/s (% roofline); sampled block
 UNIT = "rows/s"
 FALLBACK_HBM_GBS = 6650.0
 PARTS = (("apply", W.APPLY_320), ("greedy", W.greedy(32)), ("temperature", W.TEMPERATURE))
-EXTRA = (("apply_2560", W.APPLY_2560),)
+EXTRA = (("apply_2560", W.APPLY_2560), ("transition", W.TRANSITION_320))
 L2_BYTES = 126 * 1024 * 1024
 
 
 def part_rows(wl: W.Workload) -> int:
-    return wl.rows if wl.mode == "apply" else wl.batch * wl.proposal_len
+    return wl.rows if wl.mode in ("apply", "transition") else wl.batch * wl.proposal_len
 
 
 # --------------------------------------------------------------- helpers --
@@ -160,6 +160,10 @@ class Part:
             dev["head"] = VanillaMarkov(dev["w1"], dev["w2"])
             if wl.mode == "apply":
                 dev["out"] = torch.empty_like(dev["base"])
+            elif wl.mode == "transition":
+                ids = dev["prev_ids"]
+                dev["out"] = torch.empty(*ids.shape, wl.vocab, dtype=torch.bfloat16, device=device)
+                dev["emb"] = torch.empty(*ids.shape, wl.rank, dtype=torch.bfloat16, device=device)
             else:
                 dev["tokens"] = torch.empty(wl.batch, wl.proposal_len, dtype=torch.long, device=device)
                 dev["out"] = torch.empty_like(dev["base"])
@@ -170,6 +174,8 @@ class Part:
         s = self.sets[i % self.nsets]
         if self.wl.mode == "apply":
             s["head"].apply_block_logits(s["base"], token_ids=s["prev_ids"], out=s["out"])
+        elif self.wl.mode == "transition":
+            s["head"].transition_logits(s["prev_ids"], out=s["out"], out_embeddings=s["emb"])
         else:
             s["head"].sample_block_tokens(s["base"], first_prev_token_ids=s["first_prev"],
                                           temperature=self.wl.temperature, seed=self.wl.philox_seed,

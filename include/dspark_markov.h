@@ -79,6 +79,28 @@ int dspark_markov_apply_block_logits(const void* base_logits, void* out, const i
                                      int32_t logits_dtype, int32_t weight_dtype, void* stream);
 
 /*
+ * The transition bias alone, and its conditioning embeddings
+ * (nemo_automodel.components.models.deepseek_v41.dspark,
+ * _DeepseekV41DSparkMarkovHead.forward: "transition logits of shape [..., vocab]
+ * and embeddings"). For each row i with token x = token_ids[i]:
+ *
+ *     transition_out[i, v] = round( sum_j W1[x, j] * W2[v, j] )   (weight_dtype)
+ *     embeddings_out[i, j] = W1[x, j]                             (exact copy)
+ *
+ *   token_ids       [rows] int64 (the pages' [...] leading shape, flattened).
+ *   w1, w2          [vocab, rank] weight_dtype.
+ *   transition_out  [rows, vocab] weight_dtype, written.
+ *   embeddings_out  [rows, rank] weight_dtype, written; may be NULL (not wanted).
+ *
+ * The sum is accumulated in fp32 and rounded once (nearest even). An id outside
+ * [0, vocab) gives a zero bias row and a zero embedding row and sets
+ * DSPARK_STATUS_TOKEN_RANGE. rows == 0 is OK and enqueues nothing.
+ */
+int dspark_markov_transition_logits(const int64_t* token_ids, int64_t rows, int64_t vocab, const void* w1,
+                                    const void* w2, int32_t rank, void* transition_out, void* embeddings_out,
+                                    int32_t weight_dtype, void* stream);
+
+/*
  * Left-to-right sampling of B blocks of M positions
  * (VanillaMarkov.sample_block_tokens and _sample_tokens; markov_head API docs:
  * "sample_block_tokens").

@@ -20,6 +20,7 @@ from .markov import (  # noqa: F401
     sample_tokens,
     select_greedy,
     temperature_scores,
+    transition_logits,
 )
 from .philox import gumbel_noise, noise_words, philox4x32, uniform_from_word  # noqa: F401
 from .rounding import round_to, round_to_bfloat16, round_to_float32, ulp_bfloat16  # noqa: F401

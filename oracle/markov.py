@@ -92,6 +92,19 @@ def exact_block_logits(base_logits, w1, w2, token_ids, hidden_states=None) -> np
     return (base.reshape(-1, vocab) + bias).reshape(base.shape)
 
 
+def transition_logits(w1, w2, token_ids, out_dtype: str):
+    """``_DeepseekV41DSparkMarkovHead.forward`` (page
+    nemo_automodel.components.models.deepseek_v41.dspark): for token ids of
+    any shape (...), the transition bias alone, shape (..., V), rounded once to
+    ``out_dtype`` (the module's dtype), and the conditioning embeddings W1[x],
+    shape (..., r), which are exact copies of W1's rows."""
+    ids = np.asarray(token_ids, dtype=np.int64)
+    emb = get_prev_embeddings(w1, ids.reshape(-1))
+    bias = project_bias(emb, w2)
+    vocab, rank = np.shape(w2)[0], np.shape(w1)[1]
+    return (round_to(out_dtype, bias).reshape(ids.shape + (vocab,)), emb.reshape(ids.shape + (rank,)))
+
+
 def select_greedy(logits: np.ndarray) -> np.ndarray:
     """argmax over the last axis; the lowest index wins among equal maxima and
     NaN counts as the largest value (numpy's argmax has both properties)."""

@@ -194,6 +194,38 @@ int dspark_markov_apply_block_logits(const void* base_logits, void* out, const i
   return cuda_code(launch_generic_apply(a, logits_dtype, weight_dtype, s));
 }
 
+int dspark_markov_transition_logits(const int64_t* token_ids, int64_t rows, int64_t vocab, const void* w1,
+                                    const void* w2, int32_t rank, void* transition_out, void* embeddings_out,
+                                    int32_t weight_dtype, void* stream) {
+  t_last_algo = 0;
+  if (rows < 0 || vocab <= 0 || rank <= 0 || !dtype_ok(weight_dtype)) return DSPARK_ERR_INVALID_ARG;
+  if (rows == 0) return DSPARK_OK;
+  if (!token_ids || !w1 || !w2 || !transition_out) return DSPARK_ERR_INVALID_ARG;
+  int err = DSPARK_OK;
+  DeviceState* d = device_state(&err);
+  if (!d) return err;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int32_t algo = g_algo.load();
+  const bool tc_ok = tc_apply_supported(rows, vocab, rank, weight_dtype, weight_dtype) &&
+                     (reinterpret_cast<uintptr_t>(transition_out) % 16 == 0) &&
+                     (reinterpret_cast<uintptr_t>(w2) % 16 == 0) && (reinterpret_cast<uintptr_t>(w1) % 16 == 0);
+  if (algo == DSPARK_ALGO_TENSOR_CORE && !tc_ok) return DSPARK_ERR_UNSUPPORTED;
+  cudaError_t e;
+  if (tc_ok && algo != DSPARK_ALGO_GENERIC) {
+    TcApplyArgs a{nullptr, transition_out, token_ids, rows, vocab, w1, w2, rank, d->status, g_wait_limit_ns.load()};
+    t_last_algo = 2;
+    e = launch_tc_apply(a, d->num_sms, s);
+  } else {
+    GenericApplyArgs a{nullptr, transition_out, token_ids, rows, vocab, vocab, vocab, 1, w1, w2, rank, d->status};
+    t_last_algo = 1;
+    e = launch_generic_apply(a, weight_dtype, weight_dtype, s);
+  }
+  if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+  if (embeddings_out)
+    e = launch_gather_rows(token_ids, w1, embeddings_out, rows, vocab, rank, weight_dtype, d->status, d->num_sms, s);
+  return cuda_code(e);
+}
+
 int dspark_markov_sample_block(const void* base_logits, const int64_t* first_prev_token_ids, int64_t batch,
                                int64_t proposal_len, int64_t vocab, const void* w1, const void* w2, int32_t rank,
                                float temperature, uint64_t seed, int64_t* sampled_tokens, void* corrected_logits,

@@ -142,7 +142,10 @@ __device__ __forceinline__ void gather_tile_to_tmem(const ApplyParams& p, int m,
   tmem_st_wait();
 }
 
-template <int KA>
+// HAS_BASE false: no U (the bias alone, rounded once): the producer loads no
+// U tile and the epilogue adds zero, using the stage only to assemble the
+// output tile for its TMA store.
+template <int KA, bool HAS_BASE>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_apply_kernel(const __grid_constant__ ApplyMaps maps, const ApplyParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -217,10 +220,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int s = (int)(it % p.u_stages);
         if (!mbar_wait(&sh->u_empty[s], ((uint32_t)(it / p.u_stages) & 1u) ^ 1u, ctl)) break;
-        mbar_arrive_expect_tx(&sh->u_full[s], kUStageBytes);
-        uint8_t* st = u_smem + s * kUStageBytes;
-        tma_load_2d(st, &maps.u, &sh->u_full[s], n * kBN, m * kBM, pol_stream);
-        tma_load_2d(st + kAtomBytes, &maps.u, &sh->u_full[s], n * kBN + 64, m * kBM, pol_stream);
+        if constexpr (HAS_BASE) {
+          mbar_arrive_expect_tx(&sh->u_full[s], kUStageBytes);
+          uint8_t* st = u_smem + s * kUStageBytes;
+          tma_load_2d(st, &maps.u, &sh->u_full[s], n * kBN, m * kBM, pol_stream);
+          tma_load_2d(st + kAtomBytes, &maps.u, &sh->u_full[s], n * kBN + 64, m * kBM, pol_stream);
+        } else {
+          mbar_arrive(&sh->u_full[s]);  // the stage is free for the epilogue
+        }
         ++fills[s];
       }
       // Wait (bounded, even after an abort) for every copy this thread
@@ -328,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint4* ptr = reinterpret_cast<uint4*>(box + ((c ^ (row & 7)) << 4));
-          uint4 x = *ptr;
+          uint4 x = HAS_BASE ? *ptr : make_uint4(0u, 0u, 0u, 0u);
           x.x = add_round_pair(x.x, acc[c * 8 + 0], acc[c * 8 + 1]);
           x.y = add_round_pair(x.y, acc[c * 8 + 2], acc[c * 8 + 3]);
           x.z = add_round_pair(x.z, acc[c * 8 + 4], acc[c * 8 + 5]);
@@ -395,7 +402,9 @@ cudaError_t launch_ka(const TcApplyArgs& a, int num_sms, cudaStream_t stream) {
   const uint64_t ldim[2] = {(uint64_t)a.vocab, (uint64_t)a.rows};
   const uint64_t lstr[1] = {(uint64_t)a.vocab * 2};
   const uint32_t lbox[2] = {64, 128};
-  if (!encode_tensor_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.base, ldim, lstr, lbox,
+  const bool has_base = a.base != nullptr;
+  // Without a base the U map is never read; it is encoded on `out` to stay valid.
+  if (!encode_tensor_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, has_base ? a.base : a.out, ldim, lstr, lbox,
                          CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tensor_map(&maps.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.out, ldim, lstr, lbox,
                          CU_TENSOR_MAP_SWIZZLE_128B))
@@ -421,12 +430,12 @@ cudaError_t launch_ka(const TcApplyArgs& a, int num_sms, cudaStream_t stream) {
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns;
 
-  cudaError_t e = cudaFuncSetAttribute(tc_apply_kernel<KA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)c.smem_bytes);
+  auto kernel = has_base ? tc_apply_kernel<KA, true> : tc_apply_kernel<KA, false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)c.smem_bytes);
   if (e != cudaSuccess) return e;
   const int64_t units = (int64_t)p.row_tiles * p.vocab_tiles;
   const int grid = (int)(units < num_sms ? units : num_sms);
-  tc_apply_kernel<KA><<<grid, kThreads, c.smem_bytes, stream>>>(maps, p);
+  kernel<<<grid, kThreads, c.smem_bytes, stream>>>(maps, p);
   note_launch();
   return cudaGetLastError();
 }

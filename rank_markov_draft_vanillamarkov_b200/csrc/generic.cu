@@ -32,7 +32,8 @@ __global__ void __launch_bounds__(kApplyThreads) generic_apply_kernel(GenericApp
   const TW* w2 = static_cast<const TW*>(a.w2);
   for (int j = threadIdx.x; j < a.rank; j += blockDim.x) latent[j] = valid ? to_f32(w1[id * a.rank + j]) : 0.0f;
   __syncthreads();
-  const TL* in = static_cast<const TL*>(a.base) + row * a.ld_in;
+  // A null base means U = 0: the output is the bias alone.
+  const TL* in = a.base ? static_cast<const TL*>(a.base) + row * a.ld_in : nullptr;
   TL* out = static_cast<TL*>(a.out) + row * a.ld_out;
   const int64_t v0 = (int64_t)blockIdx.y * kApplySlice + threadIdx.x;
 #pragma unroll
@@ -42,7 +43,7 @@ __global__ void __launch_bounds__(kApplyThreads) generic_apply_kernel(GenericApp
     const TW* wrow = w2 + v * a.rank;
     float acc = 0.0f;
     for (int j = 0; j < a.rank; ++j) acc = fmaf(latent[j], to_f32(wrow[j]), acc);
-    out[v] = from_f32<TL>(to_f32(in[v]) + acc);
+    out[v] = from_f32<TL>((in ? to_f32(in[v]) : 0.0f) + acc);
   }
 }
 
@@ -88,7 +89,7 @@ cudaError_t launch_apply_t(const GenericApplyArgs& a, cudaStream_t stream) {
   for (int64_t r0 = 0; r0 < a.rows; r0 += kMaxRows) {
     GenericApplyArgs c = a;
     c.rows = a.rows - r0 < kMaxRows ? a.rows - r0 : kMaxRows;
-    c.base = static_cast<const char*>(a.base) + r0 * a.ld_in * (int64_t)sizeof(TL);
+    c.base = a.base ? static_cast<const char*>(a.base) + r0 * a.ld_in * (int64_t)sizeof(TL) : nullptr;
     c.out = static_cast<char*>(a.out) + r0 * a.ld_out * (int64_t)sizeof(TL);
     c.ids = a.ids + r0 * a.ld_id;
     dim3 grid((unsigned)c.rows, (unsigned)slices);
@@ -113,12 +114,42 @@ cudaError_t launch_generic_apply(const GenericApplyArgs& a, int logits_dtype, in
 }
 
 namespace {
+// Embedding rows W1[ids[i]] into out[i, :] (exact copies); an out-of-range id
+// gives a zero row and sets DSPARK_STATUS_TOKEN_RANGE.
+template <typename TW>
+__global__ void gather_rows_kernel(const int64_t* __restrict__ ids, const TW* __restrict__ w1, TW* __restrict__ out,
+                                   int64_t rows, int64_t vocab, int32_t rank, uint32_t* status) {
+  for (int64_t i = blockIdx.x; i < rows; i += gridDim.x) {
+    const int64_t id = ids[i];
+    const bool valid = id >= 0 && id < vocab;
+    if (!valid && threadIdx.x == 0) report_status(status, DSPARK_STATUS_TOKEN_RANGE);
+    for (int j = threadIdx.x; j < rank; j += blockDim.x)
+      out[i * rank + j] = valid ? w1[id * rank + j] : from_f32<TW>(0.0f);
+  }
+}
+
 // Test hook: the Gumbel variate every sampler kernel draws for each word.
 __global__ void gumbel_probe_kernel(const uint32_t* __restrict__ words, float* __restrict__ out, int64_t n) {
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
     out[i] = gumbel_from_word(words[i]);
 }
 }  // namespace
+
+cudaError_t launch_gather_rows(const int64_t* ids, const void* w1, void* out, int64_t rows, int64_t vocab,
+                               int32_t rank, int weight_dtype, uint32_t* status, int num_sms, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  const int grid = (int)(rows < 16ll * num_sms ? rows : 16ll * num_sms);
+  const int threads = rank < 256 ? ((rank + 31) / 32) * 32 : 256;
+  if (weight_dtype == DSPARK_DTYPE_FP32)
+    gather_rows_kernel<float><<<grid, threads, 0, s>>>(ids, static_cast<const float*>(w1), static_cast<float*>(out),
+                                                        rows, vocab, rank, status);
+  else
+    gather_rows_kernel<__nv_bfloat16><<<grid, threads, 0, s>>>(ids, static_cast<const __nv_bfloat16*>(w1),
+                                                                static_cast<__nv_bfloat16*>(out), rows, vocab, rank,
+                                                                status);
+  note_launch();
+  return cudaGetLastError();
+}
 
 cudaError_t launch_gumbel_probe(const uint32_t* words, float* out, int64_t n, int num_sms, cudaStream_t s) {
   if (n <= 0) return cudaSuccess;

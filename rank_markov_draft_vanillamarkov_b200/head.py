@@ -109,6 +109,40 @@ class VanillaMarkov:
         return self.apply_block_logits(logits.unsqueeze(-2), token_ids=token_ids.unsqueeze(-1),
                                        hidden_states=hidden_states).squeeze(-2)
 
+    def transition_logits(self, token_ids: torch.Tensor, *, with_embeddings: bool = True,
+                          out: Optional[torch.Tensor] = None,
+                          out_embeddings: Optional[torch.Tensor] = None):
+        """The bias alone and its conditioning embeddings, for token ids of
+        any shape (...): returns (transition (..., V), embeddings (..., r) or
+        None), both in the weights' dtype (_DeepseekV41DSparkMarkovHead.forward).
+        The bias is accumulated in fp32 and rounded once."""
+        ids = token_ids if token_ids.dtype == torch.int64 else token_ids.long()
+        ids = ids.contiguous()
+        _check_cuda(ids, "token_ids", self.device)
+        shape = tuple(ids.shape)
+        wdt = self.weight_dtype
+        if out is None:
+            out = torch.empty(*shape, self.vocab_size, dtype=wdt, device=self.device)
+        elif tuple(out.shape) != shape + (self.vocab_size,) or out.dtype != wdt:
+            raise ValueError("out must be (..., V) in the weights' dtype")
+        emb = None
+        if with_embeddings:
+            emb = out_embeddings if out_embeddings is not None else \
+                torch.empty(*shape, self.markov_rank, dtype=wdt, device=self.device)
+            if tuple(emb.shape) != shape + (self.markov_rank,) or emb.dtype != wdt:
+                raise ValueError("out_embeddings must be (..., r) in the weights' dtype")
+            _check_cuda(emb, "out_embeddings", self.device)
+        _check_cuda(out, "out", self.device)
+        rows = ids.numel()
+        if rows == 0:
+            return out, emb
+        code = self._lib.dspark_markov_transition_logits(
+            ids.data_ptr(), rows, self.vocab_size, self.markov_w1.data_ptr(), self.markov_w2.data_ptr(),
+            self.markov_rank, out.data_ptr(), emb.data_ptr() if emb is not None else None, _DT[wdt],
+            _stream_ptr(self.device))
+        N.check(code, "dspark_markov_transition_logits")
+        return out, emb
+
     # ----------------------------------------------------------------- sample
     def sample_block_tokens(self, base_logits: torch.Tensor, *, first_prev_token_ids: torch.Tensor,
                             hidden_states: Optional[torch.Tensor] = None, temperature: Optional[float] = 0.0,

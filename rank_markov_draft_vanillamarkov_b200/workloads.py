@@ -38,8 +38,9 @@ class Workload:
     """One seeded synthetic workload.
 
     ``mode`` is ``"apply"`` (teacher-forced, rows = batch * num_blocks *
-    block_size) or ``"sample"`` (left-to-right, ``batch`` blocks of
-    ``proposal_len`` positions).
+    block_size), ``"transition"`` (the bias alone and the embeddings of the
+    same rows, no base logits) or ``"sample"`` (left-to-right, ``batch``
+    blocks of ``proposal_len`` positions).
     """
 
     name: str
@@ -76,12 +77,15 @@ class Workload:
         if self.mode == "apply":
             r = self.rows
             return 2 * r * self.vocab * lb + self.vocab * self.rank * wb + r * self.rank * wb + r * 8
+        if self.mode == "transition":  # bias out, W2, W1 rows in and embeddings out, ids
+            r = self.rows
+            return r * self.vocab * wb + self.vocab * self.rank * wb + 2 * r * self.rank * wb + r * 8
         r = self.batch * self.proposal_len
         return (2 * r * self.vocab * lb + self.vocab * self.rank * wb + r * self.rank * wb
                 + self.batch * 8 + r * 8)
 
     def flops(self) -> int:
-        r = self.rows if self.mode == "apply" else self.batch * self.proposal_len
+        r = self.rows if self.mode in ("apply", "transition") else self.batch * self.proposal_len
         return 2 * r * self.vocab * self.rank
 
 
@@ -98,6 +102,8 @@ GREEDY = Workload("greedy_m5_v129280_k128", "sample", vocab=129280, rank=128, ba
 TEMPERATURE = Workload("temp0.7_b32_m8_v151936_k64", "sample", vocab=151936, rank=64, batch=32,
                        proposal_len=8, logit_std=1.5, weight_std=0.05, temperature=0.7,
                        philox_seed=1234, data_seed=0)
+TRANSITION_320 = Workload("transition_r320_v129280_k128", "transition", vocab=129280, rank=128, batch=4,
+                          num_blocks=16, block_size=5, weight_std=0.02, prev_dist="zipf1.1", data_seed=0)
 APPLY_2560 = Workload("apply_r2560_v129280_k256_pad20", "apply", vocab=129280, rank=256, batch=8,
                       num_blocks=64, block_size=5, logit_std=2.0, weight_std=0.02,
                       prev_dist="zipf1.1", pad_frac=0.2, data_seed=0)
@@ -147,7 +153,11 @@ def make_inputs(wl: Workload) -> dict:
     g = torch.Generator().manual_seed(wl.data_seed)
     w1, w2 = make_weights(wl, g)
     out = {"w1": w1, "w2": w2}
-    if wl.mode == "apply":
+    if wl.mode == "transition":
+        n = wl.rows
+        ids = zipf_ids(g, n, wl.vocab, 1.1) if wl.prev_dist == "zipf1.1" else uniform_ids(g, n, wl.vocab)
+        out["prev_ids"] = ids.view(wl.batch, wl.num_blocks, wl.block_size)
+    elif wl.mode == "apply":
         shape = (wl.batch, wl.num_blocks, wl.block_size, wl.vocab)
         base = _normal(g, shape, wl.logit_std, wl.logits_dtype)
         n = wl.rows

@@ -71,6 +71,17 @@ def test_argument_errors_are_caught_on_the_host(lib):
         N.DSPARK_ERR_UNSUPPORTED
 
 
+def test_transition_argument_checks(lib):
+    p = ctypes.c_void_p(16)  # never dereferenced
+    tr = lib.dspark_markov_transition_logits
+    assert tr(None, 0, 128, None, None, 16, None, None, 1, None) == N.DSPARK_OK  # empty: nothing enqueued
+    assert tr(p, 4, 128, p, p, 0, p, None, 1, None) == N.DSPARK_ERR_INVALID_ARG  # rank 0
+    assert tr(p, 4, 0, p, p, 16, p, None, 1, None) == N.DSPARK_ERR_INVALID_ARG
+    assert tr(p, -1, 128, p, p, 16, p, None, 1, None) == N.DSPARK_ERR_INVALID_ARG
+    assert tr(p, 4, 128, p, p, 16, p, None, 5, None) == N.DSPARK_ERR_INVALID_ARG  # bad dtype
+    assert tr(p, 4, 128, p, p, 16, None, p, 1, None) == N.DSPARK_ERR_INVALID_ARG  # no output
+
+
 def test_host_utilities(lib):
     assert lib.dspark_markov_strerror(0) == b"ok"
     assert lib.dspark_markov_strerror(N.DSPARK_ERR_UNSUPPORTED).startswith(b"unsupported")

@@ -121,6 +121,25 @@ def test_bigram_special_case_is_a_table_lookup():
         np.testing.assert_array_equal(got[i], table[x])
 
 
+def test_transition_logits_worked_example_and_bigram():
+    """The head's forward (bias alone + embeddings): the hand-worked bias
+    table rows and W1's rows for the worked example, and, with W1 = identity,
+    the bigram table rows and one-hot embeddings, for ids of shape (2, 3)."""
+    d = _worked()
+    w1, w2 = np.array(d["w1"], float), np.array(d["w2"], float)
+    ids = np.array([[2, 0, 1], [1, 1, 0]])
+    tr, emb = oracle.transition_logits(w1, w2, ids, "fp32")
+    assert tr.shape == (2, 3, w2.shape[0]) and emb.shape == (2, 3, w1.shape[1])
+    table = np.array(d["bias_table"]["rows"], float)
+    np.testing.assert_array_equal(tr, table[ids])
+    np.testing.assert_array_equal(emb, w1[ids])
+    bw1, bw2, btable = _bigram_case()
+    bids = np.array([[3, 0, 15], [7, 7, 1]])
+    tr, emb = oracle.transition_logits(bw1, bw2, bids, "bf16")
+    np.testing.assert_array_equal(tr, btable[bids])
+    np.testing.assert_array_equal(emb, np.eye(16)[bids])
+
+
 def test_zero_w2_passes_logits_through_bit_for_bit():
     rng = np.random.default_rng(1)
     base = oracle.round_to_bfloat16(rng.standard_normal((3, 4, 5, 64)) * 3)

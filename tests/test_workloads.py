@@ -46,3 +46,11 @@ def test_greedy_spike_present():
 def test_byte_counts():
     assert W.APPLY_320.bytes_moved() == 2 * 320 * 129280 * 2 + 129280 * 128 * 2 + 320 * 128 * 2 + 320 * 8
     assert W.APPLY_320.flops() == 2 * 320 * 129280 * 128
+
+
+def test_transition_workload():
+    wl = W.TRANSITION_320
+    assert wl.bytes_moved() == 320 * 129280 * 2 + 129280 * 128 * 2 + 2 * 320 * 128 * 2 + 320 * 8
+    d = W.make_inputs(wl)
+    assert tuple(d["prev_ids"].shape) == (4, 16, 5) and "base" not in d
+    assert torch.equal(d["prev_ids"], W.make_inputs(wl)["prev_ids"])
