@@ -89,3 +89,30 @@ def test_highest_index_tie_break_is_caught(monkeypatch):
     monkeypatch.setattr(om, "select_greedy",
                         lambda x: (np.shape(x)[-1] - 1 - np.argmax(np.asarray(x)[..., ::-1], axis=-1)))
     _fails(pins.test_worked_example_greedy_chain)
+
+
+def test_transition_embeddings_from_the_wrong_table_are_caught(monkeypatch):
+    """The head's forward returning rows of W2 (the Linear weight) as the
+    conditioning embeddings instead of rows of W1."""
+    real = om.transition_logits
+
+    def wrong(w1, w2, ids, out_dtype):
+        tr, _ = real(w1, w2, ids, out_dtype)
+        i = np.asarray(ids, np.int64)
+        return tr, np.asarray(w2, float)[i.reshape(-1)][:, :np.shape(w1)[1]].reshape(i.shape + (np.shape(w1)[1],))
+    monkeypatch.setattr(oracle, "transition_logits", wrong)
+    _fails(pins.test_transition_logits_worked_example_and_bigram)
+
+
+def test_transition_with_transposed_lookup_is_caught(monkeypatch):
+    """The bias read from the bigram table's column (W2[x] . W1^T) instead of
+    its row."""
+    def wrong(w1, w2, ids, out_dtype):
+        i = np.asarray(ids, np.int64)
+        flat = i.reshape(-1)
+        bias = np.asarray(w2, float)[flat] @ np.asarray(w1, float).T if np.shape(w1)[1] == np.shape(w2)[1] else None
+        emb = np.asarray(w1, float)[flat]
+        return (oracle.round_to(out_dtype, bias).reshape(i.shape + (np.shape(w2)[0],)),
+                emb.reshape(i.shape + (np.shape(w1)[1],)))
+    monkeypatch.setattr(oracle, "transition_logits", wrong)
+    _fails(pins.test_transition_logits_worked_example_and_bigram)
