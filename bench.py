@@ -42,12 +42,12 @@ METRIC = "corrected-logit rows/s + achieved HBM GB/s (% roofline); sampled block
 UNIT = "rows/s"
 FALLBACK_HBM_GBS = 6650.0
 PARTS = (("apply", W.APPLY_320), ("greedy", W.greedy(32)), ("temperature", W.TEMPERATURE))
-EXTRA = (("apply_2560", W.APPLY_2560), ("transition", W.TRANSITION_320))
+EXTRA = (("apply_2560", W.APPLY_2560), ("transition", W.TRANSITION_320), ("backward", W.BACKWARD_320))
 L2_BYTES = 126 * 1024 * 1024
 
 
 def part_rows(wl: W.Workload) -> int:
-    return wl.rows if wl.mode in ("apply", "transition") else wl.batch * wl.proposal_len
+    return wl.rows if wl.mode in ("apply", "transition", "backward") else wl.batch * wl.proposal_len
 
 
 # --------------------------------------------------------------- helpers --
@@ -160,6 +160,9 @@ class Part:
             dev["head"] = VanillaMarkov(dev["w1"], dev["w2"])
             if wl.mode == "apply":
                 dev["out"] = torch.empty_like(dev["base"])
+            elif wl.mode == "backward":
+                dev["gw1"] = torch.empty(wl.vocab, wl.rank, dtype=torch.float32, device=device)
+                dev["gw2"] = torch.empty(wl.vocab, wl.rank, dtype=torch.float32, device=device)
             elif wl.mode == "transition":
                 ids = dev["prev_ids"]
                 dev["out"] = torch.empty(*ids.shape, wl.vocab, dtype=torch.bfloat16, device=device)
@@ -176,6 +179,9 @@ class Part:
             s["head"].apply_block_logits(s["base"], token_ids=s["prev_ids"], out=s["out"])
         elif self.wl.mode == "transition":
             s["head"].transition_logits(s["prev_ids"], out=s["out"], out_embeddings=s["emb"])
+        elif self.wl.mode == "backward":
+            s["head"].apply_block_logits_backward(s["base"], token_ids=s["prev_ids"], grad_w1=s["gw1"],
+                                                  grad_w2=s["gw2"])
         else:
             s["head"].sample_block_tokens(s["base"], first_prev_token_ids=s["first_prev"],
                                           temperature=self.wl.temperature, seed=self.wl.philox_seed,

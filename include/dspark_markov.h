@@ -79,6 +79,31 @@ int dspark_markov_apply_block_logits(const void* base_logits, void* out, const i
                                      int32_t logits_dtype, int32_t weight_dtype, void* stream);
 
 /*
+ * Gradients of the teacher-forced apply, its train-time use
+ * (markov_head.py, the vendored DSpark-style low-rank Markov head: "At TRAIN time
+ * x_{k-1} is the teacher-forced ground-truth predecessor (apply_block_logits)").
+ * With out = U + W1[x] W2^T and grad_out = dOut [rows, vocab]:
+ *
+ *     grad of base_logits = grad_out           (identity: nothing is computed)
+ *     grad_w2[v, j] (+)= sum_i dOut[i, v] W1[x_i, j]
+ *     grad_w1[x, j] (+)= sum over rows i with x_i = x of sum_v dOut[i, v] W2[v, j]
+ *
+ *   grad_out        [rows, vocab] logits_dtype; prev_token_ids [rows] int64.
+ *   w1, w2          [vocab, rank] weight_dtype (rank <= 1024).
+ *   grad_w1/grad_w2 [vocab, rank] fp32, caller-owned; either may be NULL (not wanted).
+ *   accumulate      nonzero: add into the buffers (as autograd accumulates .grad);
+ *                   zero: overwrite them.
+ *
+ * Sums are accumulated in fp32 (grad_w1 with atomics, so the order of its
+ * additions varies from run to run). A row whose id is outside [0, vocab)
+ * contributes nothing and sets DSPARK_STATUS_TOKEN_RANGE. CUDA-core kernels.
+ */
+int dspark_markov_apply_block_logits_backward(const void* grad_out, const int64_t* prev_token_ids, int64_t rows,
+                                              int64_t vocab, const void* w1, const void* w2, int32_t rank,
+                                              float* grad_w1, float* grad_w2, int32_t accumulate,
+                                              int32_t logits_dtype, int32_t weight_dtype, void* stream);
+
+/*
  * The transition bias alone, and its conditioning embeddings
  * (nemo_automodel.components.models.deepseek_v41.dspark,
  * _DeepseekV41DSparkMarkovHead.forward: "transition logits of shape [..., vocab]

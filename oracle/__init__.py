@@ -12,6 +12,7 @@ names start with ``test_oracle``.
 from .markov import (  # noqa: F401
     GREEDY_TEMPERATURE,
     apply_block_logits,
+    apply_block_logits_backward,
     apply_step_logits,
     compute_step_bias,
     get_prev_embeddings,

@@ -105,6 +105,29 @@ def transition_logits(w1, w2, token_ids, out_dtype: str):
     return (round_to(out_dtype, bias).reshape(ids.shape + (vocab,)), emb.reshape(ids.shape + (rank,)))
 
 
+def apply_block_logits_backward(grad_out, w1, w2, token_ids):
+    """Gradients of the teacher-forced ``apply_block_logits`` (its train-time
+    use: "At TRAIN time x_{k-1} is the teacher-forced ground-truth
+    predecessor (apply_block_logits)"), in fp64. With out = U + W1[x] W2^T:
+
+        dU = dOut (returned unchanged),
+        dW2[v, j] = sum_i dOut[i, v] W1[x_i, j],
+        dW1[x, j] = sum over rows i with x_i = x of sum_v dOut[i, v] W2[v, j]
+
+    (the embedding lookup's backward adds each row's gradient at its id).
+    ``grad_out`` is (..., M, V) and ``token_ids`` (..., M); returns
+    (dW1 [V, r], dW2 [V, r])."""
+    vocab = np.shape(w2)[0]
+    dout = np.asarray(grad_out, dtype=np.float64).reshape(-1, vocab)
+    ids = np.asarray(token_ids, dtype=np.int64).reshape(-1)
+    emb = get_prev_embeddings(w1, ids)
+    dw2 = dout.T @ emb
+    d_emb = dout @ np.asarray(w2, dtype=np.float64)
+    dw1 = np.zeros(np.shape(w1), dtype=np.float64)
+    np.add.at(dw1, ids, d_emb)
+    return dw1, dw2
+
+
 def select_greedy(logits: np.ndarray) -> np.ndarray:
     """argmax over the last axis; the lowest index wins among equal maxima and
     NaN counts as the largest value (numpy's argmax has both properties)."""

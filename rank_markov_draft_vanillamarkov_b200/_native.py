@@ -37,6 +37,8 @@ SIGNATURES = {
     "dspark_markov_apply_block_logits": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i64, _vp, _vp, _i32, _i32, _i32, _vp]),
     "dspark_markov_sample_block": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _i32, _f32, _u64, _vp, _vp,
                                                   _i32, _i32, _vp]),
+    "dspark_markov_apply_block_logits_backward": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _i32, _vp, _vp,
+                                                                 _i32, _i32, _i32, _vp]),
     "dspark_markov_transition_logits": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp, _i32, _vp, _vp, _i32, _vp]),
     "dspark_markov_sample_block_noalloc": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _i32, _f32, _u64,
                                                           _vp, _vp, _i32, _i32, _vp]),

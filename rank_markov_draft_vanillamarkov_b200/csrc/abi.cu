@@ -194,6 +194,31 @@ int dspark_markov_apply_block_logits(const void* base_logits, void* out, const i
   return cuda_code(launch_generic_apply(a, logits_dtype, weight_dtype, s));
 }
 
+int dspark_markov_apply_block_logits_backward(const void* grad_out, const int64_t* prev_token_ids, int64_t rows,
+                                              int64_t vocab, const void* w1, const void* w2, int32_t rank,
+                                              float* grad_w1, float* grad_w2, int32_t accumulate,
+                                              int32_t logits_dtype, int32_t weight_dtype, void* stream) {
+  t_last_algo = 0;
+  if (rows < 0 || vocab <= 0 || rank <= 0 || !dtype_ok(logits_dtype) || !dtype_ok(weight_dtype))
+    return DSPARK_ERR_INVALID_ARG;
+  if (!grad_w1 && !grad_w2) return DSPARK_OK;  // nothing wanted
+  if (rows > 0 && (!grad_out || !prev_token_ids || !w1 || !w2)) return DSPARK_ERR_INVALID_ARG;
+  if (rank > 1024) return DSPARK_ERR_UNSUPPORTED;
+  int err = DSPARK_OK;
+  DeviceState* d = device_state(&err);
+  if (!d) return err;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = (size_t)vocab * (size_t)rank * sizeof(float);
+  if (!accumulate) {  // the gradients start from zero (dW2 is overwritten in full)
+    if (grad_w1 && cudaMemsetAsync(grad_w1, 0, bytes, s) != cudaSuccess) return DSPARK_ERR_CUDA;
+    if (grad_w2 && rows == 0 && cudaMemsetAsync(grad_w2, 0, bytes, s) != cudaSuccess) return DSPARK_ERR_CUDA;
+  }
+  if (rows == 0) return DSPARK_OK;
+  BackwardArgs a{grad_out, prev_token_ids, rows, vocab, w1, w2, rank, grad_w1, grad_w2, accumulate, d->status};
+  t_last_algo = 1;
+  return cuda_code(launch_backward(a, logits_dtype, weight_dtype, s));
+}
+
 int dspark_markov_transition_logits(const int64_t* token_ids, int64_t rows, int64_t vocab, const void* w1,
                                     const void* w2, int32_t rank, void* transition_out, void* embeddings_out,
                                     int32_t weight_dtype, void* stream) {

@@ -135,6 +135,117 @@ __global__ void gumbel_probe_kernel(const uint32_t* __restrict__ words, float* _
 }
 }  // namespace
 
+namespace {
+constexpr int kBwdSlice = 4096;  // vocabulary ids per dW1 block
+
+// dW1[x_i, :] += sum over one vocabulary slice of dOut[i, v] W2[v, :]: block
+// (row i, slice); thread j owns column j (reads of W2 rows are coalesced,
+// dOut[i, v] is a broadcast), and adds its partial sum with one atomic.
+template <typename TL, typename TW>
+__global__ void backward_dw1_kernel(BackwardArgs a) {
+  const int64_t i = blockIdx.x;
+  const int64_t id = a.ids[i];
+  if (id < 0 || id >= a.vocab) {
+    if (threadIdx.x == 0 && blockIdx.y == 0) report_status(a.status, DSPARK_STATUS_TOKEN_RANGE);
+    return;
+  }
+  const TL* g = static_cast<const TL*>(a.grad_out) + i * a.vocab;
+  const TW* w2 = static_cast<const TW*>(a.w2);
+  const int64_t v0 = (int64_t)blockIdx.y * kBwdSlice;
+  const int64_t v1 = v0 + kBwdSlice < a.vocab ? v0 + kBwdSlice : a.vocab;
+  for (int j = threadIdx.x; j < a.rank; j += blockDim.x) {
+    float acc = 0.0f;
+    for (int64_t v = v0; v < v1; ++v) acc = fmaf(to_f32(g[v]), to_f32(w2[v * a.rank + j]), acc);
+    atomicAdd(&a.grad_w1[id * a.rank + j], acc);
+  }
+}
+
+// dW2[v, :] = sum_i dOut[i, v] W1[x_i, :]: block of 32 ids (one per lane),
+// warp w owns columns 32w .. 32w+31; the embedding rows of 32 rows at a time
+// are staged in shared memory and read as broadcasts.
+template <typename TL, typename TW>
+__global__ void backward_dw2_kernel(BackwardArgs a) {
+  extern __shared__ float emb[];  // [32][rank]
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t v = (int64_t)blockIdx.x * 32 + lane;
+  const TL* g = static_cast<const TL*>(a.grad_out);
+  const TW* w1 = static_cast<const TW*>(a.w1);
+  float acc[32];
+#pragma unroll
+  for (int jj = 0; jj < 32; ++jj) acc[jj] = 0.0f;
+  for (int64_t i0 = 0; i0 < a.rows; i0 += 32) {
+    for (int t = threadIdx.x; t < 32 * a.rank; t += blockDim.x) {
+      const int r = t / a.rank, j = t % a.rank;
+      const int64_t i = i0 + r;
+      float x = 0.0f;
+      if (i < a.rows) {
+        const int64_t id = a.ids[i];
+        if (id >= 0 && id < a.vocab) x = to_f32(w1[id * a.rank + j]);
+      }
+      emb[r * a.rank + j] = x;
+    }
+    __syncthreads();
+    const int nr = a.rows - i0 < 32 ? (int)(a.rows - i0) : 32;
+    for (int r = 0; r < nr; ++r) {
+      const float d = v < a.vocab ? to_f32(g[(i0 + r) * a.vocab + v]) : 0.0f;
+      const float* e = emb + r * a.rank + 32 * w;
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj)
+        if (32 * w + jj < a.rank) acc[jj] = fmaf(d, e[jj], acc[jj]);
+    }
+    __syncthreads();
+  }
+  if (v >= a.vocab) return;
+#pragma unroll
+  for (int jj = 0; jj < 32; ++jj) {
+    const int j = 32 * w + jj;
+    if (j >= a.rank) break;
+    float* dst = &a.grad_w2[v * a.rank + j];
+    *dst = a.accumulate ? *dst + acc[jj] : acc[jj];
+  }
+}
+
+template <typename TL, typename TW>
+cudaError_t launch_backward_t(const BackwardArgs& a, cudaStream_t s) {
+  if (a.grad_w1) {
+    const int64_t slices = (a.vocab + kBwdSlice - 1) / kBwdSlice;
+    if (slices > 65535 || a.rows > 0x7fffffffll) return cudaErrorInvalidConfiguration;
+    if (a.rows > 0) {
+      const int threads = a.rank < 256 ? ((a.rank + 31) / 32) * 32 : 256;
+      backward_dw1_kernel<TL, TW><<<dim3((unsigned)a.rows, (unsigned)slices), threads, 0, s>>>(a);
+      note_launch();
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+  }
+  if (a.grad_w2) {
+    const int warps = (a.rank + 31) / 32;
+    if (warps > 32) return cudaErrorInvalidConfiguration;
+    const size_t smem = (size_t)32 * a.rank * sizeof(float);
+    if (smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(backward_dw2_kernel<TL, TW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    const int64_t blocks = (a.vocab + 31) / 32;
+    backward_dw2_kernel<TL, TW><<<(unsigned)blocks, 32 * warps, smem, s>>>(a);
+    note_launch();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+}  // namespace
+
+cudaError_t launch_backward(const BackwardArgs& a, int logits_dtype, int weight_dtype, cudaStream_t s) {
+  if (logits_dtype == DSPARK_DTYPE_FP32 && weight_dtype == DSPARK_DTYPE_FP32) return launch_backward_t<float, float>(a, s);
+  if (logits_dtype == DSPARK_DTYPE_BF16 && weight_dtype == DSPARK_DTYPE_BF16)
+    return launch_backward_t<__nv_bfloat16, __nv_bfloat16>(a, s);
+  if (logits_dtype == DSPARK_DTYPE_FP32 && weight_dtype == DSPARK_DTYPE_BF16)
+    return launch_backward_t<float, __nv_bfloat16>(a, s);
+  return launch_backward_t<__nv_bfloat16, float>(a, s);
+}
+
 cudaError_t launch_gather_rows(const int64_t* ids, const void* w1, void* out, int64_t rows, int64_t vocab,
                                int32_t rank, int weight_dtype, uint32_t* status, int num_sms, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;

@@ -37,6 +37,21 @@ struct GenericSelectArgs {
 
 cudaError_t launch_generic_apply(const GenericApplyArgs& a, int logits_dtype, int weight_dtype, cudaStream_t s);
 cudaError_t launch_generic_select(const GenericSelectArgs& a, int logits_dtype, cudaStream_t s);
+// Gradients of the teacher-forced apply (fp32, accumulated into or written).
+struct BackwardArgs {
+  const void* grad_out;  // [rows, vocab] logits dtype
+  const int64_t* ids;    // [rows]
+  int64_t rows, vocab;
+  const void* w1;
+  const void* w2;
+  int32_t rank;
+  float* grad_w1;  // [vocab, rank] or null
+  float* grad_w2;  // [vocab, rank] or null
+  int32_t accumulate;
+  uint32_t* status;
+};
+cudaError_t launch_backward(const BackwardArgs& a, int logits_dtype, int weight_dtype, cudaStream_t s);
+
 cudaError_t launch_gather_rows(const int64_t* ids, const void* w1, void* out, int64_t rows, int64_t vocab,
                                int32_t rank, int weight_dtype, uint32_t* status, int num_sms, cudaStream_t s);
 cudaError_t launch_gumbel_probe(const uint32_t* words, float* out, int64_t n, int num_sms, cudaStream_t s);

@@ -109,6 +109,43 @@ class VanillaMarkov:
         return self.apply_block_logits(logits.unsqueeze(-2), token_ids=token_ids.unsqueeze(-1),
                                        hidden_states=hidden_states).squeeze(-2)
 
+    def apply_block_logits_backward(self, grad_out: torch.Tensor, *, token_ids: torch.Tensor,
+                                    grad_w1: Optional[torch.Tensor] = None, grad_w2: Optional[torch.Tensor] = None,
+                                    accumulate: bool = False, want_w1: bool = True, want_w2: bool = True):
+        """Gradients of ``apply_block_logits`` with respect to W1 and W2 (fp32,
+        [V, r]) for ``grad_out`` (..., M, V) and the teacher-forced
+        ``token_ids`` (..., M); the gradient of the base logits is
+        ``grad_out`` itself. ``accumulate`` adds into given buffers."""
+        vocab, rank = self.vocab_size, self.markov_rank
+        if grad_out.shape[-1] != vocab or tuple(token_ids.shape) != tuple(grad_out.shape[:-1]):
+            raise ValueError("grad_out must be (..., V) with token_ids (...)")
+        if grad_out.dtype not in _DT:
+            raise ValueError("grad_out must be float32 or bfloat16")
+        g = grad_out.contiguous()
+        _check_cuda(g, "grad_out", self.device)
+        ids = (token_ids if token_ids.dtype == torch.int64 else token_ids.long()).contiguous()
+        _check_cuda(ids, "token_ids", self.device)
+        outs = []
+        for want, buf, name in ((want_w1, grad_w1, "grad_w1"), (want_w2, grad_w2, "grad_w2")):
+            if not want:
+                outs.append(None)
+                continue
+            if buf is None:
+                if accumulate:
+                    raise ValueError(f"accumulate needs {name}")
+                buf = torch.empty(vocab, rank, dtype=torch.float32, device=self.device)
+            elif tuple(buf.shape) != (vocab, rank) or buf.dtype != torch.float32:
+                raise ValueError(f"{name} must be fp32 (V, r)")
+            _check_cuda(buf, name, self.device)
+            outs.append(buf)
+        code = self._lib.dspark_markov_apply_block_logits_backward(
+            g.data_ptr(), ids.data_ptr(), ids.numel(), vocab, self.markov_w1.data_ptr(), self.markov_w2.data_ptr(),
+            rank, outs[0].data_ptr() if outs[0] is not None else None,
+            outs[1].data_ptr() if outs[1] is not None else None, 1 if accumulate else 0, _DT[g.dtype],
+            _DT[self.weight_dtype], _stream_ptr(self.device))
+        N.check(code, "dspark_markov_apply_block_logits_backward")
+        return outs[0], outs[1]
+
     def transition_logits(self, token_ids: torch.Tensor, *, with_embeddings: bool = True,
                           out: Optional[torch.Tensor] = None,
                           out_embeddings: Optional[torch.Tensor] = None):

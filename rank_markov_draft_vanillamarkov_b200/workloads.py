@@ -38,9 +38,11 @@ class Workload:
     """One seeded synthetic workload.
 
     ``mode`` is ``"apply"`` (teacher-forced, rows = batch * num_blocks *
-    block_size), ``"transition"`` (the bias alone and the embeddings of the
-    same rows, no base logits) or ``"sample"`` (left-to-right, ``batch``
-    blocks of ``proposal_len`` positions).
+    block_size), ``"backward"`` (the apply's gradients for W1 and W2; the
+    base-logit tensor serves as the incoming gradient), ``"transition"``
+    (the bias alone and the embeddings of the same rows, no base logits) or
+    ``"sample"`` (left-to-right, ``batch`` blocks of ``proposal_len``
+    positions).
     """
 
     name: str
@@ -77,6 +79,10 @@ class Workload:
         if self.mode == "apply":
             r = self.rows
             return 2 * r * self.vocab * lb + self.vocab * self.rank * wb + r * self.rank * wb + r * 8
+        if self.mode == "backward":  # grad in, W2 and W1 rows in, ids, two fp32 [V, r] gradients out
+            r = self.rows
+            return r * self.vocab * lb + self.vocab * self.rank * wb + r * self.rank * wb + r * 8 \
+                + 2 * self.vocab * self.rank * 4
         if self.mode == "transition":  # bias out, W2, W1 rows in and embeddings out, ids
             r = self.rows
             return r * self.vocab * wb + self.vocab * self.rank * wb + 2 * r * self.rank * wb + r * 8
@@ -86,6 +92,8 @@ class Workload:
 
     def flops(self) -> int:
         r = self.rows if self.mode in ("apply", "transition") else self.batch * self.proposal_len
+        if self.mode == "backward":  # dW2 and dW1 each cost one product per (row, id, rank) term
+            return 4 * self.rows * self.vocab * self.rank
         return 2 * r * self.vocab * self.rank
 
 
@@ -102,6 +110,9 @@ GREEDY = Workload("greedy_m5_v129280_k128", "sample", vocab=129280, rank=128, ba
 TEMPERATURE = Workload("temp0.7_b32_m8_v151936_k64", "sample", vocab=151936, rank=64, batch=32,
                        proposal_len=8, logit_std=1.5, weight_std=0.05, temperature=0.7,
                        philox_seed=1234, data_seed=0)
+BACKWARD_320 = Workload("backward_r320_v129280_k128", "backward", vocab=129280, rank=128, batch=4,
+                        num_blocks=16, block_size=5, logit_std=1.0, weight_std=0.02, prev_dist="zipf1.1",
+                        data_seed=0)
 TRANSITION_320 = Workload("transition_r320_v129280_k128", "transition", vocab=129280, rank=128, batch=4,
                           num_blocks=16, block_size=5, weight_std=0.02, prev_dist="zipf1.1", data_seed=0)
 APPLY_2560 = Workload("apply_r2560_v129280_k256_pad20", "apply", vocab=129280, rank=256, batch=8,
@@ -157,7 +168,7 @@ def make_inputs(wl: Workload) -> dict:
         n = wl.rows
         ids = zipf_ids(g, n, wl.vocab, 1.1) if wl.prev_dist == "zipf1.1" else uniform_ids(g, n, wl.vocab)
         out["prev_ids"] = ids.view(wl.batch, wl.num_blocks, wl.block_size)
-    elif wl.mode == "apply":
+    elif wl.mode in ("apply", "backward"):
         shape = (wl.batch, wl.num_blocks, wl.block_size, wl.vocab)
         base = _normal(g, shape, wl.logit_std, wl.logits_dtype)
         n = wl.rows

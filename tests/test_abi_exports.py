@@ -82,6 +82,16 @@ def test_transition_argument_checks(lib):
     assert tr(p, 4, 128, p, p, 16, None, p, 1, None) == N.DSPARK_ERR_INVALID_ARG  # no output
 
 
+def test_backward_argument_checks(lib):
+    p = ctypes.c_void_p(16)  # never dereferenced
+    bw = lib.dspark_markov_apply_block_logits_backward
+    assert bw(p, p, 4, 128, p, p, 16, None, None, 0, 1, 1, None) == N.DSPARK_OK  # nothing wanted
+    assert bw(p, p, 4, 128, p, p, 0, p, p, 0, 1, 1, None) == N.DSPARK_ERR_INVALID_ARG  # rank 0
+    assert bw(p, p, -1, 128, p, p, 16, p, p, 0, 1, 1, None) == N.DSPARK_ERR_INVALID_ARG
+    assert bw(p, p, 4, 128, p, p, 16, p, p, 0, 9, 1, None) == N.DSPARK_ERR_INVALID_ARG  # bad dtype
+    assert bw(None, p, 4, 128, p, p, 16, p, p, 0, 1, 1, None) == N.DSPARK_ERR_INVALID_ARG
+
+
 def test_host_utilities(lib):
     assert lib.dspark_markov_strerror(0) == b"ok"
     assert lib.dspark_markov_strerror(N.DSPARK_ERR_UNSUPPORTED).startswith(b"unsupported")

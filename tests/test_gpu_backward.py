@@ -1,0 +1,105 @@
+"""Parity of the CUDA backward of the teacher-forced apply against the fp64
+oracle (B200).
+
+The gradients are fp32 sums of products that are exact in fp32 (bf16 x bf16,
+or fp32 x fp32 for the fp32 case only up to one rounding each), so the only
+error is the fp32 accumulation. A sum of K terms in any order is within about
+u * sqrt(K) * sum|terms| of the exact value for random-sign terms (u = 2^-24);
+the tests allow 16 u sqrt(K) * sum|terms| per element, with K the number of
+terms of that element.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from rank_markov_draft_vanillamarkov_b200 import VanillaMarkov, device_status
+from rank_markov_draft_vanillamarkov_b200 import _native as N
+from rank_markov_draft_vanillamarkov_b200 import workloads as W
+from rank_markov_draft_vanillamarkov_b200.build import build
+
+from _helpers import f64
+
+pytestmark = pytest.mark.gpu
+
+U = 2.0 ** -24
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build()
+    N.load()
+
+
+def _inputs(rows, vocab, rank, seed, ldt=torch.bfloat16, wdt=torch.bfloat16):
+    g = torch.Generator().manual_seed(seed)
+    w1 = (torch.randn(vocab, rank, generator=g) * 0.3).to(wdt)
+    w2 = (torch.randn(vocab, rank, generator=g) * 0.3).to(wdt)
+    dout = torch.randn(rows, vocab, generator=g).to(ldt)
+    ids = W.zipf_ids(g, rows, vocab)
+    return w1, w2, dout, ids
+
+
+def _check(w1, w2, dout, ids, gw1, gw2):
+    d, a1, a2, i = f64(dout), f64(w1), f64(w2), ids.numpy()
+    want1, want2 = oracle.apply_block_logits_backward(d, a1, a2, i)
+    # sum of |terms| of every element, and its number of terms
+    abs2 = np.abs(d).T @ np.abs(a1[i])
+    abs1 = np.zeros_like(a1)
+    np.add.at(abs1, i, np.abs(d) @ np.abs(a2))
+    counts = np.bincount(i, minlength=a1.shape[0])[:, None]
+    k1 = np.maximum(counts * d.shape[1], 1)
+    tol1 = 16 * U * np.sqrt(k1) * abs1 + 1e-30
+    tol2 = 16 * U * np.sqrt(d.shape[0]) * abs2 + 1e-30
+    e1 = np.abs(gw1.cpu().double().numpy() - want1)
+    e2 = np.abs(gw2.cpu().double().numpy() - want2)
+    assert (e1 <= tol1).all(), (e1.max(), np.unravel_index(np.argmax(e1 - tol1), e1.shape))
+    assert (e2 <= tol2).all(), (e2.max(), np.unravel_index(np.argmax(e2 - tol2), e2.shape))
+
+
+@pytest.mark.parametrize("rows,vocab,rank", [(200, 1000, 64), (37, 4099, 96), (330, 2056, 256)])
+def test_backward_small(rows, vocab, rank):
+    w1, w2, dout, ids = _inputs(rows, vocab, rank, seed=rows)
+    head = VanillaMarkov(w1.cuda(), w2.cuda())
+    gw1, gw2 = head.apply_block_logits_backward(dout.cuda(), token_ids=ids.cuda())
+    torch.cuda.synchronize()
+    assert device_status() == 0
+    _check(w1, w2, dout, ids, gw1, gw2)
+
+
+def test_backward_full_size_block_shape():
+    """320 rows shaped (4, 16, 5) at V = 129280, rank 128, Zipf(1.1) ids
+    (so many rows share an id and their dW1 contributions add up)."""
+    d = W.make_inputs(W.APPLY_320)
+    g = torch.Generator().manual_seed(1)
+    dout = torch.randn(4, 16, 5, 129280, generator=g).to(torch.bfloat16)
+    head = VanillaMarkov(d["w1"].cuda(), d["w2"].cuda())
+    gw1, gw2 = head.apply_block_logits_backward(dout.cuda(), token_ids=d["prev_ids"].cuda())
+    torch.cuda.synchronize()
+    assert device_status() == 0
+    _check(d["w1"], d["w2"], dout.view(-1, 129280), d["prev_ids"].view(-1), gw1, gw2)
+
+
+def test_backward_fp32_and_accumulate():
+    """fp32 operands, and accumulate = True adds onto given buffers."""
+    w1, w2, dout, ids = _inputs(50, 1024, 16, seed=3, ldt=torch.float32, wdt=torch.float32)
+    head = VanillaMarkov(w1.cuda(), w2.cuda())
+    b1 = torch.full((1024, 16), 0.5, device="cuda")
+    b2 = torch.full((1024, 16), -0.25, device="cuda")
+    head.apply_block_logits_backward(dout.cuda(), token_ids=ids.cuda(), grad_w1=b1, grad_w2=b2, accumulate=True)
+    torch.cuda.synchronize()
+    _check(w1, w2, dout, ids, b1 - 0.5, b2 + 0.25)
+
+
+def test_backward_out_of_range_ids():
+    """A row with an id outside [0, V) contributes nothing and sets the
+    TOKEN_RANGE status."""
+    w1, w2, dout, ids = _inputs(64, 1000, 64, seed=5)
+    ids[10] = 1000
+    ids[20] = -3
+    head = VanillaMarkov(w1.cuda(), w2.cuda())
+    gw1, gw2 = head.apply_block_logits_backward(dout.cuda(), token_ids=ids.cuda())
+    torch.cuda.synchronize()
+    assert device_status() & N.DSPARK_STATUS_TOKEN_RANGE
+    keep = torch.from_numpy(np.setdiff1d(np.arange(64), [10, 20]))
+    _check(w1, w2, dout[keep], ids[keep], gw1, gw2)

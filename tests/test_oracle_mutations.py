@@ -116,3 +116,17 @@ def test_transition_with_transposed_lookup_is_caught(monkeypatch):
                 emb.reshape(i.shape + (np.shape(w1)[1],)))
     monkeypatch.setattr(oracle, "transition_logits", wrong)
     _fails(pins.test_transition_logits_worked_example_and_bigram)
+
+
+def test_backward_overwriting_repeated_ids_is_caught(monkeypatch):
+    """dW1 written (not added) at ids that occur in several rows."""
+    def wrong(grad_out, w1, w2, token_ids):
+        vocab = np.shape(w2)[0]
+        dout = np.asarray(grad_out, float).reshape(-1, vocab)
+        ids = np.asarray(token_ids, np.int64).reshape(-1)
+        emb = np.asarray(w1, float)[ids]
+        dw1 = np.zeros(np.shape(w1))
+        dw1[ids] = dout @ np.asarray(w2, float)
+        return dw1, dout.T @ emb
+    monkeypatch.setattr(oracle, "apply_block_logits_backward", wrong)
+    _fails(pins.test_backward_matches_torch_autograd)

@@ -140,6 +140,38 @@ def test_transition_logits_worked_example_and_bigram():
     np.testing.assert_array_equal(emb, np.eye(16)[bids])
 
 
+def test_backward_matches_torch_autograd():
+    """The backward against torch.autograd (a library implementation) on the
+    fp64 forward U + Embedding(W1)(x) @ W2^T, with repeated ids."""
+    rng = np.random.default_rng(7)
+    v, r = 37, 6
+    w1, w2 = rng.standard_normal((v, r)), rng.standard_normal((v, r))
+    ids = np.array([[3, 3, 0, 36], [5, 3, 9, 0]])
+    dout = rng.standard_normal((2, 4, v))
+    dw1, dw2 = oracle.apply_block_logits_backward(dout, w1, w2, ids)
+    t1 = torch.tensor(w1, requires_grad=True)
+    t2 = torch.tensor(w2, requires_grad=True)
+    base = torch.tensor(rng.standard_normal((2, 4, v)))
+    out = base + torch.nn.functional.embedding(torch.tensor(ids), t1) @ t2.T
+    out.backward(torch.tensor(dout))
+    np.testing.assert_allclose(dw1, t1.grad.numpy(), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dw2, t2.grad.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_backward_bigram_closed_form():
+    """W1 = identity: dW2[v, x] is the sum of dOut[i, v] over rows with
+    previous token x, and dW1[x] the sum of dOut[i] @ W2 over those rows;
+    exact with integer values."""
+    w1, w2, _ = _bigram_case()
+    ids = np.array([3, 0, 15, 3, 7, 3])
+    dout = np.random.default_rng(2).integers(-4, 5, size=(6, 16)).astype(float)
+    dw1, dw2 = oracle.apply_block_logits_backward(dout, w1, w2, ids)
+    for x in range(16):
+        rows = ids == x
+        np.testing.assert_array_equal(dw2[:, x], dout[rows].sum(0))
+        np.testing.assert_array_equal(dw1[x], (dout[rows] @ w2).sum(0))
+
+
 def test_zero_w2_passes_logits_through_bit_for_bit():
     rng = np.random.default_rng(1)
     base = oracle.round_to_bfloat16(rng.standard_normal((3, 4, 5, 64)) * 3)
