@@ -136,99 +136,152 @@ __global__ void gumbel_probe_kernel(const uint32_t* __restrict__ words, float* _
 }  // namespace
 
 namespace {
-constexpr int kBwdSlice = 4096;  // vocabulary ids per dW1 block
+// Register-tiled fp32 contractions on CUDA cores: 256 threads, operand tiles
+// of 32 along the summed dimension staged in shared memory as fp32.
+constexpr int kBwdK = 32;       // summed-dimension tile
+constexpr int kBwdSlice = 2048;  // vocabulary ids per dW1 block (split of the sum over V)
 
-// dW1[x_i, :] += sum over one vocabulary slice of dOut[i, v] W2[v, :]: block
-// (row i, slice); thread j owns column j (reads of W2 rows are coalesced,
-// dOut[i, v] is a broadcast), and adds its partial sum with one atomic.
+// dW1: G = dOut . W2 for 64 rows x 128 rank columns over one vocabulary
+// slice; each thread owns 4 rows x 8 columns; the partial sums are added at
+// the rows' ids (the embedding lookup's backward) with atomics.
 template <typename TL, typename TW>
-__global__ void backward_dw1_kernel(BackwardArgs a) {
-  const int64_t i = blockIdx.x;
-  const int64_t id = a.ids[i];
-  if (id < 0 || id >= a.vocab) {
-    if (threadIdx.x == 0 && blockIdx.y == 0) report_status(a.status, DSPARK_STATUS_TOKEN_RANGE);
-    return;
-  }
-  const TL* g = static_cast<const TL*>(a.grad_out) + i * a.vocab;
+__global__ void __launch_bounds__(256) backward_dw1_kernel(BackwardArgs a) {
+  __shared__ float sa[kBwdK][64 + 1];  // dOut^T tile [k][row]; the pad spreads the transposed stores over banks
+  __shared__ __align__(16) float sb[kBwdK][128];  // W2 tile [k][column]
+  const int tid = threadIdx.x, tr = tid >> 4, tc = tid & 15;
+  const int64_t m0 = (int64_t)blockIdx.x * 64, n0 = (int64_t)blockIdx.z * 128;
+  const int64_t k0 = (int64_t)blockIdx.y * kBwdSlice;
+  const int64_t k1 = k0 + kBwdSlice < a.vocab ? k0 + kBwdSlice : a.vocab;
+  const TL* g = static_cast<const TL*>(a.grad_out);
   const TW* w2 = static_cast<const TW*>(a.w2);
-  const int64_t v0 = (int64_t)blockIdx.y * kBwdSlice;
-  const int64_t v1 = v0 + kBwdSlice < a.vocab ? v0 + kBwdSlice : a.vocab;
-  for (int j = threadIdx.x; j < a.rank; j += blockDim.x) {
-    float acc = 0.0f;
-    for (int64_t v = v0; v < v1; ++v) acc = fmaf(to_f32(g[v]), to_f32(w2[v * a.rank + j]), acc);
-    atomicAdd(&a.grad_w1[id * a.rank + j], acc);
+  float acc[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+  for (int64_t kk = k0; kk < k1; kk += kBwdK) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {  // 64 rows x 32 ids, consecutive threads along the ids
+      const int e = tid + 256 * q, row = e >> 5, kx = e & 31;
+      const int64_t gr = m0 + row, gk = kk + kx;
+      sa[kx][row] = (gr < a.rows && gk < k1) ? to_f32(g[gr * a.vocab + gk]) : 0.0f;
+    }
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {  // 32 ids x 128 columns, consecutive threads along the columns
+      const int e = tid + 256 * q, kx = e >> 7, c = e & 127;
+      const int64_t gk = kk + kx, gc = n0 + c;
+      sb[kx][c] = (gk < k1 && gc < a.rank) ? to_f32(w2[gk * a.rank + gc]) : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int k = 0; k < kBwdK; ++k) {
+      float av[4], bv[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) av[i] = sa[k][tr * 4 + i];
+      const float4 b0 = *reinterpret_cast<const float4*>(&sb[k][tc * 8]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&sb[k][tc * 8 + 4]);
+      bv[0] = b0.x; bv[1] = b0.y; bv[2] = b0.z; bv[3] = b0.w;
+      bv[4] = b1.x; bv[5] = b1.y; bv[6] = b1.z; bv[7] = b1.w;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t gr = m0 + tr * 4 + i;
+    if (gr >= a.rows) break;
+    const int64_t id = a.ids[gr];
+    if (id < 0 || id >= a.vocab) {
+      if (blockIdx.y == 0 && blockIdx.z == 0 && tc == 0) report_status(a.status, DSPARK_STATUS_TOKEN_RANGE);
+      continue;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int64_t gc = n0 + tc * 8 + j;
+      if (gc < a.rank) atomicAdd(&a.grad_w1[id * a.rank + gc], acc[i][j]);
+    }
   }
 }
 
-// dW2[v, :] = sum_i dOut[i, v] W1[x_i, :]: block of 32 ids (one per lane),
-// warp w owns columns 32w .. 32w+31; the embedding rows of 32 rows at a time
-// are staged in shared memory and read as broadcasts.
+// dW2 = dOut^T . W1[x] for 128 ids x 128 rank columns; each thread owns
+// 8 ids x 8 columns and sums over all rows, 32 at a time.
 template <typename TL, typename TW>
-__global__ void backward_dw2_kernel(BackwardArgs a) {
-  extern __shared__ float emb[];  // [32][rank]
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int64_t v = (int64_t)blockIdx.x * 32 + lane;
+__global__ void __launch_bounds__(256) backward_dw2_kernel(BackwardArgs a) {
+  __shared__ __align__(16) float sd[kBwdK][128];  // dOut tile [row][id]
+  __shared__ __align__(16) float se[kBwdK][128];  // embedding tile [row][column]
+  const int tid = threadIdx.x, tr = tid >> 4, tc = tid & 15;
+  const int64_t v0 = (int64_t)blockIdx.x * 128, n0 = (int64_t)blockIdx.y * 128;
   const TL* g = static_cast<const TL*>(a.grad_out);
   const TW* w1 = static_cast<const TW*>(a.w1);
-  float acc[32];
+  float acc[8][8];
 #pragma unroll
-  for (int jj = 0; jj < 32; ++jj) acc[jj] = 0.0f;
-  for (int64_t i0 = 0; i0 < a.rows; i0 += 32) {
-    for (int t = threadIdx.x; t < 32 * a.rank; t += blockDim.x) {
-      const int r = t / a.rank, j = t % a.rank;
-      const int64_t i = i0 + r;
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+  for (int64_t i0 = 0; i0 < a.rows; i0 += kBwdK) {
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int e = tid + 256 * q, k = e >> 7, c = e & 127;
+      const int64_t gi = i0 + k, gv = v0 + c, gc = n0 + c;
+      sd[k][c] = (gi < a.rows && gv < a.vocab) ? to_f32(g[gi * a.vocab + gv]) : 0.0f;
       float x = 0.0f;
-      if (i < a.rows) {
-        const int64_t id = a.ids[i];
-        if (id >= 0 && id < a.vocab) x = to_f32(w1[id * a.rank + j]);
+      if (gi < a.rows && gc < a.rank) {
+        const int64_t id = a.ids[gi];
+        if (id >= 0 && id < a.vocab)
+          x = to_f32(w1[id * a.rank + gc]);
+        else if (blockIdx.x == 0 && blockIdx.y == 0 && c == 0)
+          report_status(a.status, DSPARK_STATUS_TOKEN_RANGE);
       }
-      emb[r * a.rank + j] = x;
+      se[k][c] = x;
     }
     __syncthreads();
-    const int nr = a.rows - i0 < 32 ? (int)(a.rows - i0) : 32;
-    for (int r = 0; r < nr; ++r) {
-      const float d = v < a.vocab ? to_f32(g[(i0 + r) * a.vocab + v]) : 0.0f;
-      const float* e = emb + r * a.rank + 32 * w;
+#pragma unroll 4
+    for (int k = 0; k < kBwdK; ++k) {
+      const float4 d0 = *reinterpret_cast<const float4*>(&sd[k][tr * 8]);
+      const float4 d1 = *reinterpret_cast<const float4*>(&sd[k][tr * 8 + 4]);
+      const float4 e0 = *reinterpret_cast<const float4*>(&se[k][tc * 8]);
+      const float4 e1 = *reinterpret_cast<const float4*>(&se[k][tc * 8 + 4]);
+      const float dv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+      const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj)
-        if (32 * w + jj < a.rank) acc[jj] = fmaf(d, e[jj], acc[jj]);
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(dv[i], ev[j], acc[i][j]);
     }
     __syncthreads();
   }
-  if (v >= a.vocab) return;
 #pragma unroll
-  for (int jj = 0; jj < 32; ++jj) {
-    const int j = 32 * w + jj;
-    if (j >= a.rank) break;
-    float* dst = &a.grad_w2[v * a.rank + j];
-    *dst = a.accumulate ? *dst + acc[jj] : acc[jj];
+  for (int i = 0; i < 8; ++i) {
+    const int64_t gv = v0 + tr * 8 + i;
+    if (gv >= a.vocab) break;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int64_t gc = n0 + tc * 8 + j;
+      if (gc >= a.rank) break;
+      float* dst = &a.grad_w2[gv * a.rank + gc];
+      *dst = a.accumulate ? *dst + acc[i][j] : acc[i][j];
+    }
   }
 }
 
 template <typename TL, typename TW>
 cudaError_t launch_backward_t(const BackwardArgs& a, cudaStream_t s) {
-  if (a.grad_w1) {
-    const int64_t slices = (a.vocab + kBwdSlice - 1) / kBwdSlice;
-    if (slices > 65535 || a.rows > 0x7fffffffll) return cudaErrorInvalidConfiguration;
-    if (a.rows > 0) {
-      const int threads = a.rank < 256 ? ((a.rank + 31) / 32) * 32 : 256;
-      backward_dw1_kernel<TL, TW><<<dim3((unsigned)a.rows, (unsigned)slices), threads, 0, s>>>(a);
-      note_launch();
-      cudaError_t e = cudaGetLastError();
-      if (e != cudaSuccess) return e;
-    }
+  const int64_t ntiles = (a.rank + 127) / 128;
+  if (a.grad_w1 && a.rows > 0) {
+    const int64_t mtiles = (a.rows + 63) / 64, slices = (a.vocab + kBwdSlice - 1) / kBwdSlice;
+    if (mtiles > 0x7fffffffll || slices > 65535 || ntiles > 65535) return cudaErrorInvalidConfiguration;
+    backward_dw1_kernel<TL, TW><<<dim3((unsigned)mtiles, (unsigned)slices, (unsigned)ntiles), 256, 0, s>>>(a);
+    note_launch();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
   }
   if (a.grad_w2) {
-    const int warps = (a.rank + 31) / 32;
-    if (warps > 32) return cudaErrorInvalidConfiguration;
-    const size_t smem = (size_t)32 * a.rank * sizeof(float);
-    if (smem > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(backward_dw2_kernel<TL, TW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)smem);
-      if (e != cudaSuccess) return e;
-    }
-    const int64_t blocks = (a.vocab + 31) / 32;
-    backward_dw2_kernel<TL, TW><<<(unsigned)blocks, 32 * warps, smem, s>>>(a);
+    const int64_t vtiles = (a.vocab + 127) / 128;
+    if (vtiles > 0x7fffffffll || ntiles > 65535) return cudaErrorInvalidConfiguration;
+    backward_dw2_kernel<TL, TW><<<dim3((unsigned)vtiles, (unsigned)ntiles), 256, 0, s>>>(a);
     note_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
