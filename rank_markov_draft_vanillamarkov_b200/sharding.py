@@ -1,10 +1,14 @@
 """Splitting the head's work across GPUs (one process per GPU).
 
-Both entry points are data-parallel with no exchange step: teacher-forced rows
-are independent, and so are the blocks of the sampler (each block's chain
-depends only on its own earlier tokens). So N GPUs hold replicas of W1/W2 and
-each processes a contiguous slice of rows or blocks; no collective is needed
-on the data path. These helpers compute the slices.
+The forward entry points are data-parallel with no exchange step:
+teacher-forced rows are independent, and so are the blocks of the sampler
+(each block's chain depends only on its own earlier tokens). So N GPUs hold
+replicas of W1/W2 and each processes a contiguous slice of rows or blocks; no
+collective is needed on the data path. These helpers compute the slices.
+
+Training is the one place with a real exchange: every rank's rows contribute
+to the same W1/W2 gradients, so the per-rank gradients are summed across the
+ranks (an all-reduce; NCCL over NVLink on GPUs) before any update.
 """
 from __future__ import annotations
 
@@ -47,3 +51,17 @@ def sample_block_tokens_shard(head, base_logits, first_prev_token_ids, rank: int
     lo, hi = shard_range(base_logits.shape[0], rank, world)
     return head.sample_block_tokens(base_logits[lo:hi], first_prev_token_ids=first_prev_token_ids[lo:hi],
                                     temperature=temperature, seed=shard_seed(seed, lo))
+
+
+def apply_block_logits_backward_shard(head, grad_out, token_ids, rank: int, world: int, group=None):
+    """Gradients of W1 and W2 (fp32, [V, r]) for the whole batch: this rank
+    differentiates its slice of the leading (batch) axis, then the two
+    gradients are summed over the ranks in place (torch.distributed
+    all_reduce). With world == 1 no collective runs."""
+    import torch.distributed as dist
+    lo, hi = shard_range(grad_out.shape[0], rank, world)
+    gw1, gw2 = head.apply_block_logits_backward(grad_out[lo:hi], token_ids=token_ids[lo:hi])
+    if world > 1:
+        dist.all_reduce(gw1, op=dist.ReduceOp.SUM, group=group)
+        dist.all_reduce(gw2, op=dist.ReduceOp.SUM, group=group)
+    return gw1, gw2

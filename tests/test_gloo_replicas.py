@@ -28,6 +28,11 @@ class OracleHead:
         return torch.from_numpy(oracle.apply_block_logits(base_logits.to(torch.float64).numpy(), self.w1, self.w2,
                                                           token_ids.numpy(), "bf16"))
 
+    def apply_block_logits_backward(self, grad_out, *, token_ids):
+        g1, g2 = oracle.apply_block_logits_backward(grad_out.to(torch.float64).numpy(), self.w1, self.w2,
+                                                    token_ids.numpy())
+        return torch.from_numpy(g1), torch.from_numpy(g2)
+
     def sample_block_tokens(self, base_logits, *, first_prev_token_ids, temperature=0.0, seed=0):
         t, c = oracle.sample_block_tokens(base_logits.to(torch.float64).numpy(), self.w1, self.w2,
                                           first_prev_token_ids.numpy(), "bf16", temperature, seed)
@@ -124,3 +129,43 @@ def test_shard_range_tiles_exactly():
             assert max(sizes) - min(sizes) <= 1
     with pytest.raises(ValueError):
         sharding.shard_range(4, 2, 2)
+
+
+def _backward_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        wl = W.small_variants()[0]  # 2 x 20 blocks x 5, V = 1000, Zipf ids (shared across the two slices)
+        d = W.make_inputs(wl)
+        grad = torch.randn(d["base"].shape, generator=torch.Generator().manual_seed(4), dtype=torch.float64)
+        head = OracleHead(d["w1"], d["w2"])
+        g1, g2 = sharding.apply_block_logits_backward_shard(head, grad, d["prev_ids"], rank, world)
+        q.put((rank, g1.numpy(), g2.numpy()))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(300)
+def test_two_rank_backward_all_reduce_matches_full_batch():
+    """Each rank differentiates its half of the batch; after the all-reduce
+    both ranks hold the full-batch gradients of W1 and W2."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_backward_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=240) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    wl = W.small_variants()[0]
+    d = W.make_inputs(wl)
+    grad = torch.randn(d["base"].shape, generator=torch.Generator().manual_seed(4), dtype=torch.float64)
+    want1, want2 = oracle.apply_block_logits_backward(grad.numpy(), d["w1"].double().numpy(),
+                                                      d["w2"].double().numpy(), d["prev_ids"].numpy())
+    for _, g1, g2 in got:
+        np.testing.assert_allclose(g1, want1, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(g2, want2, rtol=1e-12, atol=1e-12)
