@@ -232,49 +232,76 @@ def time_e2e(parts, steps, world):
     """The same step through the public API with host buffers: each step
     copies its inputs host->device from pinned memory, runs the three calls
     and copies every output (corrected logits and tokens) back to pinned host
-    memory; all inside the timed region."""
+    memory; all inside the timed region. Copies in the two directions and the
+    calls run on three streams with two sets of device buffers, so the link's
+    two directions and the kernels overlap across consecutive parts and steps
+    (the link is full duplex); every step still moves all its bytes."""
     import torch.distributed as dist
     from rank_markov_draft_vanillamarkov_b200 import VanillaMarkov
     dev = parts[0].device
-    host, devb, h2d, d2h = [], [], 0, 0
+    s_in, s_run, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    jobs, h2d, d2h = [], 0, 0
     for p in parts:
         h = {k: v.pin_memory() for k, v in p.host.items() if isinstance(v, torch.Tensor) and k not in ("w1", "w2")}
-        d = {k: torch.empty_like(v, device=dev) for k, v in h.items()}
-        d["head"] = VanillaMarkov(p.sets[0]["w1"], p.sets[0]["w2"])
-        out_host = torch.empty_like(p.host["base"]).pin_memory()
+        keys = ["base", "prev_ids"] if p.wl.mode == "apply" else ["base", "first_prev"]
+        head = VanillaMarkov(p.sets[0]["w1"], p.sets[0]["w2"])
+        bufs = []
+        for _ in range(2):  # device inputs and outputs, one set per step parity
+            d = {k: torch.empty_like(h[k], device=dev) for k in keys}
+            d["out"] = torch.empty_like(d["base"])
+            if p.wl.mode == "sample":
+                d["tok"] = torch.empty(p.wl.batch, p.wl.proposal_len, dtype=torch.long, device=dev)
+            d["copied"], d["done"], d["read"] = (torch.cuda.Event() for _ in range(3))
+            d["read"].record(s_out)
+            bufs.append(d)
+        out_host = torch.empty_like(h["base"]).pin_memory()
         tok_host = torch.empty(p.wl.batch, p.wl.proposal_len, dtype=torch.long).pin_memory() \
             if p.wl.mode == "sample" else None
-        keys = ["base", "prev_ids"] if p.wl.mode == "apply" else ["base", "first_prev"]
         h2d += sum(h[k].numel() * h[k].element_size() for k in keys)
         d2h += out_host.numel() * out_host.element_size() + (tok_host.numel() * 8 if tok_host is not None else 0)
-        host.append((p, h, keys, out_host, tok_host))
-        devb.append(d)
+        jobs.append((p, head, h, keys, bufs, out_host, tok_host))
 
-    def one():
-        for (p, h, keys, out_host, tok_host), d in zip(host, devb):
-            for k in keys:
-                d[k].copy_(h[k], non_blocking=True)
-            if p.wl.mode == "apply":
-                out = d["head"].apply_block_logits(d["base"], token_ids=d["prev_ids"])
-                out_host.copy_(out, non_blocking=True)
-            else:
-                t, c = d["head"].sample_block_tokens(d["base"], first_prev_token_ids=d["first_prev"],
-                                                     temperature=p.wl.temperature, seed=p.wl.philox_seed)
-                out_host.copy_(c, non_blocking=True)
-                tok_host.copy_(t, non_blocking=True)
+    def one(i):
+        for p, head, h, keys, bufs, out_host, tok_host in jobs:
+            d = bufs[i & 1]
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(d["read"])  # this set's previous outputs have been read back
+                for k in keys:
+                    d[k].copy_(h[k], non_blocking=True)
+                d["copied"].record(s_in)
+            with torch.cuda.stream(s_run):
+                s_run.wait_event(d["copied"])
+                if p.wl.mode == "apply":
+                    head.apply_block_logits(d["base"], token_ids=d["prev_ids"], out=d["out"])
+                else:
+                    head.sample_block_tokens(d["base"], first_prev_token_ids=d["first_prev"],
+                                             temperature=p.wl.temperature, seed=p.wl.philox_seed,
+                                             out_tokens=d["tok"], out_logits=d["out"])
+                d["done"].record(s_run)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(d["done"])
+                out_host.copy_(d["out"], non_blocking=True)
+                if tok_host is not None:
+                    tok_host.copy_(d["tok"], non_blocking=True)
+                d["read"].record(s_out)
 
-    for _ in range(3):
-        one()
+    for i in range(3):
+        one(i)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(steps):
-        one()
-    b.record()
+    cur = torch.cuda.current_stream(dev)
+    a.record(cur)
+    for st in (s_in, s_run, s_out):
+        st.wait_stream(cur)  # nothing of the timed region starts before `a`
+    for i in range(steps):
+        one(i)
+    for st in (s_in, s_run, s_out):
+        cur.wait_stream(st)
+    b.record(cur)
     torch.cuda.synchronize()
     sec = a.elapsed_time(b) / 1e3
     if world > 1:
