@@ -327,3 +327,16 @@ def test_gumbel_noise_every_word_within_bound():
     assert err.max() < 1e-5, (err.max(), int(err.argmax()))
     # u closest to 1 (the largest draws) and closest to 0
     assert abs(out[-1].item() - exact[-1]) < 1e-5 and abs(out[0].item() - exact[0]) < 1e-5
+
+
+@pytest.mark.parametrize("temperature", [0.0, 0.9])
+@pytest.mark.parametrize("batch", [1, 3, 4])
+def test_small_batch_cuda_core_bias(batch, temperature):
+    """Batches of one to four on the tensor-core sampler at full vocabulary,
+    rank 128 (so a CTA keeps W2 tiles in both shared and tensor memory),
+    with weights that move tokens: every (b, k) against the oracle."""
+    wl = W.greedy(batch).with_(weight_std=0.3, spike=0.0, data_seed=20 + batch)
+    d = W.make_inputs(wl)
+    toks, corr, used, st = _sample(d, TC, temperature, seed=5)
+    assert used == 2 and st == 0
+    _check(d, toks, corr, temperature, 5)
