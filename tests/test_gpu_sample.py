@@ -331,7 +331,7 @@ def test_gumbel_noise_every_word_within_bound():
 
 @pytest.mark.parametrize("temperature", [0.0, 0.9])
 @pytest.mark.parametrize("batch", [1, 3, 4])
-def test_small_batch_cuda_core_bias(batch, temperature):
+def test_small_batches_full_vocabulary(batch, temperature):
     """Batches of one to four on the tensor-core sampler at full vocabulary,
     rank 128 (so a CTA keeps W2 tiles in both shared and tensor memory),
     with weights that move tokens: every (b, k) against the oracle."""
