@@ -42,7 +42,8 @@ METRIC = "corrected-logit rows/s + achieved HBM GB/s (% roofline); sampled block
 UNIT = "rows/s"
 FALLBACK_HBM_GBS = 6650.0
 PARTS = (("apply", W.APPLY_320), ("greedy", W.greedy(32)), ("temperature", W.TEMPERATURE))
-EXTRA = (("apply_2560", W.APPLY_2560), ("transition", W.TRANSITION_320), ("backward", W.BACKWARD_320))
+EXTRA = (("apply_2560", W.APPLY_2560), ("apply_fp32", W.APPLY_320_FP32), ("transition", W.TRANSITION_320),
+         ("backward", W.BACKWARD_320))
 L2_BYTES = 126 * 1024 * 1024
 
 

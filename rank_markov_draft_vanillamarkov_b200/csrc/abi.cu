@@ -185,7 +185,8 @@ int dspark_markov_apply_block_logits(const void* base_logits, void* out, const i
                      (reinterpret_cast<uintptr_t>(w2) % 16 == 0) && (reinterpret_cast<uintptr_t>(w1) % 16 == 0);
   if (algo == DSPARK_ALGO_TENSOR_CORE && !tc_ok) return DSPARK_ERR_UNSUPPORTED;
   if (tc_ok && algo != DSPARK_ALGO_GENERIC) {
-    TcApplyArgs a{base_logits, out, prev_token_ids, rows, vocab, w1, w2, rank, d->status, g_wait_limit_ns.load()};
+    TcApplyArgs a{base_logits, out, prev_token_ids, rows, vocab, w1, w2, rank, d->status, g_wait_limit_ns.load(),
+                  logits_dtype == DSPARK_DTYPE_FP32 ? 1 : 0};
     t_last_algo = 2;
     return cuda_code(launch_tc_apply(a, d->num_sms, s));
   }
@@ -237,7 +238,8 @@ int dspark_markov_transition_logits(const int64_t* token_ids, int64_t rows, int6
   if (algo == DSPARK_ALGO_TENSOR_CORE && !tc_ok) return DSPARK_ERR_UNSUPPORTED;
   cudaError_t e;
   if (tc_ok && algo != DSPARK_ALGO_GENERIC) {
-    TcApplyArgs a{nullptr, transition_out, token_ids, rows, vocab, w1, w2, rank, d->status, g_wait_limit_ns.load()};
+    TcApplyArgs a{nullptr, transition_out, token_ids, rows, vocab, w1, w2, rank, d->status, g_wait_limit_ns.load(),
+                  0};
     t_last_algo = 2;
     e = launch_tc_apply(a, d->num_sms, s);
   } else {

@@ -41,8 +41,10 @@ namespace {
 constexpr int kBM = 128;              // rows per unit (MMA M)
 constexpr int kBN = 128;              // vocabulary ids per unit (MMA N)
 constexpr int kAtomK = 64;            // bf16 elements in one 128-byte swizzle row
-constexpr int kAtomBytes = 128 * 128; // one 128-row x 64-element W2 atom / one U box
-constexpr int kUStageBytes = 2 * kAtomBytes;  // 128 rows x 128 ids of bf16
+constexpr int kAtomBytes = 128 * 128; // one 128-row x 64-element W2 atom / one U box (128-byte rows)
+// A U stage holds one unit, 128 rows x 128 ids: two boxes of 64 bf16 ids, or
+// four boxes of 32 fp32 ids (every box row is 128 bytes).
+__host__ __device__ constexpr int u_stage_bytes(bool f32) { return (f32 ? 4 : 2) * kAtomBytes; }
 constexpr int kThreads = 512;
 constexpr int kTmemCols = 512;
 constexpr int kAccCols = 2 * kBN;     // accumulators occupy [0, 256)
@@ -144,14 +146,17 @@ __device__ __forceinline__ void gather_tile_to_tmem(const ApplyParams& p, int m,
 
 // HAS_BASE false: no U (the bias alone, rounded once): the producer loads no
 // U tile and the epilogue adds zero, using the stage only to assemble the
-// output tile for its TMA store.
-template <int KA, bool HAS_BASE>
+// output tile for its TMA store. F32: fp32 logits (U and out); the bias is
+// added in fp32, which is the one rounding.
+template <int KA, bool HAS_BASE, bool F32>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_apply_kernel(const __grid_constant__ ApplyMaps maps, const ApplyParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* w2_smem = smem;                                     // w2_slots x KA atoms
-  uint8_t* u_smem = w2_smem + (size_t)p.w2_slots * KA * kAtomBytes;  // u_stages x 32 KB
+  constexpr int kUStageBytes = u_stage_bytes(F32);
+  constexpr int kBoxIds = F32 ? 32 : 64;  // ids per 128-byte box row
+  uint8_t* u_smem = w2_smem + (size_t)p.w2_slots * KA * kAtomBytes;  // u_stages x kUStageBytes
   SharedTail* sh = reinterpret_cast<SharedTail*>(u_smem + (size_t)p.u_stages * kUStageBytes);
 
   constexpr int kACols = KA * 32;  // TMEM columns of one A tile
@@ -223,8 +228,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (HAS_BASE) {
           mbar_arrive_expect_tx(&sh->u_full[s], kUStageBytes);
           uint8_t* st = u_smem + s * kUStageBytes;
-          tma_load_2d(st, &maps.u, &sh->u_full[s], n * kBN, m * kBM, pol_stream);
-          tma_load_2d(st + kAtomBytes, &maps.u, &sh->u_full[s], n * kBN + 64, m * kBM, pol_stream);
+#pragma unroll
+          for (int bx = 0; bx < kUStageBytes / kAtomBytes; ++bx)
+            tma_load_2d(st + bx * kAtomBytes, &maps.u, &sh->u_full[s], n * kBN + bx * kBoxIds, m * kBM, pol_stream);
         } else {
           mbar_arrive(&sh->u_full[s]);  // the stage is free for the epilogue
         }
@@ -331,16 +337,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_32x32b_x32(tbase + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&acc[0]));
         tmem_ld_32x32b_x32(tbase + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&acc[32]));
         tmem_ld_wait();
-        uint8_t* box = st + h * kAtomBytes + row * 128;
+        if constexpr (F32) {
+          // The half's 64 ids are boxes 2h and 2h+1, 32 fp32 each: chunk c
+          // of a box row holds ids 4c .. 4c+3.
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4* ptr = reinterpret_cast<uint4*>(box + ((c ^ (row & 7)) << 4));
-          uint4 x = HAS_BASE ? *ptr : make_uint4(0u, 0u, 0u, 0u);
-          x.x = add_round_pair(x.x, acc[c * 8 + 0], acc[c * 8 + 1]);
-          x.y = add_round_pair(x.y, acc[c * 8 + 2], acc[c * 8 + 3]);
-          x.z = add_round_pair(x.z, acc[c * 8 + 4], acc[c * 8 + 5]);
-          x.w = add_round_pair(x.w, acc[c * 8 + 6], acc[c * 8 + 7]);
-          *ptr = x;
+          for (int sub = 0; sub < 2; ++sub) {
+            uint8_t* box = st + (2 * h + sub) * kAtomBytes + row * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              float4* ptr = reinterpret_cast<float4*>(box + ((c ^ (row & 7)) << 4));
+              float4 x = HAS_BASE ? *ptr : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+              const uint32_t* a4 = &acc[sub * 32 + c * 4];
+              x.x += __uint_as_float(a4[0]);
+              x.y += __uint_as_float(a4[1]);
+              x.z += __uint_as_float(a4[2]);
+              x.w += __uint_as_float(a4[3]);
+              *ptr = x;
+            }
+          }
+        } else {
+          uint8_t* box = st + h * kAtomBytes + row * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint4* ptr = reinterpret_cast<uint4*>(box + ((c ^ (row & 7)) << 4));
+            uint4 x = HAS_BASE ? *ptr : make_uint4(0u, 0u, 0u, 0u);
+            x.x = add_round_pair(x.x, acc[c * 8 + 0], acc[c * 8 + 1]);
+            x.y = add_round_pair(x.y, acc[c * 8 + 2], acc[c * 8 + 3]);
+            x.z = add_round_pair(x.z, acc[c * 8 + 4], acc[c * 8 + 5]);
+            x.w = add_round_pair(x.w, acc[c * 8 + 6], acc[c * 8 + 7]);
+            *ptr = x;
+          }
         }
       }
       tc_fence_before_sync();
@@ -350,8 +376,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       named_barrier_sync(bar_id, 128);
       if (et == 0) {
-        tma_store_2d(&maps.out, st, n * kBN, m * kBM);
-        tma_store_2d(&maps.out, st + kAtomBytes, n * kBN + 64, m * kBM);
+#pragma unroll
+        for (int bx = 0; bx < kUStageBytes / kAtomBytes; ++bx)
+          tma_store_2d(&maps.out, st + bx * kAtomBytes, n * kBN + bx * kBoxIds, m * kBM);
         bulk_commit_group();
         bulk_wait_group_read<0>();  // the stage may be refilled once the store has read it
         mbar_arrive(&sh->u_empty[s]);
@@ -375,7 +402,8 @@ struct ApplyConfig {
   size_t smem_bytes;
 };
 
-ApplyConfig plan(int ka, int row_tiles) {
+ApplyConfig plan(int ka, int row_tiles, bool f32) {
+  const int kUStageBytes = u_stage_bytes(f32);
   ApplyConfig c{};
   c.resident = (row_tiles <= kMaxResidentTiles && row_tiles * ka * 32 <= kTmemCols - kAccCols) ? 1 : 0;
   const size_t fixed = 1024 + sizeof(SharedTail) + 64;
@@ -399,15 +427,16 @@ ApplyConfig plan(int ka, int row_tiles) {
 template <int KA>
 cudaError_t launch_ka(const TcApplyArgs& a, int num_sms, cudaStream_t stream) {
   ApplyMaps maps;
+  const bool f32 = a.logits_f32 != 0;
+  const CUtensorMapDataType ldt = f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const uint64_t ldim[2] = {(uint64_t)a.vocab, (uint64_t)a.rows};
-  const uint64_t lstr[1] = {(uint64_t)a.vocab * 2};
+  const uint64_t lstr[1] = {(uint64_t)a.vocab * (f32 ? 4 : 2)};
+  const uint32_t ubox[2] = {f32 ? 32u : 64u, 128};  // 128-byte rows
   const uint32_t lbox[2] = {64, 128};
   const bool has_base = a.base != nullptr;
   // Without a base the U map is never read; it is encoded on `out` to stay valid.
-  if (!encode_tensor_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, has_base ? a.base : a.out, ldim, lstr, lbox,
-                         CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tensor_map(&maps.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.out, ldim, lstr, lbox,
-                         CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!encode_tensor_map(&maps.u, ldt, 2, has_base ? a.base : a.out, ldim, lstr, ubox, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tensor_map(&maps.out, ldt, 2, a.out, ldim, lstr, ubox, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   const uint64_t wdim[2] = {(uint64_t)a.rank, (uint64_t)a.vocab};
   const uint64_t wstr[1] = {(uint64_t)a.rank * 2};
@@ -423,14 +452,15 @@ cudaError_t launch_ka(const TcApplyArgs& a, int num_sms, cudaStream_t stream) {
   p.rank = a.rank;
   p.row_tiles = (int32_t)((a.rows + kBM - 1) / kBM);
   p.vocab_tiles = (int32_t)((a.vocab + kBN - 1) / kBN);
-  const ApplyConfig c = plan(KA, p.row_tiles);
+  const ApplyConfig c = plan(KA, p.row_tiles, f32);
   p.w2_slots = c.w2_slots;
   p.u_stages = c.u_stages;
   p.resident = c.resident;
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns;
 
-  auto kernel = has_base ? tc_apply_kernel<KA, true> : tc_apply_kernel<KA, false>;
+  auto kernel = f32 ? (has_base ? tc_apply_kernel<KA, true, true> : tc_apply_kernel<KA, false, true>)
+                    : (has_base ? tc_apply_kernel<KA, true, false> : tc_apply_kernel<KA, false, false>);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)c.smem_bytes);
   if (e != cudaSuccess) return e;
   const int64_t units = (int64_t)p.row_tiles * p.vocab_tiles;
@@ -443,7 +473,9 @@ cudaError_t launch_ka(const TcApplyArgs& a, int num_sms, cudaStream_t stream) {
 }  // namespace
 
 bool tc_apply_supported(int64_t rows, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype) {
-  if (logits_dtype != DSPARK_DTYPE_BF16 || weight_dtype != DSPARK_DTYPE_BF16) return false;
+  // bf16 weights; logits bf16 or fp32 (fp32 logits with a bf16 head).
+  if (weight_dtype != DSPARK_DTYPE_BF16) return false;
+  if (logits_dtype != DSPARK_DTYPE_BF16 && logits_dtype != DSPARK_DTYPE_FP32) return false;
   if (vocab % 8 != 0 || rank % 64 != 0 || rank < 64 || rank > 256) return false;
   const int64_t row_tiles = (rows + kBM - 1) / kBM;
   const int64_t vocab_tiles = (vocab + kBN - 1) / kBN;

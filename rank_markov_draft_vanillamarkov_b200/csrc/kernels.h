@@ -69,6 +69,7 @@ struct TcApplyArgs {
   int32_t rank;
   uint32_t* status;
   uint64_t wait_limit_ns;
+  int32_t logits_f32;  // base/out are fp32 (else bf16); the weights are bf16
 };
 bool tc_apply_supported(int64_t rows, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype);
 cudaError_t launch_tc_apply(const TcApplyArgs& a, int num_sms, cudaStream_t s);

@@ -113,6 +113,9 @@ TEMPERATURE = Workload("temp0.7_b32_m8_v151936_k64", "sample", vocab=151936, ran
 BACKWARD_320 = Workload("backward_r320_v129280_k128", "backward", vocab=129280, rank=128, batch=4,
                         num_blocks=16, block_size=5, logit_std=1.0, weight_std=0.02, prev_dist="zipf1.1",
                         data_seed=0)
+APPLY_320_FP32 = Workload("apply_fp32logits_r320_v129280_k128", "apply", vocab=129280, rank=128, batch=4,
+                          num_blocks=16, block_size=5, logits_dtype="fp32", weight_dtype="bf16", logit_std=2.0,
+                          weight_std=0.02, prev_dist="zipf1.1", data_seed=0)
 TRANSITION_320 = Workload("transition_r320_v129280_k128", "transition", vocab=129280, rank=128, batch=4,
                           num_blocks=16, block_size=5, weight_std=0.02, prev_dist="zipf1.1", data_seed=0)
 APPLY_2560 = Workload("apply_r2560_v129280_k256_pad20", "apply", vocab=129280, rank=256, batch=8,

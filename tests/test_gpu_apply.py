@@ -92,14 +92,42 @@ def test_tiny_fp32_workload():
 
 
 @pytest.mark.parametrize("ldt,wdt", [(torch.float32, torch.bfloat16), (torch.bfloat16, torch.float32)])
-def test_mixed_dtypes_generic(ldt, wdt):
+def test_mixed_dtypes(ldt, wdt):
     wl = W.small_variants()[0]
     d = W.make_inputs(wl)
     d = dict(d, base=d["base"].to(ldt), w1=d["w1"].to(wdt), w2=d["w2"].to(wdt))
     got, used, st = _run(d, N.DSPARK_ALGO_AUTO)
-    assert used == 1 and st == 0
+    # fp32 logits with bf16 weights run on the tensor-core kernel, the other pairs on the generic one
+    assert used == (2 if (ldt == torch.float32 and wdt == torch.bfloat16) else 1) and st == 0
     exact = _exact(d)
     _assert_ok(check_logits(f64(got).reshape(exact.shape), exact, dtype_name(ldt), _acc(d)), "mixed")
+
+
+_NON_RESIDENT = W.APPLY_320.with_(name="apply_small_r1100_v1000_k64", vocab=1000, rank=64, batch=4, num_blocks=55,
+                                  weight_std=0.3, data_seed=14)  # 9 row tiles: per-unit A
+
+
+@pytest.mark.parametrize("wl", W.small_variants() + [_NON_RESIDENT], ids=lambda w: w.name)
+def test_fp32_logits_tensor_core(wl):
+    """fp32 logits with a bf16 head (the stage's compute_logits returns fp32)
+    on the tensor-core kernel: ragged tiles, resident and per-unit A, in place."""
+    d = W.make_inputs(wl)
+    d = dict(d, base=d["base"].float())
+    got, used, st = _run(d, TC)
+    assert used == 2 and st == 0 and got.dtype == torch.float32
+    exact = _exact(d)
+    _assert_ok(check_logits(f64(got).reshape(exact.shape), exact, "fp32", _acc(d)), "fp32 logits")
+    base = d["base"].clone().cuda()
+    same, used, st = _run(d, TC, base=base, out=base)
+    assert same.data_ptr() == base.data_ptr() and torch.equal(same.cpu(), got.cpu())
+
+
+def test_apply_320_fp32_logits_full_size():
+    d = W.make_inputs(W.APPLY_320_FP32)
+    got, used, st = _run(d, N.DSPARK_ALGO_AUTO)
+    assert used == 2 and st == 0
+    exact = _exact(d)
+    _assert_ok(check_logits(f64(got).reshape(exact.shape), exact, "fp32", _acc(d)), "apply 320 fp32 logits")
 
 
 def test_apply_320_full_size():
