@@ -96,7 +96,14 @@ int dspark_markov_apply_block_logits(const void* base_logits, void* out, const i
  *
  * Sums are accumulated in fp32 (grad_w1 with atomics, so the order of its
  * additions varies from run to run). A row whose id is outside [0, vocab)
- * contributes nothing and sets DSPARK_STATUS_TOKEN_RANGE. CUDA-core kernels.
+ * contributes nothing and sets DSPARK_STATUS_TOKEN_RANGE.
+ *
+ * bf16 grad_out with bf16 weights, vocab % 8 == 0, rank in {64, 128, 192, 256}
+ * and 16-byte aligned pointers run on the tensor cores (two launches: dW2, then
+ * dW1); everything else on CUDA-core kernels. DSPARK_ALGO_TENSOR_CORE set by
+ * dspark_markov_set_algo makes an unsupported call return
+ * DSPARK_ERR_UNSUPPORTED; dspark_markov_last_algo reports 2 (tensor cores) or
+ * 1 (CUDA cores).
  */
 int dspark_markov_apply_block_logits_backward(const void* grad_out, const int64_t* prev_token_ids, int64_t rows,
                                               int64_t vocab, const void* w1, const void* w2, int32_t rank,

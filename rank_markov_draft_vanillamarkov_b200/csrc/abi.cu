@@ -216,6 +216,15 @@ int dspark_markov_apply_block_logits_backward(const void* grad_out, const int64_
   }
   if (rows == 0) return DSPARK_OK;
   BackwardArgs a{grad_out, prev_token_ids, rows, vocab, w1, w2, rank, grad_w1, grad_w2, accumulate, d->status};
+  const int32_t algo = g_algo.load();
+  const auto aligned = [](const void* q) { return reinterpret_cast<uintptr_t>(q) % 16 == 0; };
+  const bool tc_ok = tc_backward_supported(rows, vocab, rank, logits_dtype, weight_dtype) && aligned(grad_out) &&
+                     aligned(w1) && aligned(w2) && aligned(grad_w1) && aligned(grad_w2);
+  if (algo == DSPARK_ALGO_TENSOR_CORE && !tc_ok) return DSPARK_ERR_UNSUPPORTED;
+  if (tc_ok && algo != DSPARK_ALGO_GENERIC) {
+    t_last_algo = 2;
+    return cuda_code(launch_tc_backward(a, d->num_sms, g_wait_limit_ns.load(), s));
+  }
   t_last_algo = 1;
   return cuda_code(launch_backward(a, logits_dtype, weight_dtype, s));
 }

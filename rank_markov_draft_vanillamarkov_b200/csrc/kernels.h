@@ -99,6 +99,13 @@ bool tc_sample_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_
                          int num_sms);
 cudaError_t launch_tc_sample(const TcSampleArgs& a, int num_sms, cudaStream_t s);
 
+// Backward of the teacher-forced apply on tcgen05: bf16 gradient and bf16
+// weights, vocab % 8 == 0, rank in {64, 128, 192, 256}, every pointer 16-byte
+// aligned. grad_w1 must already hold its starting value (zero, or the sum to
+// add to); grad_w2 is written, or added to when accumulate is set.
+bool tc_backward_supported(int64_t rows, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype);
+cudaError_t launch_tc_backward(const BackwardArgs& a, int num_sms, uint64_t wait_limit_ns, cudaStream_t s);
+
 // Encodes a tiled TMA descriptor through the driver entry point.
 bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t rank, const void* base,
                        const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,

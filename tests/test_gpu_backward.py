@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import oracle
-from rank_markov_draft_vanillamarkov_b200 import VanillaMarkov, device_status
+from rank_markov_draft_vanillamarkov_b200 import VanillaMarkov, device_status, last_algo, set_algo
 from rank_markov_draft_vanillamarkov_b200 import _native as N
 from rank_markov_draft_vanillamarkov_b200 import workloads as W
 from rank_markov_draft_vanillamarkov_b200.build import build
@@ -25,10 +25,15 @@ pytestmark = pytest.mark.gpu
 U = 2.0 ** -24
 
 
+TC, GEN = N.DSPARK_ALGO_TENSOR_CORE, N.DSPARK_ALGO_GENERIC
+
+
 @pytest.fixture(scope="module", autouse=True)
 def _lib():
     build()
     N.load()
+    yield
+    set_algo(N.DSPARK_ALGO_AUTO)
 
 
 def _inputs(rows, vocab, rank, seed, ldt=torch.bfloat16, wdt=torch.bfloat16):
@@ -57,14 +62,41 @@ def _check(w1, w2, dout, ids, gw1, gw2):
     assert (e2 <= tol2).all(), (e2.max(), np.unravel_index(np.argmax(e2 - tol2), e2.shape))
 
 
-@pytest.mark.parametrize("rows,vocab,rank", [(200, 1000, 64), (37, 4099, 96), (330, 2056, 256)])
-def test_backward_small(rows, vocab, rank):
-    w1, w2, dout, ids = _inputs(rows, vocab, rank, seed=rows)
+def _run(w1, w2, dout, ids, algo, **kw):
+    set_algo(algo)
     head = VanillaMarkov(w1.cuda(), w2.cuda())
-    gw1, gw2 = head.apply_block_logits_backward(dout.cuda(), token_ids=ids.cuda())
+    gw1, gw2 = head.apply_block_logits_backward(dout.cuda(), token_ids=ids.cuda(), **kw)
     torch.cuda.synchronize()
+    return gw1, gw2, last_algo()
+
+
+@pytest.mark.parametrize("algo", [TC, GEN], ids=["tc", "generic"])
+@pytest.mark.parametrize("rows,vocab,rank", [
+    (200, 1000, 64),     # ragged 128-id tile and 64-row stage
+    (330, 2056, 256),    # four 64-column blocks, 6 row stages
+    (150, 2048, 192),    # three column blocks
+    (700, 20480, 128),   # 160 id tiles: CTAs take two dW2 units
+    (19000, 64, 128),    # 149 row tiles: CTAs take two dW1 units; one dW2 unit over 297 stages
+])
+def test_backward_small(rows, vocab, rank, algo):
+    w1, w2, dout, ids = _inputs(rows, vocab, rank, seed=rows)
+    gw1, gw2, used = _run(w1, w2, dout, ids, algo)
+    assert used == (2 if algo == TC else 1)
     assert device_status() == 0
     _check(w1, w2, dout, ids, gw1, gw2)
+
+
+def test_backward_generic_only_shapes():
+    """rank 96 and V = 4099 (not a multiple of 8) take the CUDA-core kernels
+    under AUTO; forcing the tensor cores is refused."""
+    w1, w2, dout, ids = _inputs(37, 4099, 96, seed=37)
+    gw1, gw2, used = _run(w1, w2, dout, ids, N.DSPARK_ALGO_AUTO)
+    assert used == 1 and device_status() == 0
+    _check(w1, w2, dout, ids, gw1, gw2)
+    set_algo(TC)
+    head = VanillaMarkov(w1.cuda(), w2.cuda())
+    with pytest.raises(RuntimeError):
+        head.apply_block_logits_backward(dout.cuda(), token_ids=ids.cuda())
 
 
 def test_backward_full_size_block_shape():
@@ -73,15 +105,40 @@ def test_backward_full_size_block_shape():
     d = W.make_inputs(W.APPLY_320)
     g = torch.Generator().manual_seed(1)
     dout = torch.randn(4, 16, 5, 129280, generator=g).to(torch.bfloat16)
-    head = VanillaMarkov(d["w1"].cuda(), d["w2"].cuda())
-    gw1, gw2 = head.apply_block_logits_backward(dout.cuda(), token_ids=d["prev_ids"].cuda())
-    torch.cuda.synchronize()
-    assert device_status() == 0
+    gw1, gw2, used = _run(d["w1"], d["w2"], dout, d["prev_ids"], N.DSPARK_ALGO_AUTO)
+    assert used == 2 and device_status() == 0
     _check(d["w1"], d["w2"], dout.view(-1, 129280), d["prev_ids"].view(-1), gw1, gw2)
 
 
+@pytest.mark.parametrize("algo", [TC, GEN], ids=["tc", "generic"])
+def test_backward_bf16_accumulate(algo):
+    """accumulate = True adds onto the given buffers (dW2 by TMA reduce-add on
+    the tensor-core path)."""
+    w1, w2, dout, ids = _inputs(260, 1032, 128, seed=11)
+    b1 = torch.full((1032, 128), 0.5, device="cuda")
+    b2 = torch.full((1032, 128), -0.25, device="cuda")
+    _, _, used = _run(w1, w2, dout, ids, algo, grad_w1=b1, grad_w2=b2, accumulate=True)
+    assert used == (2 if algo == TC else 1) and device_status() == 0
+    _check(w1, w2, dout, ids, b1 - 0.5, b2 + 0.25)
+
+
+@pytest.mark.parametrize("algo", [TC, GEN], ids=["tc", "generic"])
+def test_backward_one_gradient(algo):
+    """Only dW2 (want_w1 = False), then only dW1 (want_w2 = False): each
+    kernel alone."""
+    w1, w2, dout, ids = _inputs(90, 512, 64, seed=4)
+    set_algo(algo)
+    head = VanillaMarkov(w1.cuda(), w2.cuda())
+    only1, g2 = head.apply_block_logits_backward(dout.cuda(), token_ids=ids.cuda(), want_w1=False)
+    g1, only2 = head.apply_block_logits_backward(dout.cuda(), token_ids=ids.cuda(), want_w2=False)
+    torch.cuda.synchronize()
+    assert only1 is None and only2 is None and device_status() == 0
+    _check(w1, w2, dout, ids, g1, g2)
+
+
 def test_backward_fp32_and_accumulate():
-    """fp32 operands, and accumulate = True adds onto given buffers."""
+    """fp32 operands (CUDA-core kernels), and accumulate = True adds onto
+    given buffers."""
     w1, w2, dout, ids = _inputs(50, 1024, 16, seed=3, ldt=torch.float32, wdt=torch.float32)
     head = VanillaMarkov(w1.cuda(), w2.cuda())
     b1 = torch.full((1024, 16), 0.5, device="cuda")
@@ -91,15 +148,15 @@ def test_backward_fp32_and_accumulate():
     _check(w1, w2, dout, ids, b1 - 0.5, b2 + 0.25)
 
 
-def test_backward_out_of_range_ids():
+@pytest.mark.parametrize("algo", [TC, GEN], ids=["tc", "generic"])
+def test_backward_out_of_range_ids(algo):
     """A row with an id outside [0, V) contributes nothing and sets the
     TOKEN_RANGE status."""
     w1, w2, dout, ids = _inputs(64, 1000, 64, seed=5)
     ids[10] = 1000
     ids[20] = -3
-    head = VanillaMarkov(w1.cuda(), w2.cuda())
-    gw1, gw2 = head.apply_block_logits_backward(dout.cuda(), token_ids=ids.cuda())
-    torch.cuda.synchronize()
+    gw1, gw2, used = _run(w1, w2, dout, ids, algo)
+    assert used == (2 if algo == TC else 1)
     assert device_status() & N.DSPARK_STATUS_TOKEN_RANGE
     keep = torch.from_numpy(np.setdiff1d(np.arange(64), [10, 20]))
     _check(w1, w2, dout[keep], ids[keep], gw1, gw2)
