@@ -19,7 +19,7 @@
 // A operand, MN-major) and gathers the stage's 64 W1 rows with tile::gather4
 // (the B operand, MN-major; invalid ids and rows past the end read row
 // `vocab`, outside the tensor, i.e. zeros). The epilogue writes the fp32 tile
-// through two swizzled 32-column staging boxes with TMA stores, or TMA
+// through up to four swizzled 32-column staging boxes with TMA stores, or TMA
 // reduce-adds when accumulating.
 //
 // dW1 instance: split-K over the vocabulary. One unit = 128 rows (M) x rank
@@ -46,9 +46,12 @@ constexpr int kMaxStages = 8;
 constexpr uint32_t kBlockBytes = kKc * 128;  // one 64-element-wide box of kKc 128-byte rows
 constexpr uint32_t kOutBoxBytes = 128 * 128; // dW2 staging: 128 ids x 32 fp32
 constexpr size_t kSmemLimit = 232448;
+constexpr int32_t kRidCacheRows = 8192;     // dW2: rows whose W1 coordinates stay in shared memory
 
 __host__ __device__ constexpr uint32_t a_bytes_of(bool dw1) { return dw1 ? kBM * 128u : 2u * kBlockBytes; }
 __host__ __device__ constexpr uint32_t stage_bytes_of(int na, bool dw1) { return a_bytes_of(dw1) + na * kBlockBytes; }
+// dW2 staging boxes (128 ids x 32 fp32 each): one per 32-column chunk, at most four.
+__host__ __device__ constexpr int out_boxes_of(int na) { return 2 * na < 4 ? 2 * na : 4; }
 __host__ __device__ constexpr uint32_t tmem_cols_of(int na) {
   return 2 * na * 64 <= 128 ? 128u : 2 * na * 64 <= 256 ? 256u : 512u;
 }
@@ -113,6 +116,8 @@ struct BwdParams {
   int32_t stages;     // ring depth
   int32_t accumulate;
   int32_t keep_g;     // dW2: the dW1 kernel reads G next (ask L2 to keep it)
+  int32_t rid_cached; // dW2: rows (rounded up to 64) whose W1 coordinates are cached in
+                      // shared memory once per CTA; 0 = read per stage
   uint32_t* status;
   uint64_t wait_limit_ns;
 };
@@ -155,8 +160,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_backward_kernel(const __grid_c
   constexpr uint32_t kStageBytes = stage_bytes_of(NA, DW1);
   constexpr uint32_t kTmemCols = tmem_cols_of(NA);
   uint8_t* stage_smem = smem;
-  uint8_t* out_smem = smem + (size_t)p.stages * kStageBytes;  // dW2: two staging boxes
-  BwdShared* sh = reinterpret_cast<BwdShared*>(out_smem + (DW1 ? 0 : 2 * kOutBoxBytes));
+  uint8_t* out_smem = smem + (size_t)p.stages * kStageBytes;  // dW2: staging boxes
+  BwdShared* sh = reinterpret_cast<BwdShared*>(out_smem + (DW1 ? 0 : out_boxes_of(NA) * kOutBoxBytes));
+  int32_t* rid_all = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(sh) + sizeof(BwdShared));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -199,6 +205,33 @@ __global__ void __launch_bounds__(kThreads, 1) tc_backward_kernel(const __grid_c
     // first) asks L2 to keep it, and the dW1 pass reads it as evict-first.
     const uint64_t pol_g = (!DW1 && p.keep_g) ? policy_evict_last() : policy_evict_first();
     const uint64_t pol_w = policy_evict_last();
+    if constexpr (!DW1) {
+      // Every unit walks the same rows: their W1 coordinates are read once,
+      // eight loads in flight per lane, and padded with `vocab` to a whole stage.
+      for (int32_t r0 = 0; r0 < p.rid_cached; r0 += 32 * 8) {
+        int64_t idv[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int64_t r = (int64_t)r0 + 32 * t + lane;
+          idv[t] = r < p.rows ? p.ids[r] : 0;
+        }
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int32_t r = r0 + 32 * t + lane;
+          if (r < p.rid_cached) {
+            int32_t c = (int32_t)p.vocab;
+            if (r < p.rows) {
+              if (idv[t] >= 0 && idv[t] < p.vocab)
+                c = (int32_t)idv[t];
+              else
+                report_status(p.status, DSPARK_STATUS_TOKEN_RANGE);
+            }
+            rid_all[r] = c;
+          }
+        }
+      }
+      __syncwarp();
+    }
     uint32_t it = 0;
     bool ok = true;
     for (int64_t u = u_begin; u < u_end && ok; ++u) {
@@ -222,8 +255,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_backward_kernel(const __grid_c
         } else {
           const int32_t v0 = (int32_t)u * kBM;
           const int64_t r0 = (int64_t)kc * kKc;
-          sh->rid[lane] = w1_row_of(p, r0 + lane);
-          sh->rid[32 + lane] = w1_row_of(p, r0 + 32 + lane);
+          const int32_t* rsrc = rid_all + r0;
+          if (!p.rid_cached) {
+            sh->rid[lane] = w1_row_of(p, r0 + lane);
+            sh->rid[32 + lane] = w1_row_of(p, r0 + 32 + lane);
+            rsrc = sh->rid;
+          }
           if (lane == 0) {
             mbar_arrive_expect_tx(&sh->full[s], kStageBytes);
             tma_load_2d(st, &maps.g, &sh->full[s], v0, (int32_t)r0, pol_g);
@@ -232,10 +269,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_backward_kernel(const __grid_c
           __syncwarp();
           for (int i = lane; i < NA * (kKc / 4); i += 32) {
             const int c = i / (kKc / 4), j = i % (kKc / 4);
-            tma_gather4(st + kABytes + c * kBlockBytes + j * 512, &maps.w, &sh->full[s], c * 64, sh->rid[4 * j],
-                        sh->rid[4 * j + 1], sh->rid[4 * j + 2], sh->rid[4 * j + 3], pol_w);
+            tma_gather4(st + kABytes + c * kBlockBytes + j * 512, &maps.w, &sh->full[s], c * 64, rsrc[4 * j],
+                        rsrc[4 * j + 1], rsrc[4 * j + 2], rsrc[4 * j + 3], pol_w);
           }
-          __syncwarp();  // rid is rewritten for the next stage
+          __syncwarp();  // sh->rid is rewritten for the next stage
         }
       }
     }
@@ -291,7 +328,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_backward_kernel(const __grid_c
     const int row = 32 * q + lane;    // M index within the unit
     const uint32_t bar_id = 1;
     int64_t ui = 0;
-    uint32_t stores = 0;
     for (int64_t u = u_begin; u < u_end; ++u, ++ui) {
       const int abuf = (int)(ui & 1);
       const uint32_t par = (uint32_t)(ui >> 1) & 1u;
@@ -303,54 +339,100 @@ __global__ void __launch_bounds__(kThreads, 1) tc_backward_kernel(const __grid_c
       tc_fence_after_sync();
       const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(abuf * kN);
       float* dst = nullptr;
+      bool leader = false;
+      uint32_t others = 0;  // lanes whose sums this lane adds in before its atomics
+      uint32_t rounds = 0;
       if constexpr (DW1) {
         int32_t m, c0, c1;
         dw1_unit(p, u, m, c0, c1);
         const int64_t r = (int64_t)m * kBM + row;
+        int64_t id = -1;
         if (r < p.rows) {
-          const int64_t id = p.ids[r];
+          id = p.ids[r];
           if (id >= 0 && id < p.vocab)
             dst = p.dw1 + id * p.rank;
           else
-            report_status(p.status, DSPARK_STATUS_TOKEN_RANGE);
+            id = -1, report_status(p.status, DSPARK_STATUS_TOKEN_RANGE);
         }
-      }
+        // Rows of this warp with the same id are summed first (Zipf ids
+        // repeat), so one atomic per id and warp reaches L2: the lowest lane of
+        // each group pulls its peers' sums, one peer per round.
+        const uint32_t peers = __match_any_sync(0xffffffffu, (unsigned long long)id);
+        leader = (uint32_t)(__ffs(peers) - 1) == (uint32_t)lane;
+        others = leader ? (peers & ~(1u << lane)) : 0u;
+        rounds = __reduce_max_sync(0xffffffffu, (uint32_t)__popc(others));
 #pragma unroll 1
-      for (int c = 0; c < kN / 32; ++c) {
-        uint32_t acc[32];
-        tmem_ld_32x32b_x32(tb + c * 32, acc);
-        tmem_ld_wait();
-        if (c == kN / 32 - 1) {
-          tc_fence_before_sync();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sh->acc_empty[abuf]);
-        }
-        if constexpr (DW1) {
-          if (dst) {
+        for (int c = 0; c < kN / 32; ++c) {
+          uint32_t acc[32];
+          tmem_ld_32x32b_x32(tb + c * 32, acc);
+          tmem_ld_wait();
+          if (c == kN / 32 - 1) {
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh->acc_empty[abuf]);
+          }
+          uint32_t rest = others;
+          for (uint32_t k = 0; k < rounds; ++k) {
+            const int src = rest ? __ffs(rest) - 1 : lane;
+            rest &= rest - 1u;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float x = __shfl_sync(0xffffffffu, __uint_as_float(acc[e]), src);
+              if (src != lane) acc[e] = __float_as_uint(__uint_as_float(acc[e]) + x);
+            }
+          }
+          if (leader && dst) {
 #pragma unroll
             for (int k = 0; k < 8; ++k)
               red_add_v4(dst + c * 32 + 4 * k, acc[4 * k], acc[4 * k + 1], acc[4 * k + 2], acc[4 * k + 3]);
           }
-        } else {
-          // Staging box `stores & 1` is free once the store issued two boxes
-          // ago has read it.
-          if (stores >= 2 && et == 0) bulk_wait_group_read<1>();
-          named_barrier_sync(bar_id, 128);
-          uint8_t* box = out_smem + (stores & 1u) * kOutBoxBytes;
+        }
+      } else {
+        // Up to four 32-column chunks at a time: all are read from TMEM first
+        // (the accumulator is released as soon as the last group is in
+        // registers), staged in their own swizzled boxes and stored together.
+        constexpr int kChunks = kN / 32;
+        constexpr int kBoxes = out_boxes_of(NA);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            *reinterpret_cast<uint4*>(box + row * 128 + ((k ^ (row & 7)) << 4)) =
-                make_uint4(acc[4 * k], acc[4 * k + 1], acc[4 * k + 2], acc[4 * k + 3]);
+        for (int h = 0; h < kChunks; h += kBoxes) {
+          uint32_t acc[kBoxes][32];
+#pragma unroll
+          for (int cc = 0; cc < kBoxes; ++cc)
+            if (h + cc < kChunks) tmem_ld_32x32b_x32(tb + (h + cc) * 32, acc[cc]);
+          tmem_ld_wait();
+          if (h + kBoxes >= kChunks) {
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh->acc_empty[abuf]);
+          }
+          // The boxes are free once the stores issued from them have read them.
+          if (et == 0) bulk_wait_group_read<0>();
+          named_barrier_sync(bar_id, 128);
+#pragma unroll
+          for (int cc = 0; cc < kBoxes; ++cc) {
+            if (h + cc < kChunks) {
+              uint8_t* box = out_smem + cc * kOutBoxBytes + row * 128;
+#pragma unroll
+              for (int k = 0; k < 8; ++k)
+                *reinterpret_cast<uint4*>(box + ((k ^ (row & 7)) << 4)) =
+                    make_uint4(acc[cc][4 * k], acc[cc][4 * k + 1], acc[cc][4 * k + 2], acc[cc][4 * k + 3]);
+            }
+          }
           fence_proxy_async_smem();
           named_barrier_sync(bar_id, 128);
           if (et == 0) {
-            if (p.accumulate)
-              tma_reduce_add_2d(&maps.dw2, box, c * 32, (int32_t)u * kBM);
-            else
-              tma_store_2d(&maps.dw2, box, c * 32, (int32_t)u * kBM);
+#pragma unroll
+            for (int cc = 0; cc < kBoxes; ++cc) {
+              if (h + cc < kChunks) {
+                const uint8_t* box = out_smem + cc * kOutBoxBytes;
+                if (p.accumulate)
+                  tma_reduce_add_2d(&maps.dw2, box, (h + cc) * 32, (int32_t)u * kBM);
+                else
+                  tma_store_2d(&maps.dw2, box, (h + cc) * 32, (int32_t)u * kBM);
+              }
+            }
             bulk_commit_group();
           }
-          ++stores;
         }
       }
     }
@@ -410,8 +492,10 @@ cudaError_t launch_one(const BackwardArgs& a, int num_sms, uint64_t wait_limit_n
   } else {
     p.units = (int32_t)((a.vocab + kBM - 1) / kBM);
     p.k_stages = (int32_t)((a.rows + kKc - 1) / kKc);
+    p.rid_cached = a.rows <= kRidCacheRows ? p.k_stages * kKc : 0;
   }
-  const size_t fixed = 1024 + sizeof(BwdShared) + 64 + (DW1 ? 0 : 2 * kOutBoxBytes);
+  const size_t fixed =
+      1024 + sizeof(BwdShared) + (size_t)p.rid_cached * 4 + 64 + (DW1 ? 0 : out_boxes_of(NA) * kOutBoxBytes);
   int stages = (int)((kSmemLimit - fixed) / stage_bytes_of(NA, DW1));
   if (stages > kMaxStages) stages = kMaxStages;
   p.stages = stages;
