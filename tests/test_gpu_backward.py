@@ -140,6 +140,7 @@ def test_backward_fp32_and_accumulate():
     """fp32 operands (CUDA-core kernels), and accumulate = True adds onto
     given buffers."""
     w1, w2, dout, ids = _inputs(50, 1024, 16, seed=3, ldt=torch.float32, wdt=torch.float32)
+    set_algo(N.DSPARK_ALGO_AUTO)
     head = VanillaMarkov(w1.cuda(), w2.cuda())
     b1 = torch.full((1024, 16), 0.5, device="cuda")
     b2 = torch.full((1024, 16), -0.25, device="cuda")
