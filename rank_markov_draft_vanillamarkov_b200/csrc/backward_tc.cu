@@ -18,7 +18,9 @@
 // stages of 64. Per stage the producer warp loads two 64-id boxes of G (the
 // A operand, MN-major) and gathers the stage's 64 W1 rows with tile::gather4
 // (the B operand, MN-major; invalid ids and rows past the end read row
-// `vocab`, outside the tensor, i.e. zeros). The epilogue writes the fp32 tile
+// `vocab`, outside the tensor, i.e. zeros). When all rows' W1 rows fit in
+// shared memory beside three stages, they are gathered once per CTA instead
+// (RES), and a stage carries only the G boxes. The epilogue writes the fp32 tile
 // through up to four swizzled 32-column staging boxes with TMA stores, or TMA
 // reduce-adds when accumulating.
 //
@@ -125,6 +127,7 @@ struct BwdParams {
 struct BwdShared {
   uint64_t full[kMaxStages], empty[kMaxStages];
   uint64_t acc_full[2], acc_empty[2];
+  uint64_t w1_full;  // dW2 with resident W1 rows: the one-time gather
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -151,16 +154,22 @@ __device__ __forceinline__ void dw1_unit(const BwdParams& p, int64_t u, int32_t&
   c1 = (int32_t)((int64_t)p.chunks * (s + 1) / p.splits);
 }
 
-template <int NA, bool DW1>
+// RES (dW2 only): the W1 rows of all rows are gathered once per CTA into a
+// resident MN-major B operand (rank/64 blocks of rid_cached 128-byte rows),
+// and a stage carries only the two G boxes.
+template <int NA, bool DW1, bool RES>
 __global__ void __launch_bounds__(kThreads, 1) tc_backward_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
+  static_assert(!(DW1 && RES), "resident W1 rows are a dW2 layout");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int kN = NA * 64;
   constexpr uint32_t kABytes = a_bytes_of(DW1);
-  constexpr uint32_t kStageBytes = stage_bytes_of(NA, DW1);
+  constexpr uint32_t kStageBytes = RES ? kABytes : stage_bytes_of(NA, DW1);
   constexpr uint32_t kTmemCols = tmem_cols_of(NA);
   uint8_t* stage_smem = smem;
-  uint8_t* out_smem = smem + (size_t)p.stages * kStageBytes;  // dW2: staging boxes
+  uint8_t* w1_res = smem + (size_t)p.stages * kStageBytes;  // RES: NA blocks of rid_cached rows
+  const uint32_t res_block = RES ? (uint32_t)p.rid_cached * 128u : 0u;
+  uint8_t* out_smem = w1_res + (size_t)NA * res_block;  // dW2: staging boxes
   BwdShared* sh = reinterpret_cast<BwdShared*>(out_smem + (DW1 ? 0 : out_boxes_of(NA) * kOutBoxBytes));
   int32_t* rid_all = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(sh) + sizeof(BwdShared));
 
@@ -178,6 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_backward_kernel(const __grid_c
       mbar_init(&sh->acc_full[i], 1);
       mbar_init(&sh->acc_empty[i], 4);  // one arrival per epilogue warp
     }
+    mbar_init(&sh->w1_full, 1);
     mbar_init(&sh->drain, 1);
     sh->abort_flag = 0;
     fence_barrier_init();
@@ -231,6 +241,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_backward_kernel(const __grid_c
         }
       }
       __syncwarp();
+      if constexpr (RES) {
+        const int quads = p.rid_cached / 4;
+        if (lane == 0) mbar_arrive_expect_tx(&sh->w1_full, (uint32_t)NA * res_block);
+        __syncwarp();
+        for (int i = lane; i < NA * quads; i += 32) {
+          const int c = i / quads, j = i % quads;
+          tma_gather4(w1_res + (size_t)c * res_block + j * 512, &maps.w, &sh->w1_full, c * 64, rid_all[4 * j],
+                      rid_all[4 * j + 1], rid_all[4 * j + 2], rid_all[4 * j + 3], pol_w);
+        }
+        __syncwarp();
+      }
     }
     uint32_t it = 0;
     bool ok = true;
@@ -255,6 +276,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_backward_kernel(const __grid_c
         } else {
           const int32_t v0 = (int32_t)u * kBM;
           const int64_t r0 = (int64_t)kc * kKc;
+          if constexpr (RES) {
+            if (lane == 0) {
+              mbar_arrive_expect_tx(&sh->full[s], kStageBytes);
+              tma_load_2d(st, &maps.g, &sh->full[s], v0, (int32_t)r0, pol_g);
+              tma_load_2d(st + kBlockBytes, &maps.g, &sh->full[s], v0 + 64, (int32_t)r0, pol_g);
+            }
+            __syncwarp();
+            continue;
+          }
           const int32_t* rsrc = rid_all + r0;
           if (!p.rid_cached) {
             sh->rid[lane] = w1_row_of(p, r0 + lane);
@@ -280,15 +310,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_backward_kernel(const __grid_c
     if (lane == 0) {
       const uint32_t S = (uint32_t)p.stages;
       for (uint32_t j = it > S ? it - S : 0; j < it; ++j) mbar_wait(&sh->full[j % S], (j / S) & 1u, drain_ctl);
+      if (RES) mbar_wait(&sh->w1_full, 0, drain_ctl);
     }
   } else if (warp == 1) {
     // ------------------------------------------------- MMA issuer -----
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(kBM, kN) | kBMnMajor | (DW1 ? 0u : kAMnMajor);
       const uint32_t stage_addr = smem_u32(stage_smem);
+      const uint32_t res_addr = smem_u32(w1_res);
       uint32_t it = 0;
       int64_t ui = 0;
-      bool ok = true;
+      bool ok = !RES || mbar_wait(&sh->w1_full, 0, ctl);
       for (int64_t u = u_begin; u < u_end && ok; ++u, ++ui) {
         int32_t m = 0, c0 = 0, c1 = p.k_stages;
         if constexpr (DW1) dw1_unit(p, u, m, c0, c1);
@@ -304,14 +336,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_backward_kernel(const __grid_c
           }
           tc_fence_after_sync();
           const uint32_t a_addr = stage_addr + (uint32_t)s * kStageBytes;
-          const uint32_t b_addr = a_addr + kABytes;
+          // B: this stage's rows of the resident block, or the stage's own gather.
+          const uint32_t b_addr = RES ? res_addr + (uint32_t)kc * kBlockBytes : a_addr + kABytes;
+          const uint32_t b_stride = RES ? res_block : kBlockBytes;
 #pragma unroll
           for (int kk = 0; kk < kKc / 16; ++kk) {
             // K = 16 per instruction: 32 bytes along a K-major row, or two
             // 8-row groups (2048 bytes) of an MN-major block.
             const uint64_t ad = DW1 ? sw128_kmajor_desc(a_addr + kk * 32)
                                     : sw128_mnmajor_desc(a_addr + kk * 2048, kBlockBytes);
-            const uint64_t bd = sw128_mnmajor_desc(b_addr + kk * 2048, kBlockBytes);
+            const uint64_t bd = sw128_mnmajor_desc(b_addr + kk * 2048, b_stride);
             umma_bf16_ss(d_tmem, ad, bd, idesc, (kc != c0 || kk != 0) ? 1u : 0u);
           }
           umma_commit(&sh->empty[s]);
@@ -446,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_backward_kernel(const __grid_c
   if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
 }
 
-template <int NA, bool DW1>
+template <int NA, bool DW1, bool RES>
 cudaError_t launch_one(const BackwardArgs& a, int num_sms, uint64_t wait_limit_ns, cudaStream_t stream) {
   BwdMaps maps;
   const uint64_t gdim[2] = {(uint64_t)a.vocab, (uint64_t)a.rows};
@@ -494,14 +528,16 @@ cudaError_t launch_one(const BackwardArgs& a, int num_sms, uint64_t wait_limit_n
     p.k_stages = (int32_t)((a.rows + kKc - 1) / kKc);
     p.rid_cached = a.rows <= kRidCacheRows ? p.k_stages * kKc : 0;
   }
-  const size_t fixed =
-      1024 + sizeof(BwdShared) + (size_t)p.rid_cached * 4 + 64 + (DW1 ? 0 : out_boxes_of(NA) * kOutBoxBytes);
-  int stages = (int)((kSmemLimit - fixed) / stage_bytes_of(NA, DW1));
+  const size_t stage_bytes = RES ? a_bytes_of(false) : stage_bytes_of(NA, DW1);
+  const size_t fixed = 1024 + sizeof(BwdShared) + (size_t)p.rid_cached * 4 + 64 +
+                       (DW1 ? 0 : out_boxes_of(NA) * kOutBoxBytes) + (RES ? (size_t)NA * p.rid_cached * 128 : 0);
+  if (fixed + 2 * stage_bytes > kSmemLimit) return cudaErrorInvalidValue;
+  int stages = (int)((kSmemLimit - fixed) / stage_bytes);
   if (stages > kMaxStages) stages = kMaxStages;
   p.stages = stages;
-  const size_t smem = fixed + (size_t)stages * stage_bytes_of(NA, DW1);
+  const size_t smem = fixed + (size_t)stages * stage_bytes;
 
-  auto kernel = tc_backward_kernel<NA, DW1>;
+  auto kernel = tc_backward_kernel<NA, DW1, RES>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int grid = p.units < num_sms ? p.units : num_sms;
@@ -513,8 +549,16 @@ cudaError_t launch_one(const BackwardArgs& a, int num_sms, uint64_t wait_limit_n
 template <int NA>
 cudaError_t launch_na(const BackwardArgs& a, int num_sms, uint64_t wait_limit_ns, cudaStream_t s) {
   cudaError_t e = cudaSuccess;
-  if (a.grad_w2) e = launch_one<NA, false>(a, num_sms, wait_limit_ns, s);
-  if (e == cudaSuccess && a.grad_w1) e = launch_one<NA, true>(a, num_sms, wait_limit_ns, s);
+  if (a.grad_w2) {
+    // Resident W1 rows when they fit beside at least three G stages.
+    const int64_t kpad = (a.rows + kKc - 1) / kKc * kKc;
+    const size_t res_fixed = 1024 + sizeof(BwdShared) + (size_t)kpad * 4 + 64 + out_boxes_of(NA) * kOutBoxBytes +
+                             (size_t)NA * kpad * 128;
+    const bool res = a.rows <= kRidCacheRows && res_fixed + 3 * (size_t)a_bytes_of(false) <= kSmemLimit;
+    e = res ? launch_one<NA, false, true>(a, num_sms, wait_limit_ns, s)
+            : launch_one<NA, false, false>(a, num_sms, wait_limit_ns, s);
+  }
+  if (e == cudaSuccess && a.grad_w1) e = launch_one<NA, true, false>(a, num_sms, wait_limit_ns, s);
   return e;
 }
 
