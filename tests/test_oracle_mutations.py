@@ -130,3 +130,84 @@ def test_backward_overwriting_repeated_ids_is_caught(monkeypatch):
         return dw1, dout.T @ emb
     monkeypatch.setattr(oracle, "apply_block_logits_backward", wrong)
     _fails(pins.test_backward_matches_torch_autograd)
+
+
+# ---------------------------------------------------------------------------
+# The comparison rules (oracle/checks.py): each planted mistake makes a
+# checker pin fail.
+# ---------------------------------------------------------------------------
+from oracle import checks as oc  # noqa: E402
+
+
+def test_logit_rule_needing_only_one_clause_is_caught(monkeypatch):
+    """`or` in place of `and`: a value breaking only one clause passes."""
+    def either(got, exact, acc):
+        lo, hi = oc.bf16_allowed_interval(exact, acc)
+        near_rounding = (got >= lo) & (got <= hi)
+        near_exact = np.abs(got - exact) <= oc.LOGIT_ABS_TOL_BF16 + 0.5 * oracle.ulp_bfloat16(exact)
+        return ~(near_rounding | near_exact)
+    monkeypatch.setattr(oc, "bf16_logit_bad", either)
+    _fails(pins.test_check_logits_rejects_two_ulps_off)
+    _fails(pins.test_check_logits_rejects_a_value_far_from_the_exact_sum_inside_the_rounding_window)
+
+
+def test_logit_rule_of_one_ulp_around_the_rounded_sum_is_caught(monkeypatch):
+    """The looser rule |got - RNE(exact)| <= 1 ulp lets truncation through."""
+    def one_ulp(got, exact, acc):
+        rne = oracle.round_to_bfloat16(exact)
+        ulp = oracle.ulp_bfloat16(exact)
+        return (np.abs(got - rne) > ulp + acc) | (np.abs(got - exact) > oc.LOGIT_ABS_TOL_BF16 + 0.5 * ulp)
+    monkeypatch.setattr(oc, "bf16_logit_bad", one_ulp)
+    _fails(pins.test_check_logits_rejects_truncation_away_from_a_halfway_point)
+
+
+def test_loosened_fp32_rule_is_caught(monkeypatch):
+    monkeypatch.setattr(oc, "fp32_logit_bad", lambda got, exact: ~(np.abs(got - exact) <= 1e-3))
+    _fails(pins.test_check_logits_fp32_bound)
+
+
+def test_flipped_token_margin_is_caught(monkeypatch):
+    """Exact match demanded at near-ties and top-window membership above the
+    margin (the comparison turned around)."""
+    def flipped(scores, dev, exact_only):
+        scores = np.asarray(scores, dtype=np.float64)
+        t1 = int(np.argmax(scores))
+        mask = np.zeros(scores.shape, dtype=bool)
+        mask[t1] = True
+        window = np.maximum(oc.TOKEN_MARGIN, dev[t1] + dev)
+        mask |= (scores[t1] - scores) > window
+        return mask
+    monkeypatch.setattr(oc, "acceptable_tokens", flipped)
+    _fails(pins.test_near_tie_accepts_the_runner_up_and_rejects_the_third)
+    _fails(pins.test_wrong_token_above_the_margin_is_rejected, 0.0)
+
+
+def test_token_window_without_the_rounding_deviation_is_caught(monkeypatch):
+    """A fixed 1e-2 window rejects the legitimate one-ulp flip at |x| >= 8."""
+    monkeypatch.setattr(oc, "rounding_deviation", lambda exact, acc, dtype: np.zeros(np.shape(exact)))
+    _fails(pins.test_one_ulp_flip_at_large_logits_is_accepted_only_near_a_halfway_point)
+
+
+@pytest.mark.parametrize("scale", [2.0 ** -20, 2.0 ** 20])
+def test_accumulation_bound_off_by_a_power_of_two_is_caught(monkeypatch, scale):
+    real = oc.accumulation_bound
+    monkeypatch.setattr(oc, "accumulation_bound", lambda *a: real(*a) * scale)
+    _fails(pins.test_accumulation_bound_is_attained_within_a_factor_of_three)
+
+
+def test_accumulation_bound_without_the_base_term_is_caught(monkeypatch):
+    """Dropping |U| from the bound: sums where U dominates break it."""
+    real = oc.accumulation_bound
+    monkeypatch.setattr(oc, "accumulation_bound",
+                        lambda base, w1, w2, ids: real(np.zeros_like(np.asarray(base, float)), w1, w2, ids))
+    _fails(pins.test_accumulation_bound_is_attained_within_a_factor_of_three)
+
+
+@pytest.mark.parametrize("wrong", ["first", "same step"])
+def test_checker_teacher_forced_on_the_wrong_token_is_caught(monkeypatch, wrong):
+    if wrong == "first":
+        monkeypatch.setattr(oc, "teacher_forced_prev", lambda first, toks, rows, k: first[rows])
+    else:
+        monkeypatch.setattr(oc, "teacher_forced_prev",
+                            lambda first, toks, rows, k: first[rows] if k == 0 else toks[rows, k])
+    _fails(pins.test_chain_is_checked_against_its_own_previous_tokens)

@@ -395,3 +395,269 @@ def test_chain_joint_distribution_bigram():
     obs = np.append(counts[keep], counts[~keep].sum())
     exp = np.append(p[keep] * rows, p[~keep].sum() * rows)
     assert stats.chisquare(obs, exp).pvalue > 1e-3
+
+
+# --------------------------------------------------------------------------
+# The comparison rules (oracle/checks.py) that every GPU parity test uses.
+# Each rule is pinned from both sides: values a correct implementation may
+# return are accepted, and each plausible kind of wrong value is rejected.
+# --------------------------------------------------------------------------
+from oracle import checks as oc  # noqa: E402
+
+
+def _bf16(x):
+    return oracle.round_to_bfloat16(np.asarray(x, float))
+
+
+def test_check_logits_accepts_one_rounding_of_any_sum_within_the_bound():
+    """A correct kernel returns RNE(e) for some fp32 sum e within acc of the
+    exact sum; every such value is accepted, at every magnitude."""
+    rng = np.random.default_rng(20)
+    exact = rng.standard_normal(40_000) * np.repeat([0.01, 0.3, 3.0, 12.0, 40.0, 0.5], [8000, 8000, 8000, 8000,
+                                                                                         4000, 4000])
+    acc = np.abs(exact) * 2.0 ** -18 + 1e-9
+    for e in (exact + acc * rng.uniform(-1, 1, exact.shape), exact + acc, exact - acc, exact):
+        rep = oc.check_logits(_bf16(e), exact, "bf16", acc)
+        assert rep.ok, rep
+
+
+def test_check_logits_rejects_two_ulps_off():
+    """Clause 1 alone: near |x| = 0.3 two bf16 ulps are 4e-3, well inside the
+    2e-2 max-abs bound, and must still be rejected."""
+    exact = np.linspace(0.26, 0.49, 64)
+    acc = np.full_like(exact, 1e-7)
+    got = _bf16(exact) + 2 * oracle.ulp_bfloat16(exact)
+    assert np.all(np.abs(got - exact) < oc.LOGIT_ABS_TOL_BF16)
+    assert oc.check_logits(got, exact, "bf16", acc).bad == exact.size
+
+
+def test_check_logits_rejects_truncation_away_from_a_halfway_point():
+    """Truncating instead of rounding is one ulp off where the exact sum is
+    clearly above the halfway point (0.8 of the way to the next value)."""
+    lo = 1.0 + np.arange(1, 100) * 2.0 ** -7
+    exact = lo + 0.8 * 2.0 ** -7
+    acc = np.full_like(exact, 1e-6)
+    assert np.all(_bf16(exact) == lo + 2.0 ** -7)
+    assert oc.check_logits(lo, exact, "bf16", acc).bad == exact.size
+
+
+def test_check_logits_allows_the_other_neighbour_only_near_a_halfway_point():
+    """Within acc of a halfway point both neighbours are one rounding of an
+    allowed sum; farther away only the nearer one is."""
+    lo = 1.0 + np.arange(1, 100) * 2.0 ** -7
+    hi = lo + 2.0 ** -7
+    half = lo + 2.0 ** -8
+    acc = np.full_like(half, 1e-6)
+    near = half + 0.5e-6
+    assert oc.check_logits(lo, near, "bf16", acc).ok and oc.check_logits(hi, near, "bf16", acc).ok
+    far = half + 3e-6
+    assert oc.check_logits(hi, far, "bf16", acc).ok
+    assert oc.check_logits(lo, far, "bf16", acc).bad == far.size
+
+
+def test_check_logits_rejects_a_value_far_from_the_exact_sum_inside_the_rounding_window():
+    """Clause 2 alone. Where U and the bias cancel, acc is large and clause 1
+    admits a wide window, yet the value must stay within 2e-2 (+ ulp/2) of
+    the exact sum; so must a value one ulp from the rounded sum at
+    |x| in [4, 8), where that ulp is 1/32."""
+    exact = np.array([1e-3, -2e-3, 4e-3])
+    acc = np.full(3, 0.06)
+    got = _bf16(exact + 0.035)
+    lo, hi = oc.bf16_allowed_interval(exact, acc)
+    assert np.all((got >= lo) & (got <= hi))
+    assert oc.check_logits(got, exact, "bf16", acc).bad == 3
+    exact = np.array([5.0 + 0.4 * 2.0 ** -5])
+    got = np.array([5.0 - 2.0 ** -5])
+    acc = np.array([0.05])
+    lo, hi = oc.bf16_allowed_interval(exact, acc)
+    assert lo[0] <= got[0] <= hi[0]
+    assert abs(got[0] - exact[0]) > 3e-2
+    assert oc.check_logits(got, exact, "bf16", acc).bad == 1
+
+
+def test_check_logits_fp32_bound():
+    rng = np.random.default_rng(21)
+    exact = rng.standard_normal(1000) * 3
+    assert oc.check_logits(exact + 5e-5, exact, "fp32").ok
+    assert oc.check_logits(exact + 2e-4, exact, "fp32").bad == exact.size
+    assert oc.check_logits(exact - 2e-4, exact, "fp32").bad == exact.size
+
+
+def test_check_logits_nan_and_infinities():
+    exact = np.array([1.0, np.inf, -np.inf, np.nan, 2.0])
+    acc = np.zeros(5)
+    assert oc.check_logits(exact.copy(), exact, "bf16", acc).ok
+    for i, wrong in ((0, np.nan), (1, 3.0), (2, np.inf), (3, 1.0)):
+        got = exact.copy()
+        got[i] = wrong
+        rep = oc.check_logits(got, exact, "bf16", acc)
+        assert rep.bad == 1 and rep.first_bad == (i,), (i, rep)
+
+
+def _strong_block(seed, b=6, m=4, v=300, r=32, std=0.3, dtype="bf16"):
+    rng = np.random.default_rng(seed)
+    rnd = (lambda x: _bf16(x)) if dtype == "bf16" else oracle.round_to_float32
+    base = rnd(rng.standard_normal((b, m, v)) * 2)
+    w1, w2 = rnd(rng.standard_normal((v, r)) * std), rnd(rng.standard_normal((v, r)) * std)
+    return base, w1, w2, rng.integers(0, v, b)
+
+
+def test_dropped_bias_is_rejected_at_strong_weights():
+    """With weights ~N(0, 0.3) the bias has std ~1.7; returning the base
+    logits (bias skipped) fails the logits rule almost everywhere, in both
+    the teacher-forced and the sampled form."""
+    base, w1, w2, first = _strong_block(23)
+    ids = np.random.default_rng(24).integers(0, 300, base.shape[:2])
+    exact = oracle.markov.exact_block_logits(base, w1, w2, ids)
+    acc = oc.accumulation_bound(base, w1, w2, ids)
+    assert oc.check_logits(_bf16(exact), exact, "bf16", acc).ok
+    assert oc.check_logits(base, exact, "bf16", acc).bad > 0.9 * base.size
+    toks = np.argmax(base, axis=-1)
+    rep = oc.check_sampled_block(toks, base, base, w1, w2, first, "bf16", 0.0, 0)
+    assert not rep.ok and rep.logits.bad > 0.9 * base.size
+
+
+@pytest.mark.parametrize("dtype,temp", [("bf16", 0.0), ("bf16", 0.8), ("fp32", 0.0), ("fp32", 1.3)])
+def test_oracle_output_passes_the_check(dtype, temp):
+    base, w1, w2, first = _strong_block(25, dtype=dtype)
+    toks, corr = oracle.sample_block_tokens(base, w1, w2, first, dtype, temp, seed=5)
+    rep = oc.check_sampled_block(toks, corr, base, w1, w2, first, dtype, temp, 5)
+    assert rep.ok and rep.exact_required > 0, rep
+
+
+def _top2_gap(s):
+    o = np.sort(s)[::-1]
+    return o[0] - o[1]
+
+
+@pytest.mark.parametrize("temp", [0.0, 0.8])
+def test_wrong_token_above_the_margin_is_rejected(temp):
+    """At the last step (nothing later depends on it) of a row whose
+    top-1/top-2 score gap exceeds 5e-2, the runner-up is rejected; the
+    logits stay correct, so exactly one token is counted bad."""
+    base, w1, w2, first = _strong_block(26)
+    toks, corr = oracle.sample_block_tokens(base, w1, w2, first, "bf16", temp, seed=3)
+    k = base.shape[1] - 1
+    for b in range(base.shape[0]):
+        c = corr[b, k]
+        s = c if temp == 0.0 else oracle.temperature_scores(c, temp, 3, b, k)
+        if _top2_gap(s) > 5e-2:
+            break
+    else:
+        pytest.fail("no row with a clear margin")
+    wrong = toks.copy()
+    wrong[b, k] = int(np.argsort(s)[::-1][1])
+    rep = oc.check_sampled_block(wrong, corr, base, w1, w2, first, "bf16", temp, 3)
+    assert rep.logits.ok and rep.bad == 1
+
+
+def test_near_tie_accepts_the_runner_up_and_rejects_the_third():
+    """W2 = 0 makes the corrected logits the base logits. Margin 2^-7 (below
+    1e-2): the runner-up is accepted, an id 0.5 below is not. Margin 2^-6
+    (above 1e-2): the runner-up is rejected too."""
+    v = 64
+    w1, w2 = np.zeros((v, 4)), np.zeros((v, 4))
+    for gap, runner_ok in ((2.0 ** -7, True), (2.0 ** -6, False)):
+        base = np.zeros((1, 1, v))
+        base[0, 0, 40] = 1.5
+        base[0, 0, 7] = 1.5 - gap
+        base[0, 0, 20] = 1.0
+        for tok, ok in ((40, True), (7, runner_ok), (20, False)):
+            rep = oc.check_sampled_block(np.array([[tok]]), base, base, w1, w2, np.array([0]), "bf16", 0.0, 0)
+            assert (rep.bad == 0) == ok, (gap, tok, rep)
+
+
+def test_one_ulp_flip_at_large_logits_is_accepted_only_near_a_halfway_point():
+    """At |x| >= 8 a bf16 ulp (1/16) exceeds 1e-2. Id 0's exact sum lies just
+    below the halfway point between 10 and 10 + 1/16, so the oracle rounds it
+    to 10 and picks id 1 (10 + 1/16). Within the accumulation bound of that
+    point a correct kernel may round id 0 up instead, tie, and pick id 0 (the
+    lower index): accepted. Farther from the point it may not: rejected."""
+    w1 = np.ones((2, 1))
+    base = np.array([[[10.0, 10.0625]]])
+    for delta, ok in ((1e-6, True), (1e-5, False)):
+        w2 = np.array([[2.0 ** -5 - delta], [0.0]])
+        acc = oc.accumulation_bound(base[:, 0], w1, w2, [0])[0, 0]
+        assert (delta < acc) == ok
+        oracle_c = np.array([[[10.0, 10.0625]]])
+        flipped_c = np.array([[[10.0625, 10.0625]]])
+        rep = oc.check_sampled_block(np.array([[0]]), oracle_c, base, w1, w2, np.array([0]), "bf16", 0.0, 0)
+        assert rep.logits.ok and (rep.bad == 0) == ok, (delta, rep)
+        rep = oc.check_sampled_block(np.array([[0]]), flipped_c, base, w1, w2, np.array([0]), "bf16", 0.0, 0)
+        assert rep.ok == ok, (delta, rep)
+
+
+def test_chain_is_checked_against_its_own_previous_tokens():
+    """With a strong bias the chain's own tokens decide later steps. The
+    oracle's chain passes; a chain that fed back nothing (first_prev at every
+    step) or a token two steps old fails."""
+    base, w1, w2, first = _strong_block(27, m=5)
+    toks, corr = oracle.sample_block_tokens(base, w1, w2, first, "bf16", 0.0)
+    assert oc.check_sampled_block(toks, corr, base, w1, w2, first, "bf16", 0.0, 0).ok
+    m = base.shape[1]
+    for stale in ("none", "two back"):
+        prev = first.copy()
+        wt, wc = np.zeros_like(toks), np.zeros_like(corr)
+        for k in range(m):
+            if stale == "none":
+                p = first
+            else:
+                p = first if k < 2 else wt[:, k - 2]
+            wc[:, k] = oracle.apply_step_logits(base[:, k], w1, w2, p, "bf16")
+            wt[:, k] = np.argmax(wc[:, k], axis=-1)
+        assert not np.array_equal(wt, toks), stale  # the test has power
+        rep = oc.check_sampled_block(wt, wc, base, w1, w2, first, "bf16", 0.0, 0)
+        assert not rep.ok, stale
+
+
+def _fp32_sum(terms):
+    s = np.zeros(terms[0].shape, np.float32)
+    for t in terms:
+        s = (s + t).astype(np.float32)
+    return s
+
+
+def test_accumulation_bound_covers_fp32_sums_in_several_orders():
+    """Recursive fp32 sums of U and the r exact products, in the orders a
+    kernel may use (U first or last, forward, reversed, numpy's pairwise sum,
+    16-term blocks as a tensor-core K step, a fixed shuffle), with and without
+    cancellation, all stay within the bound."""
+    rng = np.random.default_rng(28)
+    v, r, rows = 256, 128, 8
+    w1, w2 = _bf16(rng.standard_normal((v, r)) * 0.3), _bf16(rng.standard_normal((v, r)) * 0.3)
+    ids = rng.integers(0, v, rows)
+    bias = w1[ids] @ w2.T
+    for base in (_bf16(rng.standard_normal((rows, v)) * 2), -_bf16(bias)):
+        exact = base + bias
+        bound = oc.accumulation_bound(base, w1, w2, ids)
+        prods = [(w1[ids, j][:, None].astype(np.float32) * w2[None, :, j].astype(np.float32)) for j in range(r)]
+        u32 = base.astype(np.float32)
+        perm = rng.permutation(r)
+        sums = {
+            "u first": _fp32_sum([u32] + prods),
+            "u last": _fp32_sum(prods + [u32]),
+            "reversed": _fp32_sum([u32] + prods[::-1]),
+            "pairwise": (np.sum(np.stack(prods), axis=0, dtype=np.float32) + u32).astype(np.float32),
+            "blocks of 16": _fp32_sum([u32] + [np.sum(np.stack(prods[i:i + 16]), axis=0, dtype=np.float32)
+                                               for i in range(0, r, 16)]),
+            "shuffled": _fp32_sum([prods[j] for j in perm] + [u32]),
+        }
+        for name, s in sums.items():
+            err = np.abs(s.astype(np.float64) - exact)
+            assert np.all(err <= bound), (name, float((err / bound).max()))
+
+
+def test_accumulation_bound_is_attained_within_a_factor_of_three():
+    """U = 1 and r products of 2^-24 (W1 = W2 = 2^-12): each fp32 addition of
+    2^-24 to 1 is a halfway case that rounds to even, back to 1, so the
+    recursive sum loses every product. The error r 2^-24 is reached, and the
+    bound, about 2 (r + 1) 2^-24, is no more than three times it."""
+    r = 64
+    w1 = np.full((1, r), 2.0 ** -12)
+    w2 = np.full((1, r), 2.0 ** -12)
+    u = np.array([[1.0]])
+    s = _fp32_sum([u.astype(np.float32)] + [np.full((1, 1), 2.0 ** -24, np.float32)] * r)
+    assert s[0, 0] == 1.0
+    err = abs(float(s[0, 0]) - (1.0 + r * 2.0 ** -24))
+    bound = float(oc.accumulation_bound(u, w1, w2, [0])[0, 0])
+    assert err <= bound <= 3 * err, (err, bound)
