@@ -15,6 +15,8 @@ from .markov import (  # noqa: F401
     apply_block_logits_backward,
     apply_step_logits,
     compute_step_bias,
+    fused_lm_head_exact,
+    fused_lm_head_logits,
     get_prev_embeddings,
     project_bias,
     sample_block_tokens,
@@ -25,4 +27,5 @@ from .markov import (  # noqa: F401
 )
 from .philox import gumbel_noise, noise_words, philox4x32, uniform_from_word  # noqa: F401
 from .rounding import round_to, round_to_bfloat16, round_to_float32, ulp_bfloat16  # noqa: F401
-from .checks import accumulation_bound, check_logits, check_sampled_block, check_tokens  # noqa: F401
+from .checks import (accumulation_bound, check_logits, check_sampled_block, check_tokens,  # noqa: F401
+                     fused_accumulation_bound)

@@ -87,6 +87,21 @@ def accumulation_bound(base, w1, w2, token_ids) -> np.ndarray:
     return ((r + 1) * 2.0 ** -23 * (base.reshape(-1, v) + mag)).reshape(base.shape)
 
 
+def fused_accumulation_bound(hidden, lm_head, w1, w2, token_ids) -> np.ndarray:
+    """The same bound for the fused producer's sums, whose d + r products
+    are hidden[i, j] lm_head[v, j] and W1[x_i, j] W2[v, j]:
+    (d + r + 1) * 2^-23 * (sum_j |h lm| + sum_j |W1 W2|)."""
+    h = np.abs(np.asarray(hidden, dtype=np.float64))
+    d = h.shape[-1]
+    lead = h.shape[:-1]
+    mag_u = h.reshape(-1, d) @ np.abs(np.asarray(lm_head, dtype=np.float64)).T
+    ids = np.asarray(token_ids, dtype=np.int64).reshape(-1)
+    a = np.abs(np.asarray(w1, dtype=np.float64)[ids])
+    mag_b = a @ np.abs(np.asarray(w2, dtype=np.float64)).T
+    r = a.shape[-1]
+    return ((d + r + 1) * 2.0 ** -23 * (mag_u + mag_b)).reshape(lead + (mag_u.shape[-1],))
+
+
 def bf16_allowed_interval(exact, acc):
     """Clause 1: the bf16 values a correct one-rounding implementation may
     return for exact sums ``exact`` computed with error at most ``acc``."""

@@ -128,6 +128,27 @@ def apply_block_logits_backward(grad_out, w1, w2, token_ids):
     return dw1, dw2
 
 
+def fused_lm_head_exact(hidden, lm_head, w1, w2, token_ids) -> np.ndarray:
+    """The unrounded corrected logits with the base logits produced in the
+    same pass, in fp64: U = hidden @ lm_head^T (the backbone's base logit,
+    "lm_head(hidden_k)" in the module docstring of markov_head.py; the frozen
+    vocabulary head of DeepseekV41DSparkModel.compute_logits, whose weight is
+    [vocab, hidden]) plus the transition bias of each row's previous token.
+    ``hidden`` is (..., d), ``token_ids`` (...); returns (..., V)."""
+    h = np.asarray(hidden, dtype=np.float64)
+    lm = np.asarray(lm_head, dtype=np.float64)
+    lead = h.shape[:-1]
+    ids = np.asarray(token_ids, dtype=np.int64).reshape(-1)
+    u = h.reshape(-1, h.shape[-1]) @ lm.T
+    return (u + compute_step_bias(w1, w2, ids)).reshape(lead + (lm.shape[0],))
+
+
+def fused_lm_head_logits(hidden, lm_head, w1, w2, token_ids, out_dtype: str) -> np.ndarray:
+    """``fused_lm_head_exact`` rounded once to ``out_dtype`` (compute_logits
+    returns FP32; the head then adds its bias in that dtype)."""
+    return round_to(out_dtype, fused_lm_head_exact(hidden, lm_head, w1, w2, token_ids))
+
+
 def select_greedy(logits: np.ndarray) -> np.ndarray:
     """argmax over the last axis; the lowest index wins among equal maxima and
     NaN counts as the largest value (numpy's argmax has both properties)."""

@@ -211,3 +211,25 @@ def test_checker_teacher_forced_on_the_wrong_token_is_caught(monkeypatch, wrong)
         monkeypatch.setattr(oc, "teacher_forced_prev",
                             lambda first, toks, rows, k: first[rows] if k == 0 else toks[rows, k])
     _fails(pins.test_chain_is_checked_against_its_own_previous_tokens)
+
+
+def test_fused_producer_without_the_bias_is_caught(monkeypatch):
+    monkeypatch.setattr(om, "fused_lm_head_exact",
+                        lambda h, lm, w1, w2, ids: np.asarray(h, float) @ np.asarray(lm, float).T)
+    _fails(pins.test_fused_producer_reduces_to_the_pinned_head)
+
+
+def test_fused_producer_with_a_transposed_lm_head_is_caught(monkeypatch):
+    real = om.fused_lm_head_exact
+    monkeypatch.setattr(om, "fused_lm_head_exact",
+                        lambda h, lm, w1, w2, ids: real(h, np.asarray(lm, float).T, w1, w2, ids))
+    _fails(pins.test_fused_producer_explicit_sums)
+
+
+def test_fused_producer_rounding_u_first_is_caught(monkeypatch):
+    """Base logits rounded to fp32 before the bias is added (two roundings)."""
+    def twice(h, lm, w1, w2, ids):
+        u = oracle.round_to_float32(np.asarray(h, float) @ np.asarray(lm, float).T)
+        return u + om.compute_step_bias(w1, w2, np.asarray(ids).reshape(-1))
+    monkeypatch.setattr(om, "fused_lm_head_exact", twice)
+    _fails(pins.test_fused_producer_rounds_once)

@@ -661,3 +661,93 @@ def test_accumulation_bound_is_attained_within_a_factor_of_three():
     err = abs(float(s[0, 0]) - (1.0 + r * 2.0 ** -24))
     bound = float(oc.accumulation_bound(u, w1, w2, [0])[0, 0])
     assert err <= bound <= 3 * err, (err, bound)
+
+
+# --------------------------------------------------------------------------
+# The fused producer: base logits U = hidden @ lm_head^T made in the same
+# pass as the bias, rounded once.
+# --------------------------------------------------------------------------
+
+def test_fused_producer_explicit_sums():
+    """Small integers, every sum written out as Python loops (no matrix
+    product): out[i, v] = sum_j h[i, j] lm[v, j] + sum_j W1[x_i, j] W2[v, j].
+    A square lm_head (d = V) that is not symmetric catches a transposed
+    weight."""
+    rng = np.random.default_rng(40)
+    for rows, d, v, r in ((4, 6, 6, 3), (3, 5, 4, 2)):
+        h = rng.integers(-4, 5, size=(rows, d)).astype(float)
+        lm = rng.integers(-4, 5, size=(v, d)).astype(float)
+        w1 = rng.integers(-3, 4, size=(v, r)).astype(float)
+        w2 = rng.integers(-3, 4, size=(v, r)).astype(float)
+        ids = rng.integers(0, v, size=rows)
+        want = [[sum(h[i][j] * lm[t][j] for j in range(d)) + sum(w1[ids[i]][j] * w2[t][j] for j in range(r))
+                 for t in range(v)] for i in range(rows)]
+        got = oracle.fused_lm_head_logits(h, lm, w1, w2, ids, "fp32")
+        np.testing.assert_array_equal(got, np.array(want))
+        if d == v:
+            assert not np.array_equal(lm, lm.T)
+
+
+def test_fused_producer_reduces_to_the_pinned_head():
+    """lm_head = 0 gives the transition bias alone (the head's forward); a
+    one-hot hidden row e_j gives base logits lm_head[:, j], so the result is
+    apply_block_logits on those base logits."""
+    rng = np.random.default_rng(41)
+    rows, d, v, r = 7, 12, 50, 8
+    h = _bf16(rng.standard_normal((rows, d)))
+    lm = _bf16(rng.standard_normal((v, d)) * 0.5)
+    w1, w2 = _bf16(rng.standard_normal((v, r)) * 0.3), _bf16(rng.standard_normal((v, r)) * 0.3)
+    ids = rng.integers(0, v, rows)
+    tr, _ = oracle.transition_logits(w1, w2, ids, "bf16")
+    np.testing.assert_array_equal(oracle.fused_lm_head_logits(h, np.zeros_like(lm), w1, w2, ids, "bf16"), tr)
+    onehot = np.zeros((rows, d))
+    cols = rng.integers(0, d, rows)
+    onehot[np.arange(rows), cols] = 1.0
+    base = lm[:, cols].T  # row i: lm_head[:, cols[i]]
+    want = oracle.apply_block_logits(base[:, None, :], w1, w2, ids[:, None], "bf16")[:, 0]
+    np.testing.assert_array_equal(oracle.fused_lm_head_logits(onehot, lm, w1, w2, ids, "bf16"), want)
+
+
+def test_fused_producer_rounds_once():
+    """U = 1 + 2^-30 and a bias of 2^-8: the exact sum lies just above the
+    halfway point between 1 and 1 + 2^-7, so one rounding to bf16 goes up.
+    Rounding U to fp32 first (to 1) lands exactly on the halfway point,
+    which ties to even (down)."""
+    h = np.array([[1.0, 2.0 ** -15]])
+    lm = np.array([[1.0, 2.0 ** -15]])
+    w1, w2 = np.array([[1.0]]), np.array([[2.0 ** -8]])
+    got = oracle.fused_lm_head_logits(h, lm, w1, w2, [0], "bf16")
+    assert got[0, 0] == 1.0 + 2.0 ** -7
+
+
+def test_fused_producer_matches_a_library_matmul():
+    """W2 = 0: the result is the fp64 matrix product of a library (torch)
+    rounded once, for leading dims (2, 3)."""
+    rng = np.random.default_rng(42)
+    h = _bf16(rng.standard_normal((2, 3, 64)))
+    lm = _bf16(rng.standard_normal((100, 64)) * 0.1)
+    w1, w2 = _bf16(rng.standard_normal((100, 4))), np.zeros((100, 4))
+    ids = rng.integers(0, 100, (2, 3))
+    want = torch.from_numpy(h).double() @ torch.from_numpy(lm).double().T
+    got = oracle.fused_lm_head_logits(h, lm, w1, w2, ids, "fp32")
+    np.testing.assert_array_equal(got, oracle.round_to_float32(want.numpy()))
+
+
+def test_fused_accumulation_bound_covers_fp32_sums():
+    """fp32 recursive sums of the d + r products (forward, reversed, 16-term
+    blocks) stay within the fused bound."""
+    rng = np.random.default_rng(43)
+    rows, d, v, r = 4, 256, 64, 64
+    h = _bf16(rng.standard_normal((rows, d)))
+    lm = _bf16(rng.standard_normal((v, d)) * 0.05)
+    w1, w2 = _bf16(rng.standard_normal((v, r)) * 0.3), _bf16(rng.standard_normal((v, r)) * 0.3)
+    ids = rng.integers(0, v, rows)
+    exact = oracle.fused_lm_head_exact(h, lm, w1, w2, ids)
+    bound = oc.fused_accumulation_bound(h, lm, w1, w2, ids)
+    prods = [h[:, j][:, None].astype(np.float32) * lm[None, :, j].astype(np.float32) for j in range(d)]
+    prods += [w1[ids, j][:, None].astype(np.float32) * w2[None, :, j].astype(np.float32) for j in range(r)]
+    for name, terms in (("forward", prods), ("reversed", prods[::-1]),
+                        ("blocks of 16", [np.sum(np.stack(prods[i:i + 16]), axis=0, dtype=np.float32)
+                                          for i in range(0, d + r, 16)])):
+        err = np.abs(_fp32_sum(terms).astype(np.float64) - exact)
+        assert np.all(err <= bound), name
