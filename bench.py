@@ -41,14 +41,16 @@ from rank_markov_draft_vanillamarkov_b200 import workloads as W  # noqa: E402
 METRIC = "corrected-logit rows/s + achieved HBM GB/s (% roofline); sampled blocks/s at M=5"
 UNIT = "rows/s"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 PARTS = (("apply", W.APPLY_320), ("greedy", W.greedy(32)), ("temperature", W.TEMPERATURE))
 EXTRA = (("apply_2560", W.APPLY_2560), ("apply_fp32", W.APPLY_320_FP32), ("transition", W.TRANSITION_320),
-         ("backward", W.BACKWARD_320))
+         ("backward", W.BACKWARD_320), ("fused_lm_head", W.FUSED_320), ("greedy_b1", W.greedy(1)),
+         ("greedy_b8", W.greedy(8)), ("greedy_b64", W.greedy(64)))
 L2_BYTES = 126 * 1024 * 1024
 
 
 def part_rows(wl: W.Workload) -> int:
-    return wl.rows if wl.mode in ("apply", "transition", "backward") else wl.batch * wl.proposal_len
+    return wl.rows if wl.mode in ("apply", "transition", "backward", "fused") else wl.batch * wl.proposal_len
 
 
 # --------------------------------------------------------------- helpers --
@@ -70,14 +72,26 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def profile_traffic(kernel_tag: str):
-    """DRAM bytes per launch from the committed ncu summary of this kernel,
-    valid only while the kernel source it was taken from is unchanged."""
+def measured_tensor_peak():
+    """Sustained dense bf16 TFLOP/s (a kernel timed inside a long loop)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS_SUSTAINED, "fallback"
+
+
+def profile_field(kernel_tag: str, field: str):
+    """A per-launch figure from the committed ncu summary of this kernel
+    (profiles/<tag>.md), valid only while every source file it lists still
+    has the recorded hash."""
     path = os.path.join(ROOT, "profiles", f"{kernel_tag}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
-    m_b = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    m_b = re.search(field + r":\s*([0-9.eE+]+)", text)
     pairs = re.findall(r"source_file:\s*(\S+)\s+source_sha256:\s*([0-9a-f]{64})", text)
     if not (m_b and pairs):
         return None
@@ -86,6 +100,26 @@ def profile_traffic(kernel_tag: str):
         if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != digest:
             return None
     return float(m_b.group(1))
+
+
+def profile_traffic(kernel_tag: str):
+    """DRAM read + write bytes per launch (roofline.traffic)."""
+    return profile_field(kernel_tag, "traffic_bytes_per_launch")
+
+
+ISSUE_SLOTS_PER_SM = 4  # one warp instruction per clock per SM sub-partition
+
+
+def issue_roofline(kernel_tag: str, seconds: float, sm_mhz: float, sms: int):
+    """The issue bound of a kernel limited by its instruction stream: warp
+    instructions per launch (ncu smsp__inst_executed.sum) over the launch
+    time, against SMs x 4 issue slots x the SM clock sampled during the run."""
+    inst = profile_field(kernel_tag, "inst_executed_per_launch")
+    if inst is None or not sm_mhz:
+        return None
+    peak = sms * ISSUE_SLOTS_PER_SM * sm_mhz * 1e6
+    return {"achieved": inst / seconds, "peak": peak, "unit": "warp-inst/s", "frac": inst / seconds / peak,
+            "inst_per_launch": inst, "sm_mhz": sm_mhz}
 
 
 class ClockSampler:
@@ -164,6 +198,8 @@ class Part:
             elif wl.mode == "backward":
                 dev["gw1"] = torch.empty(wl.vocab, wl.rank, dtype=torch.float32, device=device)
                 dev["gw2"] = torch.empty(wl.vocab, wl.rank, dtype=torch.float32, device=device)
+            elif wl.mode == "fused":
+                dev["out"] = torch.empty(*dev["prev_ids"].shape, wl.vocab, dtype=torch.float32, device=device)
             elif wl.mode == "transition":
                 ids = dev["prev_ids"]
                 dev["out"] = torch.empty(*ids.shape, wl.vocab, dtype=torch.bfloat16, device=device)
@@ -180,6 +216,8 @@ class Part:
             s["head"].apply_block_logits(s["base"], token_ids=s["prev_ids"], out=s["out"])
         elif self.wl.mode == "transition":
             s["head"].transition_logits(s["prev_ids"], out=s["out"], out_embeddings=s["emb"])
+        elif self.wl.mode == "fused":
+            s["head"].fused_lm_head_logits(s["hidden"], s["lm_head"], token_ids=s["prev_ids"], out=s["out"])
         elif self.wl.mode == "backward":
             s["head"].apply_block_logits_backward(s["base"], token_ids=s["prev_ids"], grad_w1=s["gw1"],
                                                   grad_w2=s["gw2"])
@@ -319,12 +357,26 @@ def _np(t):
 
 
 def oracle_threads():
+    """Threads of the BLAS library the oracle's matrix products run on."""
     try:
         from threadpoolctl import threadpool_info
         n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
         return int(max(n)) if n else 1
     except Exception:
         return 1
+
+
+def host_cores():
+    """Cores this process may run on (its CPU affinity)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_parallelism():
+    return (f"the oracle's matrix products use {oracle_threads()} BLAS threads; its rounding, selection and "
+            f"the sampler's step loop run on one thread")
 
 
 def oracle_full_step(inputs):
@@ -386,7 +438,8 @@ def reference_arm(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_block(args.gpus),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
+                         "threads": oracle_parallelism(),
                          "sample": "each step is one unit of the step's work in its proportions (one apply row, "
                                    "one greedy block of 5 or one temperature block of 8), in order"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -403,6 +456,27 @@ def config_block(n_gpus):
         "l2": "inputs rotate over >= 3 x L2 of distinct buffers per part, so no step finds its data in L2",
         "parallelism": f"replicas{n_gpus}" if n_gpus > 1 else "single",
     }
+
+
+PROFILE_TAGS = {"apply": "apply_wide_r320_v129280_k128", "greedy": "sample_rows_greedy_b32_m5_v129280_k128",
+                "temperature": "sample_rows_temp_b32_m8_v151936_k64"}
+
+
+def roofline_block(dom, tag, achieved, hbm_peak, peak_kind, partinfo):
+    """The dominant kernel's roofline, against the bound that binds it: HBM
+    (algorithmic bytes over the launch time) or, where the kernel's own
+    instruction stream takes longer than its bytes would at peak bandwidth,
+    the issue rate ("alu")."""
+    hbm = {"bound": "hbm", "kernel": dom.name, "achieved": achieved, "peak": hbm_peak, "peak_kind": peak_kind,
+           "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": profile_traffic(tag),
+           "algorithmic_bytes": dom.wl.bytes_moved()}
+    iss = partinfo[dom.name].get("issue")
+    if not iss or iss["frac"] <= hbm["frac"]:
+        return hbm
+    return {"bound": "alu", "kernel": dom.name, "achieved": iss["achieved"], "peak": iss["peak"],
+            "peak_kind": "derived: SMs x 4 issue slots x sampled SM clock", "unit": iss["unit"],
+            "frac": iss["frac"], "traffic": profile_traffic(tag), "algorithmic_bytes": dom.wl.bytes_moved(),
+            "hbm": {k: hbm[k] for k in ("achieved", "peak", "peak_kind", "unit", "frac")}}
 
 
 # ----------------------------------------------------------------- main ----
@@ -484,11 +558,22 @@ def main():
                 "bytes": p.wl.bytes_moved(), "flops": p.wl.flops()}
         if p.wl.mode == "sample":
             info["blocks_per_s"] = p.wl.batch / t
+        if p.wl.mode == "fused":  # compute-bound: the tensor pipe is its roofline
+            tf_peak, tf_kind = measured_tensor_peak()
+            info["tflops"] = p.wl.flops() / t / 1e12
+            info["frac_tensor"] = info["tflops"] / tf_peak
+            info["tensor_peak"] = tf_peak
+            info["tensor_peak_kind"] = tf_kind
         partinfo[p.name] = info
     dom = max(parts, key=lambda p: per[p.name])
-    tag = {"apply": "apply_tc_r320_v129280_k128", "greedy": "sample_tc_greedy_b32_m5_v129280_k128",
-           "temperature": "sample_tc_temp_b32_m8_v151936_k64"}[dom.name]
+    tag = PROFILE_TAGS[dom.name]
     achieved = dom.wl.bytes_moved() / per[dom.name] / 1e9
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    sm_mhz = (clk or {}).get("sm_mhz") or 1965.0
+    for p in parts:  # the issue bound beside the HBM one, where a profile gives the instruction count
+        iss = issue_roofline(PROFILE_TAGS[p.name], per[p.name], sm_mhz, sms)
+        if iss:
+            partinfo[p.name]["issue"] = iss
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": region / args.steps * 1e3, "higher_is_better": True,
@@ -496,9 +581,7 @@ def main():
         "config": config_block(world),
         "sampled_blocks_per_s_m5": partinfo["greedy"]["blocks_per_s"] * world,
         "parts": partinfo,
-        "roofline": {"bound": "hbm", "kernel": dom.name, "achieved": achieved, "peak": hbm_peak,
-                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm_peak,
-                     "traffic": profile_traffic(tag), "algorithmic_bytes": dom.wl.bytes_moved()},
+        "roofline": roofline_block(dom, tag, achieved, hbm_peak, peak_kind, partinfo),
         "gpu_launches": launches,
         "clocks": clk,
         "e2e": e2e,
@@ -511,7 +594,8 @@ def main():
             rows += oracle_full_step(inputs)
             steps += 1
         sec = time.perf_counter() - t0
-        line["cpu_baseline"] = {"value": rows / sec, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+        line["cpu_baseline"] = {"value": rows / sec, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
+                                "threads": oracle_parallelism(),
                                 "sample": f"{steps} full steps (all three parts at full size) through the fp64 oracle",
                                 "seconds": sec}
     if rank == 0:

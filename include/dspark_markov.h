@@ -111,6 +111,40 @@ int dspark_markov_apply_block_logits_backward(const void* grad_out, const int64_
                                               int32_t logits_dtype, int32_t weight_dtype, void* stream);
 
 /*
+ * Corrected logits with the base logits produced in the same pass (the step
+ * before the head on the path: "U_k is the backbone's base logit
+ * (lm_head(hidden_k))", module docstring of markov_head.py; the frozen
+ * vocabulary head of DeepseekV41DSparkModel.compute_logits, weight
+ * [vocab, hidden], FP32 result). For each row i with previous token
+ * x = prev_token_ids[i]:
+ *
+ *     out[i, v] = round( sum_{j<hidden_dim} hidden[i, j] * lm_head[v, j]
+ *                        + sum_{j<rank} W1[x, j] * W2[v, j] )
+ *
+ * one fp32 accumulation over both sums and one rounding (nearest even) to
+ * out_dtype, so the base logits are never stored.
+ *
+ *   hidden          [rows, hidden_dim] weight_dtype, row-major.
+ *   prev_token_ids  [rows] int64 (teacher-forced previous tokens).
+ *   lm_head         [vocab, hidden_dim] weight_dtype (the LM head's weight).
+ *   w1, w2          [vocab, rank] weight_dtype.
+ *   out             [rows, vocab] out_dtype (DSPARK_DTYPE_FP32, as the pages'
+ *                   compute_logits returns, or DSPARK_DTYPE_BF16), written.
+ *
+ * Supported: weight_dtype DSPARK_DTYPE_BF16; hidden_dim, rank and vocab
+ * multiples of 8; every pointer 16-byte aligned; anything else returns
+ * DSPARK_ERR_UNSUPPORTED (there is no other kernel for this entry). An id
+ * outside [0, vocab) adds a zero bias for its row and sets
+ * DSPARK_STATUS_TOKEN_RANGE. rows == 0 is OK and enqueues nothing.
+ * Ownership and errors as for dspark_markov_apply_block_logits; `out` must
+ * not overlap the inputs.
+ */
+int dspark_markov_fused_lm_head_logits(const void* hidden, const int64_t* prev_token_ids, int64_t rows,
+                                       int64_t hidden_dim, int64_t vocab, const void* lm_head, const void* w1,
+                                       const void* w2, int32_t rank, void* out, int32_t out_dtype,
+                                       int32_t weight_dtype, void* stream);
+
+/*
  * The transition bias alone, and its conditioning embeddings
  * (nemo_automodel.components.models.deepseek_v41.dspark,
  * _DeepseekV41DSparkMarkovHead.forward: "transition logits of shape [..., vocab]
@@ -217,10 +251,35 @@ int64_t dspark_markov_launch_count(void);
  * out and reports DSPARK_STATUS_TIMEOUT; no GPU fault is involved.
  */
 #define DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL 1u
+/* flags bit 1: the tensor-core apply uses 128-id units even where 256-id
+ * units apply (both kernels stay testable). */
+#define DSPARK_DEBUG_APPLY_NARROW 2u
 int dspark_markov_set_debug(uint32_t flags, uint64_t wait_limit_ns);
 
 /* Which kernel the last call on this thread selected: 0 none, 1 generic, 2 tensor core. */
 int32_t dspark_markov_last_algo(void);
+
+/*
+ * Test hook: DSPARK_VARIANT_* bits naming the tensor-core kernel variants the
+ * last call on this thread launched (0 when it launched none of them).
+ *   DSPARK_VARIANT_BWD_RESIDENT_W1: the backward's dW2 kernel gathered every
+ *     row's W1 row once into a resident shared-memory block (rows <= 8192 and
+ *     the block fits beside three gradient stages), instead of once per stage.
+ */
+#define DSPARK_VARIANT_BWD_RESIDENT_W1 1
+/*
+ *   DSPARK_VARIANT_SAMPLE_ROWS: the tensor-core sampler ran with the batch on
+ *     the MMA's M side and 256 vocabulary ids per MMA (batch <= 128);
+ *     otherwise it ran with vocabulary ids on M and the batch on N.
+ */
+#define DSPARK_VARIANT_SAMPLE_ROWS 2
+/*
+ *   DSPARK_VARIANT_APPLY_WIDE: the tensor-core apply ran with units of 128 rows
+ *     x 256 ids (bf16 logits with a base, out != base_logits); otherwise with
+ *     128 x 128.
+ */
+#define DSPARK_VARIANT_APPLY_WIDE 4
+int32_t dspark_markov_last_variant(void);
 
 /*
  * Test hook: out[i] = the Gumbel variate g = -log(-log u) that every sampler

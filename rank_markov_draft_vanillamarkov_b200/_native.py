@@ -28,8 +28,13 @@ DSPARK_ALGO_GENERIC = 1
 DSPARK_ALGO_TENSOR_CORE = 2
 
 DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL = 1
+DSPARK_DEBUG_APPLY_NARROW = 2
 
 DSPARK_NOALLOC_MAX_KEYS = 8192
+
+DSPARK_VARIANT_BWD_RESIDENT_W1 = 1
+DSPARK_VARIANT_SAMPLE_ROWS = 2
+DSPARK_VARIANT_APPLY_WIDE = 4
 
 # Every symbol include/dspark_markov.h declares, with its ctypes signature.
 _vp, _i64, _i32, _u32, _u64, _f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_uint32, ctypes.c_uint64, ctypes.c_float
@@ -40,6 +45,8 @@ SIGNATURES = {
     "dspark_markov_apply_block_logits_backward": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _i32, _vp, _vp,
                                                                  _i32, _i32, _i32, _vp]),
     "dspark_markov_transition_logits": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp, _i32, _vp, _vp, _i32, _vp]),
+    "dspark_markov_fused_lm_head_logits": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _i32, _vp,
+                                                          _i32, _i32, _vp]),
     "dspark_markov_sample_block_noalloc": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _i32, _f32, _u64,
                                                           _vp, _vp, _i32, _i32, _vp]),
     "dspark_markov_get_status": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_int32)]),
@@ -48,6 +55,7 @@ SIGNATURES = {
     "dspark_markov_launch_count": (_i64, []),
     "dspark_markov_set_debug": (ctypes.c_int, [_u32, _u64]),
     "dspark_markov_last_algo": (_i32, []),
+    "dspark_markov_last_variant": (_i32, []),
     "dspark_markov_debug_gumbel": (ctypes.c_int, [_vp, _vp, _i64, _vp]),
 }
 

@@ -13,7 +13,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libdspark_markov.so")
-SOURCES = ["abi.cu", "generic.cu", "apply_tc.cu", "sample_tc.cu", "backward_tc.cu"]
+SOURCES = ["abi.cu", "generic.cu", "apply_tc.cu", "sample_tc.cu", "backward_tc.cu", "fused_tc.cu", "sample_rows_tc.cu", "apply_wide_tc.cu"]
 HEADERS = ["common.cuh", "ptx.cuh", "kernels.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

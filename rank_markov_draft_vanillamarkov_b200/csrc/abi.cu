@@ -36,6 +36,7 @@ std::atomic<int32_t> g_algo{DSPARK_ALGO_AUTO};
 std::atomic<uint32_t> g_debug_flags{0};
 std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
 thread_local int32_t t_last_algo = 0;
+thread_local int32_t t_last_variant = 0;
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -171,6 +172,7 @@ int dspark_markov_apply_block_logits(const void* base_logits, void* out, const i
                                      int64_t vocab, const void* w1, const void* w2, int32_t rank, int32_t logits_dtype,
                                      int32_t weight_dtype, void* stream) {
   t_last_algo = 0;
+  t_last_variant = 0;
   if (rows < 0 || vocab <= 0 || rank <= 0 || !dtype_ok(logits_dtype) || !dtype_ok(weight_dtype))
     return DSPARK_ERR_INVALID_ARG;
   if (rows == 0) return DSPARK_OK;
@@ -188,6 +190,13 @@ int dspark_markov_apply_block_logits(const void* base_logits, void* out, const i
     TcApplyArgs a{base_logits, out, prev_token_ids, rows, vocab, w1, w2, rank, d->status, g_wait_limit_ns.load(),
                   logits_dtype == DSPARK_DTYPE_FP32 ? 1 : 0};
     t_last_algo = 2;
+    // In-place calls (out == base) keep the 128-id kernel, whose unit reads
+    // and writes the same tile; the 256-id kernel takes the rest it supports.
+    const bool narrow = (g_debug_flags.load() & DSPARK_DEBUG_APPLY_NARROW) != 0 || out == base_logits;
+    if (!narrow && tc_apply_wide_supported(rows, vocab, rank, logits_dtype, weight_dtype, true)) {
+      t_last_variant = DSPARK_VARIANT_APPLY_WIDE;
+      return cuda_code(launch_tc_apply_wide(a, d->num_sms, s));
+    }
     return cuda_code(launch_tc_apply(a, d->num_sms, s));
   }
   GenericApplyArgs a{base_logits, out, prev_token_ids, rows, vocab, vocab, vocab, 1, w1, w2, rank, d->status};
@@ -200,6 +209,7 @@ int dspark_markov_apply_block_logits_backward(const void* grad_out, const int64_
                                               float* grad_w1, float* grad_w2, int32_t accumulate,
                                               int32_t logits_dtype, int32_t weight_dtype, void* stream) {
   t_last_algo = 0;
+  t_last_variant = 0;
   if (rows < 0 || vocab <= 0 || rank <= 0 || !dtype_ok(logits_dtype) || !dtype_ok(weight_dtype))
     return DSPARK_ERR_INVALID_ARG;
   if (!grad_w1 && !grad_w2) return DSPARK_OK;  // nothing wanted
@@ -223,7 +233,10 @@ int dspark_markov_apply_block_logits_backward(const void* grad_out, const int64_
   if (algo == DSPARK_ALGO_TENSOR_CORE && !tc_ok) return DSPARK_ERR_UNSUPPORTED;
   if (tc_ok && algo != DSPARK_ALGO_GENERIC) {
     t_last_algo = 2;
-    return cuda_code(launch_tc_backward(a, d->num_sms, g_wait_limit_ns.load(), s));
+    int variant = 0;
+    const cudaError_t e = launch_tc_backward(a, d->num_sms, g_wait_limit_ns.load(), s, &variant);
+    t_last_variant = variant;
+    return cuda_code(e);
   }
   t_last_algo = 1;
   return cuda_code(launch_backward(a, logits_dtype, weight_dtype, s));
@@ -233,6 +246,7 @@ int dspark_markov_transition_logits(const int64_t* token_ids, int64_t rows, int6
                                     const void* w2, int32_t rank, void* transition_out, void* embeddings_out,
                                     int32_t weight_dtype, void* stream) {
   t_last_algo = 0;
+  t_last_variant = 0;
   if (rows < 0 || vocab <= 0 || rank <= 0 || !dtype_ok(weight_dtype)) return DSPARK_ERR_INVALID_ARG;
   if (rows == 0) return DSPARK_OK;
   if (!token_ids || !w1 || !w2 || !transition_out) return DSPARK_ERR_INVALID_ARG;
@@ -262,11 +276,47 @@ int dspark_markov_transition_logits(const int64_t* token_ids, int64_t rows, int6
   return cuda_code(e);
 }
 
+int dspark_markov_fused_lm_head_logits(const void* hidden, const int64_t* prev_token_ids, int64_t rows,
+                                       int64_t hidden_dim, int64_t vocab, const void* lm_head, const void* w1,
+                                       const void* w2, int32_t rank, void* out, int32_t out_dtype,
+                                       int32_t weight_dtype, void* stream) {
+  t_last_algo = 0;
+  t_last_variant = 0;
+  if (rows < 0 || hidden_dim <= 0 || vocab <= 0 || rank <= 0 || !dtype_ok(out_dtype) || !dtype_ok(weight_dtype))
+    return DSPARK_ERR_INVALID_ARG;
+  if (rows == 0) return DSPARK_OK;
+  if (!hidden || !prev_token_ids || !lm_head || !w1 || !w2 || !out) return DSPARK_ERR_INVALID_ARG;
+  const auto aligned = [](const void* q) { return reinterpret_cast<uintptr_t>(q) % 16 == 0; };
+  if (!tc_fused_supported(rows, hidden_dim, vocab, rank, out_dtype, weight_dtype) || !aligned(hidden) ||
+      !aligned(lm_head) || !aligned(w1) || !aligned(w2) || !aligned(out))
+    return DSPARK_ERR_UNSUPPORTED;
+  int err = DSPARK_OK;
+  DeviceState* d = device_state(&err);
+  if (!d) return err;
+  TcFusedArgs a{};
+  a.hidden = hidden;
+  a.lm_head = lm_head;
+  a.ids = prev_token_ids;
+  a.w1 = w1;
+  a.w2 = w2;
+  a.out = out;
+  a.rows = rows;
+  a.hidden_dim = hidden_dim;
+  a.vocab = vocab;
+  a.rank = rank;
+  a.out_f32 = out_dtype == DSPARK_DTYPE_FP32 ? 1 : 0;
+  a.status = d->status;
+  a.wait_limit_ns = g_wait_limit_ns.load();
+  t_last_algo = 2;
+  return cuda_code(launch_tc_fused(a, d->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
 int dspark_markov_sample_block(const void* base_logits, const int64_t* first_prev_token_ids, int64_t batch,
                                int64_t proposal_len, int64_t vocab, const void* w1, const void* w2, int32_t rank,
                                float temperature, uint64_t seed, int64_t* sampled_tokens, void* corrected_logits,
                                int32_t logits_dtype, int32_t weight_dtype, void* stream) {
   t_last_algo = 0;
+  t_last_variant = 0;
   if (batch < 0 || proposal_len < 0 || vocab <= 0 || rank <= 0 || !dtype_ok(logits_dtype) ||
       !dtype_ok(weight_dtype) || std::isnan(temperature))
     return DSPARK_ERR_INVALID_ARG;
@@ -317,7 +367,10 @@ int dspark_markov_sample_block(const void* base_logits, const int64_t* first_pre
     a.wait_limit_ns = g_wait_limit_ns.load();
     a.debug_flags = g_debug_flags.load();
     t_last_algo = 2;
-    return cuda_code(launch_tc_sample(a, d->num_sms, s));
+    int variant = 0;
+    const cudaError_t e = launch_tc_sample(a, d->num_sms, s, &variant);
+    t_last_variant = variant;
+    return cuda_code(e);
   }
   // Generic path: one correction launch and one selection launch per step.
   t_last_algo = 1;
@@ -360,6 +413,7 @@ int dspark_markov_sample_block_noalloc(const void* base_logits, const int64_t* f
                                        void* corrected_logits, int32_t logits_dtype, int32_t weight_dtype,
                                        void* stream) {
   t_last_algo = 0;
+  t_last_variant = 0;
   if (batch < 0 || proposal_len < 0 || vocab <= 0 || rank <= 0 || !dtype_ok(logits_dtype) ||
       !dtype_ok(weight_dtype) || std::isnan(temperature))
     return DSPARK_ERR_INVALID_ARG;
@@ -410,7 +464,10 @@ int dspark_markov_sample_block_noalloc(const void* base_logits, const int64_t* f
   a.wait_limit_ns = g_wait_limit_ns.load();
   a.debug_flags = g_debug_flags.load();
   t_last_algo = 2;
-  return cuda_code(launch_tc_sample(a, st->num_sms, s));
+  int variant = 0;
+  const cudaError_t e = launch_tc_sample(a, st->num_sms, s, &variant);
+  t_last_variant = variant;
+  return cuda_code(e);
 }
 
 int dspark_markov_get_status(void* stream, int32_t* status_out) {
@@ -459,6 +516,8 @@ int dspark_markov_set_debug(uint32_t flags, uint64_t wait_limit_ns) {
 }
 
 int32_t dspark_markov_last_algo(void) { return t_last_algo; }
+
+int32_t dspark_markov_last_variant(void) { return t_last_variant; }
 
 int dspark_markov_debug_gumbel(const uint32_t* words, float* out, int64_t n, void* stream) {
   if (n < 0 || (n > 0 && (!words || !out))) return DSPARK_ERR_INVALID_ARG;

@@ -480,6 +480,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_backward_kernel(const __grid_c
   if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
 }
 
+// Shared memory outside the stage ring: alignment slack, barriers, the cached
+// W1 coordinates of `rid_cached` rows, the dW2 output boxes and, with RES, the
+// resident block of those rows' W1 rows (NA 128-byte rows per row).
+size_t fixed_smem_bytes(int na, bool dw1, bool res, int64_t rid_cached) {
+  return 1024 + sizeof(BwdShared) + (size_t)rid_cached * 4 + 64 + (dw1 ? 0 : (size_t)out_boxes_of(na) * kOutBoxBytes) +
+         (res ? (size_t)na * (size_t)rid_cached * 128 : 0);
+}
+
+// The rows whose W1 coordinates dW2 caches in shared memory (all of them, rounded
+// up to a whole stage, when there are at most kRidCacheRows; else none).
+int64_t rid_cached_of(int64_t rows) { return rows <= kRidCacheRows ? (rows + kKc - 1) / kKc * kKc : 0; }
+
 template <int NA, bool DW1, bool RES>
 cudaError_t launch_one(const BackwardArgs& a, int num_sms, uint64_t wait_limit_ns, cudaStream_t stream) {
   BwdMaps maps;
@@ -526,11 +538,10 @@ cudaError_t launch_one(const BackwardArgs& a, int num_sms, uint64_t wait_limit_n
   } else {
     p.units = (int32_t)((a.vocab + kBM - 1) / kBM);
     p.k_stages = (int32_t)((a.rows + kKc - 1) / kKc);
-    p.rid_cached = a.rows <= kRidCacheRows ? p.k_stages * kKc : 0;
+    p.rid_cached = (int32_t)rid_cached_of(a.rows);
   }
   const size_t stage_bytes = RES ? a_bytes_of(false) : stage_bytes_of(NA, DW1);
-  const size_t fixed = 1024 + sizeof(BwdShared) + (size_t)p.rid_cached * 4 + 64 +
-                       (DW1 ? 0 : out_boxes_of(NA) * kOutBoxBytes) + (RES ? (size_t)NA * p.rid_cached * 128 : 0);
+  const size_t fixed = fixed_smem_bytes(NA, DW1, RES, p.rid_cached);
   if (fixed + 2 * stage_bytes > kSmemLimit) return cudaErrorInvalidValue;
   int stages = (int)((kSmemLimit - fixed) / stage_bytes);
   if (stages > kMaxStages) stages = kMaxStages;
@@ -547,14 +558,13 @@ cudaError_t launch_one(const BackwardArgs& a, int num_sms, uint64_t wait_limit_n
 }
 
 template <int NA>
-cudaError_t launch_na(const BackwardArgs& a, int num_sms, uint64_t wait_limit_ns, cudaStream_t s) {
+cudaError_t launch_na(const BackwardArgs& a, int num_sms, uint64_t wait_limit_ns, cudaStream_t s, int* variant) {
   cudaError_t e = cudaSuccess;
   if (a.grad_w2) {
     // Resident W1 rows when they fit beside at least three G stages.
-    const int64_t kpad = (a.rows + kKc - 1) / kKc * kKc;
-    const size_t res_fixed = 1024 + sizeof(BwdShared) + (size_t)kpad * 4 + 64 + out_boxes_of(NA) * kOutBoxBytes +
-                             (size_t)NA * kpad * 128;
-    const bool res = a.rows <= kRidCacheRows && res_fixed + 3 * (size_t)a_bytes_of(false) <= kSmemLimit;
+    const int64_t rid = rid_cached_of(a.rows);
+    const bool res = rid > 0 && fixed_smem_bytes(NA, false, true, rid) + 3 * (size_t)a_bytes_of(false) <= kSmemLimit;
+    if (res) *variant |= DSPARK_VARIANT_BWD_RESIDENT_W1;
     e = res ? launch_one<NA, false, true>(a, num_sms, wait_limit_ns, s)
             : launch_one<NA, false, false>(a, num_sms, wait_limit_ns, s);
   }
@@ -571,13 +581,14 @@ bool tc_backward_supported(int64_t rows, int64_t vocab, int32_t rank, int logits
   return rows + kBM < (1ll << 31) && vocab + kBM < (1ll << 31);
 }
 
-cudaError_t launch_tc_backward(const BackwardArgs& a, int num_sms, uint64_t wait_limit_ns, cudaStream_t s) {
+cudaError_t launch_tc_backward(const BackwardArgs& a, int num_sms, uint64_t wait_limit_ns, cudaStream_t s,
+                               int* variant) {
   if (a.rows == 0) return cudaSuccess;
   switch (a.rank / 64) {
-    case 1: return launch_na<1>(a, num_sms, wait_limit_ns, s);
-    case 2: return launch_na<2>(a, num_sms, wait_limit_ns, s);
-    case 3: return launch_na<3>(a, num_sms, wait_limit_ns, s);
-    case 4: return launch_na<4>(a, num_sms, wait_limit_ns, s);
+    case 1: return launch_na<1>(a, num_sms, wait_limit_ns, s, variant);
+    case 2: return launch_na<2>(a, num_sms, wait_limit_ns, s, variant);
+    case 3: return launch_na<3>(a, num_sms, wait_limit_ns, s, variant);
+    case 4: return launch_na<4>(a, num_sms, wait_limit_ns, s, variant);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -73,6 +73,11 @@ struct TcApplyArgs {
 };
 bool tc_apply_supported(int64_t rows, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype);
 cudaError_t launch_tc_apply(const TcApplyArgs& a, int num_sms, cudaStream_t s);
+// The same apply with 256-id units (apply_wide_tc.cu): bf16 logits with a
+// base, bf16 weights, rank in {64, 128, 192, 256}.
+bool tc_apply_wide_supported(int64_t rows, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype,
+                             bool has_base);
+cudaError_t launch_tc_apply_wide(const TcApplyArgs& a, int num_sms, cudaStream_t s);
 
 // Persistent left-to-right sampler on tcgen05: bf16 logits, bf16 weights,
 // vocab % 8 == 0, rank in {64, 128, 192, 256}, batch <= 256 (and within the
@@ -97,14 +102,42 @@ struct TcSampleArgs {
 };
 bool tc_sample_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype,
                          int num_sms);
-cudaError_t launch_tc_sample(const TcSampleArgs& a, int num_sms, cudaStream_t s);
+// Sets DSPARK_VARIANT_SAMPLE_ROWS in *variant when the row-layout kernel runs.
+cudaError_t launch_tc_sample(const TcSampleArgs& a, int num_sms, cudaStream_t s, int* variant);
+// The row-layout sampler (sample_rows_tc.cu): batch on the MMA's M side,
+// batch <= 128.
+bool tc_sample_rows_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype,
+                              int num_sms);
+cudaError_t launch_tc_sample_rows(const TcSampleArgs& a, int num_sms, cudaStream_t s);
 
 // Backward of the teacher-forced apply on tcgen05: bf16 gradient and bf16
 // weights, vocab % 8 == 0, rank in {64, 128, 192, 256}, every pointer 16-byte
 // aligned. grad_w1 must already hold its starting value (zero, or the sum to
 // add to); grad_w2 is written, or added to when accumulate is set.
 bool tc_backward_supported(int64_t rows, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype);
-cudaError_t launch_tc_backward(const BackwardArgs& a, int num_sms, uint64_t wait_limit_ns, cudaStream_t s);
+// Sets DSPARK_VARIANT_* bits in *variant for the kernel variants it launches.
+cudaError_t launch_tc_backward(const BackwardArgs& a, int num_sms, uint64_t wait_limit_ns, cudaStream_t s,
+                               int* variant);
+
+// The fused producer on tcgen05: out = round(hidden . lm_head^T + W1[x] . W2^T),
+// bf16 operands, fp32 accumulation, fp32 or bf16 output; hidden_dim, rank
+// and vocab multiples of 8, every pointer 16-byte aligned.
+struct TcFusedArgs {
+  const void* hidden;   // [rows, hidden_dim]
+  const void* lm_head;  // [vocab, hidden_dim]
+  const int64_t* ids;   // [rows]
+  const void* w1;       // [vocab, rank]
+  const void* w2;       // [vocab, rank]
+  void* out;            // [rows, vocab]
+  int64_t rows, hidden_dim, vocab;
+  int32_t rank;
+  int32_t out_f32;
+  uint32_t* status;
+  uint64_t wait_limit_ns;
+};
+bool tc_fused_supported(int64_t rows, int64_t hidden_dim, int64_t vocab, int32_t rank, int out_dtype,
+                        int weight_dtype);
+cudaError_t launch_tc_fused(const TcFusedArgs& a, int num_sms, cudaStream_t s);
 
 // Encodes a tiled TMA descriptor through the driver entry point.
 bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t rank, const void* base,

@@ -1,0 +1,751 @@
+// Left-to-right block sampling on the sm_100a tensor cores, batch rows on the
+// MMA's M side (VanillaMarkov.sample_block_tokens and _sample_tokens of the
+// vendored markov_head.py). For k = 0 .. M-1 and every block b:
+//
+//     c_k[b, v] = round_bf16( U[b, k, v] + sum_j W1[x_{k-1}[b], j] * W2[v, j] )
+//     x_k[b]    = argmax_v c_k[b, v]                    (greedy)
+//              or argmax_v c_k[b, v] / T + g(b, k, v)   (Gumbel-max, Philox noise)
+//
+// with x_{-1} = first_prev, in one cooperative persistent launch for all M
+// steps. CTA c owns a contiguous range of vocabulary ids (a multiple of 16),
+// cut into chunks of up to 256 ids.
+//
+// Why this layout. A tcgen05.mma costs the same time whatever its N (16 to
+// 256) on this part, so the ids go on N, 256 at a time, and the batch on M:
+// D[lane][id] = X[lane] . W2[id]^T with A = X = W1[x_{k-1}] rows in shared
+// memory and B = a W2 chunk. M is 128, so the batch (padded to BP = 32, 64 or
+// 128 rows) is repeated REP = 128 / BP times down the lanes; each repeat
+// serves a different part of the chunk's columns, so that all four TMEM lane
+// quarters (one per epilogue warp quarter) carry useful rows. An epilogue
+// thread owns one batch row and runs along contiguous ids: 16-byte loads of
+// U and stores of the corrected logits straight to global memory, a
+// thread-local running maximum, and one Philox call per four ids.
+//
+// W2 stays on chip: the CTA's chunks are loaded into shared memory once; when
+// they do not all fit (rank 128 and above), the rest stream from L2 through a
+// two-slot ring every step, ordered so that their loads hide behind the
+// resident chunks' MMAs and the grid barrier. U is prefetched into L2 one step
+// ahead with bulk prefetches (it does not depend on the chain).
+//
+// Per step: the gather warp waits at the grid barrier (bounded), decodes
+// x_{k-1} from the global keys and gathers X by TMA tile::gather4; the MMA
+// warp runs the chunks into two alternating 256-column accumulators; the
+// epilogue rounds, stores and selects; the CTA's per-row maxima go to the
+// global keys with one red.max each, and one release-add arrives at the
+// barrier.
+//
+// Warp roles (640 threads): 0 W2 loader and ring producer; 1 TMEM owner and
+// MMA issuer; 3 grid barrier, key decode, X gather and U prefetch; 4-19
+// epilogue (warp 4 + 4e + q reads TMEM lane quarter q); 2 has no role.
+#include <type_traits>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace dspark {
+namespace {
+
+constexpr int kChunk = 256;                      // ids per chunk (MMA N at most)
+constexpr int kGroup = 16;                       // ids per epilogue piece (one tcgen05.ld x16)
+constexpr int kEpiWarps = 16;
+constexpr int kEpiPerQuarter = kEpiWarps / 4;    // E
+constexpr int kThreads = 128 + kEpiWarps * 32;
+constexpr uint32_t kTmemCols = 512;              // two 256-column accumulators
+constexpr uint32_t kXAtomBytes = 128 * 128;      // 128 rows x 64 bf16
+constexpr uint32_t kFullBlockBytes = kChunk * 128;  // 256 ids x 64 bf16
+constexpr int kMaxChunks = 8;
+constexpr size_t kSmemLimit = 232448;
+
+struct __align__(64) RowsMaps {
+  CUtensorMap w2;     // [vocab, rank] bf16, box 64 x 256, 128B swizzle
+  CUtensorMap w2_16;  // same tensor, box 64 x 16 (the last, partial chunk)
+  CUtensorMap w1;     // [vocab, rank] bf16, box 64 x 1 (row gathers), 128B swizzle
+};
+
+struct RowsParams {
+  const __nv_bfloat16* base;  // [B, M, V]
+  __nv_bfloat16* out;         // [B, M, V]
+  const int64_t* first_prev;
+  const __nv_bfloat16* w1;
+  int64_t* tokens;
+  unsigned long long* keys;
+  uint32_t* barrier;
+  uint32_t* status;
+  int64_t vocab;
+  int32_t batch, bp, steps, ka;
+  int32_t groups;        // 16-id groups of the vocabulary
+  int32_t resident_full; // full chunks a CTA keeps in shared memory (the rest stream)
+  uint32_t w2_bytes;     // shared memory reserved for resident W2 blocks
+  int32_t ring;          // 1 when the streaming ring exists
+  float temperature;
+  PhiloxRoundKeys round_keys;
+  uint64_t wait_limit_ns;
+  uint32_t debug_flags;
+};
+
+struct RowsTail {
+  uint64_t w2_full;
+  uint64_t ring_full[2], ring_empty[2];
+  uint64_t x_full, x_empty;
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t drain;
+  int32_t xid[128];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// The CTA's vocabulary range and its chunks: ids [v0, v1), chunk j starts at
+// v0 + 256 j; all chunks but the last are full.
+struct Range {
+  int64_t v0, v1;
+  int nchunks, nfull;
+  __device__ int width(int j) const {
+    const int64_t w = ((v1 - v0 + 15) & ~15ll) - (int64_t)kChunk * j;
+    return w < kChunk ? (int)w : kChunk;  // MMA N: a multiple of 16
+  }
+};
+
+__device__ __forceinline__ Range cta_range(const RowsParams& p) {
+  Range r;
+  const int64_t g0 = (int64_t)p.groups * blockIdx.x / gridDim.x;
+  const int64_t g1 = (int64_t)p.groups * (blockIdx.x + 1) / gridDim.x;
+  r.v0 = g0 * kGroup;
+  r.v1 = g1 * kGroup < p.vocab ? g1 * kGroup : p.vocab;
+  // Chunks are counted on the length rounded up to 16 ids, as the plan does
+  // (the last range can end 8 ids short of a group; those rows read as zero).
+  const int64_t n16 = (r.v1 - r.v0 + 15) & ~15ll;
+  r.nchunks = (int)((n16 + kChunk - 1) / kChunk);
+  r.nfull = (int)(n16 / kChunk);
+  return r;
+}
+
+// Per-step chunk order: the first streamed chunk (its blocks were prefetched
+// into the ring during the previous step), then the resident chunks (the
+// remaining streamed blocks load behind their MMAs), then the other streamed
+// chunks. Chunks [0, res) are resident, [res, nfull) stream, and a partial
+// last chunk is always resident.
+__device__ __forceinline__ int resident_full_of(const Range& r, const RowsParams& p) {
+  return r.nfull < p.resident_full ? r.nfull : p.resident_full;
+}
+
+// The chunk at position i of the step's order (i < r.nchunks).
+__device__ __forceinline__ int chunk_at(int i, const Range& r, int res) {
+  if (res < r.nfull) {  // streaming: the first streamed chunk leads
+    if (i == 0) return res;
+    i -= 1;
+  }
+  if (i < res) return i;
+  i -= res;
+  if (r.nchunks > r.nfull) {  // the partial chunk
+    if (i == 0) return r.nfull;
+    i -= 1;
+  }
+  return res + 1 + i;
+}
+
+// Shared-memory offset of resident block (chunk j, atom a) inside the W2 area:
+// full chunks first (ka atoms of 32 KB each), then the partial chunk.
+__device__ __forceinline__ uint32_t resident_offset(int j, int a, const Range& r, int res, int ka) {
+  if (j < r.nfull) return (uint32_t)(j * ka + a) * kFullBlockBytes;
+  const uint32_t pw = (uint32_t)r.width(j);
+  return (uint32_t)res * ka * kFullBlockBytes + (uint32_t)a * pw * 128u;
+}
+
+__device__ __forceinline__ bool barrier_and(bool v, uint32_t id, uint32_t n) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"((uint32_t)v), "r"(id), "r"(n)
+      : "memory");
+  return out != 0;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_max_gpu(unsigned long long* p, unsigned long long v) {
+  asm volatile("red.relaxed.gpu.global.max.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ void red_add_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p) : "memory");
+}
+
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_relaxed_gpu(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void st_stream_v4(void* p, uint4 v) {
+  asm volatile("st.global.cs.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// A warp-uniform bounded wait: lane 0 waits, the warp follows its verdict, and
+// the other lanes then observe the (already completed) phase themselves.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl, int lane) {
+  bool ok = lane == 0 ? mbar_wait(bar, parity, ctl) : true;
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  if (ok && lane != 0) mbar_wait(bar, parity, ctl);
+  return ok;
+}
+
+__device__ __forceinline__ bool grid_wait(const uint32_t* counter, uint32_t target, const WaitCtl& ctl, int lane) {
+  bool ok = true;
+  if (lane == 0) {
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_gpu(counter) < target) {
+      if (*ctl.abort_flag) {
+        ok = false;
+        break;
+      }
+      if (globaltimer_ns() - t0 > ctl.limit_ns) {
+        *ctl.abort_flag = 1;
+        atomicOr(ctl.status, DSPARK_STATUS_TIMEOUT);
+        ok = false;
+        break;
+      }
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  __syncwarp();
+  return ok;
+}
+
+// Order-preserving bits of a bf16 value held in the high half of `w` (the low
+// half is ignored): the sign bit set for non-negative values, every bit
+// flipped for negative ones; the low 16 bits of the result are zero.
+__device__ __forceinline__ uint32_t ordered_hi16(uint32_t w) {
+  return (w ^ ((uint32_t)((int32_t)w >> 31) | 0x80000000u)) & 0xFFFF0000u;
+}
+
+// Order-preserving bits of an fp32 score (see the tile sampler): +0 first
+// turns -0 into +0 and any NaN into the canonical positive NaN.
+__device__ __forceinline__ uint32_t ordered_bits(float x) {
+  const uint32_t b = __float_as_uint(x + 0.0f);
+  return b ^ ((uint32_t)((int32_t)b >> 31) | 0x80000000u);
+}
+
+// Corrected logits of two ids as one bf16x2 word: U (two bf16 in `u2`) plus
+// the fp32 bias, rounded once. Adding +0 makes a -0 sum +0 and keeps NaN the
+// canonical positive NaN, so the selection keys need no further care.
+__device__ __forceinline__ uint32_t add_round2(uint32_t u2, uint32_t a_lo, uint32_t a_hi) {
+  const float lo = __uint_as_float(u2 << 16) + __uint_as_float(a_lo) + 0.0f;
+  const float hi = __uint_as_float(u2 & 0xFFFF0000u) + __uint_as_float(a_hi) + 0.0f;
+  __nv_bfloat162 o = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&o);
+}
+
+template <int KA, bool GREEDY>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_sample_rows_kernel(const __grid_constant__ RowsMaps maps, const RowsParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* w2_smem = smem;                                     // resident W2 blocks
+  uint8_t* ring_smem = w2_smem + p.w2_bytes;                   // 2 x 32 KB when streaming
+  uint8_t* x_smem = ring_smem + (p.ring ? 2 * kFullBlockBytes : 0u);  // KA atoms of 16 KB
+  unsigned long long* red = reinterpret_cast<unsigned long long*>(x_smem + KA * kXAtomBytes);  // [128]
+  RowsTail* sh = reinterpret_cast<RowsTail*>(red + 128);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int G = gridDim.x;
+  const int M = p.steps;
+  const int B = p.batch;
+  const int BP = p.bp;
+  const Range rg = cta_range(p);
+  const int res = resident_full_of(rg, p);
+  const int nc = rg.nchunks;
+  const bool has_partial = rg.nchunks > rg.nfull;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sh->w2_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh->ring_full[i], 1);
+      mbar_init(&sh->ring_empty[i], 1);
+      mbar_init(&sh->acc_full[i], 1);
+      mbar_init(&sh->acc_empty[i], kEpiWarps);
+    }
+    mbar_init(&sh->x_full, 1);
+    mbar_init(&sh->x_empty, 1);
+    mbar_init(&sh->drain, 1);
+    sh->abort_flag = 0;
+    fence_barrier_init();
+  }
+  for (int i = threadIdx.x; i < 128; i += blockDim.x) red[i] = 0ull;
+  if (warp == 1) {
+    tmem_alloc(&sh->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  __syncwarp();
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = sh->tmem_base;
+  const WaitCtl ctl{&sh->abort_flag, p.status, p.wait_limit_ns};
+  volatile int never = 0;
+  const WaitCtl drain_ctl{&never, p.status, p.wait_limit_ns};
+
+  if (warp == 0) {
+    // ------------------------- resident W2, then the streaming ring ----
+    if (lane == 0) {
+      prefetch_tensormap(&maps.w2);
+      prefetch_tensormap(&maps.w2_16);
+      const uint64_t pol = policy_evict_last();
+      const uint32_t pw = has_partial ? (uint32_t)rg.width(rg.nfull) : 0u;
+      const uint32_t bytes = (uint32_t)res * KA * kFullBlockBytes + (uint32_t)KA * pw * 128u;
+      if (bytes) {
+        mbar_arrive_expect_tx(&sh->w2_full, bytes);
+        for (int j = 0; j < res; ++j)
+          for (int a = 0; a < KA; ++a)
+            tma_load_2d(w2_smem + resident_offset(j, a, rg, res, KA), &maps.w2, &sh->w2_full, a * 64,
+                        (int32_t)(rg.v0 + (int64_t)kChunk * j), pol);
+        if (has_partial)
+          for (int a = 0; a < KA; ++a)
+            for (uint32_t r = 0; r < pw; r += 16)
+              tma_load_2d(w2_smem + resident_offset(rg.nfull, a, rg, res, KA) + r * 128u, &maps.w2_16,
+                          &sh->w2_full, a * 64, (int32_t)(rg.v0 + (int64_t)kChunk * rg.nfull + r), pol);
+      }
+      // Streamed chunks, every step, in the MMA order.
+      int64_t gs = 0;
+      bool ok = true;
+      for (int k = 0; k < M && ok; ++k)
+        for (int i = 0; i < nc && ok; ++i) {
+          const int j = chunk_at(i, rg, res);
+          if (j < res || j >= rg.nfull) continue;
+          for (int a = 0; a < KA; ++a, ++gs) {
+            const int s = (int)(gs & 1);
+            if (!mbar_wait(&sh->ring_empty[s], ((uint32_t)(gs >> 1) & 1u) ^ 1u, ctl)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&sh->ring_full[s], kFullBlockBytes);
+            tma_load_2d(ring_smem + s * kFullBlockBytes, &maps.w2, &sh->ring_full[s], a * 64,
+                        (int32_t)(rg.v0 + (int64_t)kChunk * j), pol);
+          }
+        }
+      for (int64_t j = (gs > 2 ? gs - 2 : 0); j < gs; ++j)
+        mbar_wait(&sh->ring_full[j & 1], (uint32_t)(j >> 1) & 1u, drain_ctl);
+      if (bytes) mbar_wait(&sh->w2_full, 0, drain_ctl);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------- MMA issuer ----
+    if (lane == 0) {
+      const uint64_t x_desc = sw128_kmajor_desc(smem_u32(x_smem));
+      const uint32_t w2_base = smem_u32(w2_smem);
+      const uint32_t ring_base = smem_u32(ring_smem);
+      bool ok = !(res > 0 || has_partial) || mbar_wait(&sh->w2_full, 0, ctl);
+      int64_t t = 0, gs = 0;
+      for (int k = 0; k < M && ok; ++k) {
+        if (!mbar_wait(&sh->x_full, (uint32_t)k & 1u, ctl)) break;
+        for (int i = 0; i < nc && ok; ++i, ++t) {
+          const int j = chunk_at(i, rg, res);
+          const int buf = (int)(t & 1);
+          if (!mbar_wait(&sh->acc_empty[buf], ((uint32_t)(t >> 1) & 1u) ^ 1u, ctl)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t idesc = idesc_bf16_f32(128, (uint32_t)rg.width(j));
+          const uint32_t d_tmem = tmem_base + (uint32_t)(buf * kChunk);
+          const bool streamed = j >= res && j < rg.nfull;
+          for (int a = 0; a < KA; ++a) {
+            uint32_t b_addr;
+            int s = 0;
+            if (streamed) {
+              s = (int)(gs & 1);
+              if (!mbar_wait(&sh->ring_full[s], (uint32_t)(gs >> 1) & 1u, ctl)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after_sync();
+              b_addr = ring_base + (uint32_t)s * kFullBlockBytes;
+            } else {
+              b_addr = w2_base + resident_offset(j, a, rg, res, KA);
+            }
+            const uint64_t b_desc = sw128_kmajor_desc(b_addr);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16_ss(d_tmem, desc_advance(x_desc, (uint32_t)a * kXAtomBytes + kk * 32),
+                           desc_advance(b_desc, kk * 32), idesc, (a | kk) != 0);
+            if (streamed) {
+              umma_commit(&sh->ring_empty[s]);
+              ++gs;
+            }
+          }
+          if (ok) umma_commit(&sh->acc_full[buf]);
+        }
+        if (ok) umma_commit(&sh->x_empty);
+      }
+      umma_commit(&sh->drain);
+      mbar_wait(&sh->drain, 0, drain_ctl);
+    }
+  } else if (warp == 3) {
+    // ------------------------- grid barrier, X gather, U prefetch ----
+    const uint64_t pol_w1 = policy_evict_last();
+    if (lane == 0) prefetch_tensormap(&maps.w1);
+    // U of step k is prefetched into L2 (bulk prefetch of each row's range)
+    // one step ahead: it does not depend on the chain.
+    const uint32_t row_bytes = (uint32_t)((rg.v1 - rg.v0) * 2);
+    auto prefetch_u = [&](int k) {
+      for (int b = lane; b < B && row_bytes; b += 32)
+        bulk_prefetch_l2(p.base + ((int64_t)b * M + k) * p.vocab + rg.v0, row_bytes);
+    };
+    prefetch_u(0);
+    int armed = -1;  // the last step whose gather was issued
+    for (int k = 0; k < M; ++k) {
+      if (!warp_wait(&sh->x_empty, ((uint32_t)k & 1u) ^ 1u, ctl, lane)) break;
+      // Every CTA has merged its step k-1 maxima once the counter reaches k * G.
+      if (k > 0 && !grid_wait(p.barrier, (uint32_t)k * (uint32_t)G, ctl, lane)) break;
+      bool bad = false;
+      for (int b = lane; b < BP; b += 32) {
+        int32_t row = (int32_t)p.vocab;  // outside the tensor: the gather reads zeros
+        if (b < B) {
+          const int64_t id =
+              k == 0 ? p.first_prev[b] : (int64_t)key_token(ld_relaxed_gpu(&p.keys[(size_t)(k - 1) * B + b]));
+          if (k > 0 && blockIdx.x == 0) p.tokens[(size_t)b * M + (k - 1)] = id;
+          if (id < 0 || id >= p.vocab)
+            bad = true;
+          else
+            row = (int32_t)id;
+        }
+        sh->xid[b] = row;
+      }
+      if (bad) report_status(p.status, DSPARK_STATUS_TOKEN_RANGE);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_expect_tx(&sh->x_full, (uint32_t)KA * kXAtomBytes);
+      armed = k;
+      __syncwarp();
+      // Lane L of the operand holds batch row L % BP; lane i gathers lanes 4i..4i+3.
+#pragma unroll
+      for (int a = 0; a < KA; ++a) {
+        const int l0 = 4 * lane;
+        tma_gather4(x_smem + (uint32_t)a * kXAtomBytes + (uint32_t)l0 * 128u, &maps.w1, &sh->x_full, a * 64,
+                    sh->xid[l0 % BP], sh->xid[(l0 + 1) % BP], sh->xid[(l0 + 2) % BP], sh->xid[(l0 + 3) % BP],
+                    pol_w1);
+      }
+      __syncwarp();
+      if (k + 1 < M) prefetch_u(k + 1);
+      if (k == M - 1 && blockIdx.x == 0) {
+        // The last step's tokens, once every CTA has merged its maxima.
+        if (grid_wait(p.barrier, (uint32_t)M * (uint32_t)G, ctl, lane))
+          for (int b = lane; b < B; b += 32)
+            p.tokens[(size_t)b * M + (M - 1)] = (int64_t)key_token(ld_relaxed_gpu(&p.keys[(size_t)(M - 1) * B + b]));
+      }
+    }
+    // The last gather has landed before the CTA may exit (it has unless a
+    // wait gave up before the MMAs consumed it).
+    if (lane == 0 && armed >= 0) mbar_wait(&sh->x_full, (uint32_t)armed & 1u, drain_ctl);
+  } else if (warp >= 4) {
+    // -------------------------------------------------- epilogue ----
+    const int ew = warp - 4;
+    const int q = ew & 3;             // TMEM lane quarter
+    const int e = ew >> 2;            // which of the quarter's warps
+    const int L = 32 * q + lane;      // accumulator lane = operand row
+    const int b = L % BP;             // batch row
+    const int rep = 128 / BP;
+    const int slot = (L / BP) * kEpiPerQuarter + e;
+    const int nslots = rep * kEpiPerQuarter;
+    const bool row_ok = b < B;
+    const uint32_t lane_base = tmem_base + ((uint32_t)(32 * q) << 16);
+    const int te = threadIdx.x - 128;
+    const uint32_t all_n = kEpiWarps * 32;
+    const float inv_t = GREEDY ? 0.0f : 1.0f / p.temperature;
+    // The pieces (step k, chunk position i, 16-id group g) this thread works
+    // on, in order; U of the next piece is loaded one piece ahead (across
+    // chunk and step boundaries), so its latency hides behind the current
+    // piece and the accumulator waits.
+    struct Cursor {
+      int k, i, g;
+    };
+    auto settle = [&](Cursor& c) {  // move to the first existing piece at or after c
+      while (c.k < M) {
+        if (c.g < rg.width(chunk_at(c.i, rg, res)) / kGroup) return;
+        c.g = slot;
+        if (++c.i == nc) {
+          c.i = 0;
+          ++c.k;
+        }
+      }
+    };
+    auto load_u = [&](const Cursor& c, uint4& a0, uint4& a1) {
+      if (!row_ok || c.k >= M) return;
+      const int64_t v = rg.v0 + (int64_t)kChunk * chunk_at(c.i, rg, res) + (int64_t)kGroup * c.g;
+      const __nv_bfloat16* src = p.base + ((size_t)b * M + c.k) * (size_t)p.vocab + v;
+      a0 = ld_stream_v4(src);
+      if (v + kGroup <= p.vocab) a1 = ld_stream_v4(src + 8);
+    };
+    Cursor nxt{0, 0, slot};
+    settle(nxt);
+    uint4 nu0 = make_uint4(0u, 0u, 0u, 0u), nu1 = nu0;
+    load_u(nxt, nu0, nu1);
+    int64_t t = 0;
+    bool ok = true;
+    for (int k = 0; k < M && ok; ++k) {
+      const size_t row_off = ((size_t)b * M + k) * (size_t)p.vocab;
+      uint32_t best = 0u;      // greedy: (ordered bf16 bits, 0xFFFF - local id); temperature: ordered score
+      uint32_t best_lid = 0u;  // temperature: the CTA-local id of `best`
+      for (int i = 0; i < nc; ++i, ++t) {
+        const int j = chunk_at(i, rg, res);
+        const int buf = (int)(t & 1);
+        const int ngroups = rg.width(j) / kGroup;
+        const int64_t c0 = rg.v0 + (int64_t)kChunk * j;
+        if (!warp_wait(&sh->acc_full[buf], (uint32_t)(t >> 1) & 1u, ctl, lane)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        for (int g = slot; g < ngroups; g += nslots) {
+          const int64_t v = c0 + (int64_t)kGroup * g;  // first id of the piece (== nxt)
+          const bool full = v + kGroup <= p.vocab;     // else only the first 8 ids exist
+          const uint4 u0 = nu0, u1 = nu1;
+          nxt.g += nslots;
+          settle(nxt);
+          nu1 = make_uint4(0u, 0u, 0u, 0u);
+          load_u(nxt, nu0, nu1);
+          uint32_t d[16];
+          __syncwarp();  // tcgen05.ld is warp-aligned
+          tmem_ld_32x32b_x16(lane_base + (uint32_t)(buf * kChunk + kGroup * g), d);
+          tmem_ld_wait();
+          if (!row_ok) continue;
+          uint32_t c[8];
+          c[0] = add_round2(u0.x, d[0], d[1]);
+          c[1] = add_round2(u0.y, d[2], d[3]);
+          c[2] = add_round2(u0.z, d[4], d[5]);
+          c[3] = add_round2(u0.w, d[6], d[7]);
+          c[4] = add_round2(u1.x, d[8], d[9]);
+          c[5] = add_round2(u1.y, d[10], d[11]);
+          c[6] = add_round2(u1.z, d[12], d[13]);
+          c[7] = add_round2(u1.w, d[14], d[15]);
+          st_stream_v4(p.out + row_off + v, make_uint4(c[0], c[1], c[2], c[3]));
+          if (full) st_stream_v4(p.out + row_off + v + 8, make_uint4(c[4], c[5], c[6], c[7]));
+          const int nid = full ? 16 : 8;
+          const uint32_t lid0 = (uint32_t)(v - rg.v0);
+          if constexpr (GREEDY) {
+            const uint32_t low0 = 0xFFFFu - lid0;
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+              if (2 * m >= nid) break;
+              const uint32_t klo = ordered_hi16(c[m] << 16) + (low0 - 2 * m);
+              const uint32_t khi = ordered_hi16(c[m]) + (low0 - 2 * m - 1);
+              best = max(best, max(klo, khi));
+            }
+          } else {
+#pragma unroll
+            for (int m4 = 0; m4 < 4; ++m4) {
+              if (4 * m4 >= nid) break;
+              const uint32_t vq = (uint32_t)(v + 4 * m4);
+              const Philox4 r = philox4x32_10(vq >> 2, (uint32_t)k, (uint32_t)b, 0u, p.round_keys);
+              const uint32_t w4[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+              for (int i4 = 0; i4 < 4; ++i4) {
+                const uint32_t cw = c[2 * m4 + (i4 >> 1)];
+                const float cv = __uint_as_float((i4 & 1) ? (cw & 0xFFFF0000u) : (cw << 16));
+                const uint32_t o = ordered_bits(cv * inv_t + gumbel_from_word(w4[i4]));
+                if (o > best) {
+                  best = o;
+                  best_lid = lid0 + 4 * m4 + i4;
+                }
+              }
+            }
+          }
+        }
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->acc_empty[buf]);
+      }
+      // The epilogue warps agree to go on (an abort anywhere ends every step).
+      if (!barrier_and(ok, 1, all_n)) break;
+      // This CTA's maximum per row: one shared 64-bit atomic per thread, then
+      // one global red.max per row (orderable score, complement of the id).
+      if (row_ok) {
+        unsigned long long key;
+        if constexpr (GREEDY) {
+          const uint32_t vid = (uint32_t)rg.v0 + (0xFFFFu - (best & 0xFFFFu));
+          key = best ? ((unsigned long long)(best >> 16) << 32) | (unsigned long long)(0xFFFFFFFFu - vid) : 0ull;
+        } else {
+          const uint32_t vid = (uint32_t)rg.v0 + best_lid;
+          key = best ? ((unsigned long long)best << 32) | (unsigned long long)(0xFFFFFFFFu - vid) : 0ull;
+        }
+        if (key) atomicMax(&red[b], key);
+      }
+      named_barrier_sync(1, all_n);
+      if (te < B) {
+        const unsigned long long key = red[te];
+        red[te] = 0ull;
+        if (key) {
+          red_max_gpu(&p.keys[(size_t)k * B + te], key);
+          if (k + 1 < M) prefetch_l2(p.w1 + (size_t)key_token(key) * (size_t)(KA * 64));
+        }
+      }
+      // The maxima are merged before the arrival: the release below is
+      // cumulative over the other threads' reductions ordered by this barrier.
+      named_barrier_sync(1, all_n);
+      if (te == 0) {
+        const bool skip = (p.debug_flags & DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL) && blockIdx.x == 0 && k == 0;
+        if (!skip) red_add_release_gpu(p.barrier, 1u);
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+}
+
+struct RowsPlan {
+  int bp, resident_full, ring;
+  uint32_t w2_bytes;
+  size_t smem;
+  bool ok;
+};
+
+RowsPlan rows_plan(int64_t batch, int64_t vocab, int32_t rank, int grid) {
+  RowsPlan c{};
+  if (batch < 1 || batch > 128 || rank % 64 != 0 || rank < 64 || rank > 256 || vocab % 8 != 0 || grid < 1) return c;
+  c.bp = batch <= 32 ? 32 : batch <= 64 ? 64 : 128;
+  const int ka = rank / 64;
+  const int64_t groups = (vocab + 15) / 16;
+  // CTA ranges hold floor or ceil(groups / grid) groups of 16 ids.
+  const int64_t nmin = 16 * (groups / grid), nmax = 16 * ((groups + grid - 1) / grid);
+  if (nmin < 16 || nmax > 65535 || (nmax + kChunk - 1) / kChunk > kMaxChunks) return c;
+  const int nfull = (int)(nmax / kChunk);
+  const uint32_t full_bytes = (uint32_t)ka * kFullBlockBytes;
+  uint32_t part_bytes = 0;  // the larger partial chunk of the two range sizes
+  for (int64_t n : {nmin, nmax}) {
+    const uint32_t pb = (uint32_t)ka * (uint32_t)(n % kChunk) * 128u;
+    part_bytes = pb > part_bytes ? pb : part_bytes;
+  }
+  const size_t fixed = 1024 + (size_t)ka * kXAtomBytes + 128 * 8 + sizeof(RowsTail) + 64;
+  if (fixed >= kSmemLimit) return c;
+  const size_t budget = kSmemLimit - fixed;
+  const size_t ring_bytes = 2 * (size_t)kFullBlockBytes;
+  if ((size_t)nfull * full_bytes + part_bytes <= budget) {
+    c.resident_full = nfull;
+    c.ring = 0;
+  } else {
+    if (budget < ring_bytes + part_bytes) return c;
+    c.resident_full = (int)((budget - ring_bytes - part_bytes) / full_bytes);
+    c.ring = 1;
+  }
+  // Every CTA keeps min(its full chunks, resident_full) full chunks and its
+  // partial chunk, which fit in this area.
+  c.w2_bytes = (uint32_t)c.resident_full * full_bytes + part_bytes;
+  c.smem = fixed + c.w2_bytes + (c.ring ? ring_bytes : 0);
+  c.ok = c.smem <= kSmemLimit;
+  return c;
+}
+
+template <int KA, bool GREEDY>
+cudaError_t launch_rows_ka(const TcSampleArgs& a, const RowsPlan& c, int grid, cudaStream_t stream) {
+  RowsMaps maps;
+  const uint64_t wdim[2] = {(uint64_t)a.rank, (uint64_t)a.vocab};
+  const uint64_t wstr[1] = {(uint64_t)a.rank * 2};
+  const uint32_t box[2] = {64, (uint32_t)kChunk};
+  const uint32_t box16[2] = {64, 16};
+  const uint32_t rbox[2] = {64, 1};
+  if (!encode_tensor_map(&maps.w2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.w2, wdim, wstr, box,
+                         CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tensor_map(&maps.w2_16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.w2, wdim, wstr, box16,
+                         CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tensor_map(&maps.w1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.w1, wdim, wstr, rbox,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  RowsParams p{};
+  p.base = static_cast<const __nv_bfloat16*>(a.base);
+  p.out = static_cast<__nv_bfloat16*>(a.corrected);
+  p.first_prev = a.first_prev;
+  p.w1 = static_cast<const __nv_bfloat16*>(a.w1);
+  p.tokens = a.tokens;
+  p.keys = a.keys;
+  p.barrier = a.barrier;
+  p.status = a.status;
+  p.vocab = a.vocab;
+  p.batch = (int32_t)a.batch;
+  p.bp = c.bp;
+  p.steps = (int32_t)a.steps;
+  p.ka = KA;
+  p.groups = (int32_t)((a.vocab + 15) / 16);
+  p.resident_full = c.resident_full;
+  p.w2_bytes = c.w2_bytes;
+  p.ring = c.ring;
+  p.temperature = a.temperature;
+  p.round_keys = round_keys_for(a.seed);
+  p.wait_limit_ns = a.wait_limit_ns;
+  p.debug_flags = a.debug_flags;
+
+  cudaError_t e = cudaFuncSetAttribute(tc_sample_rows_kernel<KA, GREEDY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)c.smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = c.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, tc_sample_rows_kernel<KA, GREEDY>, maps, p);
+  note_launch();
+  return e;
+}
+
+template <bool GREEDY>
+cudaError_t launch_rows_mode(const TcSampleArgs& a, const RowsPlan& c, int grid, cudaStream_t s) {
+  switch (a.rank / 64) {
+    case 1: return launch_rows_ka<1, GREEDY>(a, c, grid, s);
+    case 2: return launch_rows_ka<2, GREEDY>(a, c, grid, s);
+    case 3: return launch_rows_ka<3, GREEDY>(a, c, grid, s);
+    case 4: return launch_rows_ka<4, GREEDY>(a, c, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+int rows_grid(int64_t vocab, int num_sms) {
+  const int64_t groups = (vocab + 15) / 16;
+  return (int)(groups < num_sms ? groups : num_sms);
+}
+
+}  // namespace
+
+bool tc_sample_rows_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype,
+                              int num_sms) {
+  if (logits_dtype != DSPARK_DTYPE_BF16 || weight_dtype != DSPARK_DTYPE_BF16) return false;
+  if (vocab < 16 || vocab >= (1ll << 31) - kChunk || num_sms < 1) return false;
+  return rows_plan(batch, vocab, rank, rows_grid(vocab, num_sms)).ok;
+}
+
+cudaError_t launch_tc_sample_rows(const TcSampleArgs& a, int num_sms, cudaStream_t s) {
+  const int grid = rows_grid(a.vocab, num_sms);
+  const RowsPlan c = rows_plan(a.batch, a.vocab, a.rank, grid);
+  if (!c.ok) return cudaErrorInvalidValue;
+  return a.greedy ? launch_rows_mode<true>(a, c, grid, s) : launch_rows_mode<false>(a, c, grid, s);
+}
+
+}  // namespace dspark

@@ -725,8 +725,10 @@ cudaError_t launch_mode(const TcSampleArgs& a, int num_sms, cudaStream_t s) {
 
 }  // namespace
 
-bool tc_sample_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype,
-                         int num_sms) {
+namespace {
+
+bool tile_sample_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype,
+                           int num_sms) {
   if (logits_dtype != DSPARK_DTYPE_BF16 || weight_dtype != DSPARK_DTYPE_BF16) return false;
   if (vocab % 8 != 0 || rank % 64 != 0 || rank < 64 || rank > 256) return false;
   if (batch < 1 || batch > kMaxBatch) return false;
@@ -740,7 +742,21 @@ bool tc_sample_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_
   return plan(rank / 64, (int)batch, batch_pad_of(batch), (int)per_cta).ok;
 }
 
-cudaError_t launch_tc_sample(const TcSampleArgs& a, int num_sms, cudaStream_t s) {
+}  // namespace
+
+bool tc_sample_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype,
+                         int num_sms) {
+  return tc_sample_rows_supported(batch, vocab, rank, logits_dtype, weight_dtype, num_sms) ||
+         tile_sample_supported(batch, vocab, rank, logits_dtype, weight_dtype, num_sms);
+}
+
+// The row-layout kernel where it applies (batch up to 128), else this file's
+// tile kernel (vocabulary ids on the MMA's M side, batch up to 256).
+cudaError_t launch_tc_sample(const TcSampleArgs& a, int num_sms, cudaStream_t s, int* variant) {
+  if (tc_sample_rows_supported(a.batch, a.vocab, a.rank, DSPARK_DTYPE_BF16, DSPARK_DTYPE_BF16, num_sms)) {
+    *variant |= DSPARK_VARIANT_SAMPLE_ROWS;
+    return launch_tc_sample_rows(a, num_sms, s);
+  }
   return a.greedy ? launch_mode<true>(a, num_sms, s) : launch_mode<false>(a, num_sms, s);
 }
 

@@ -103,6 +103,46 @@ class VanillaMarkov:
         N.check(code, "dspark_markov_apply_block_logits")
         return out
 
+    def fused_lm_head_logits(self, hidden_states: torch.Tensor, lm_head_weight: torch.Tensor, *,
+                             token_ids: torch.Tensor, out_dtype: torch.dtype = torch.float32,
+                             out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Corrected logits with the base logits made in the same kernel:
+        round(hidden @ lm_head_weight^T + bias(token_ids)), one fp32
+        accumulation and one rounding, the base logits never stored.
+        ``hidden_states`` (..., d) and ``lm_head_weight`` [V, d] are bf16 like
+        the head's weights; ``token_ids`` (...) are the teacher-forced previous
+        tokens. Returns (..., V) in ``out_dtype`` (fp32, as compute_logits
+        gives, or bf16)."""
+        d = hidden_states.shape[-1]
+        if tuple(lm_head_weight.shape) != (self.vocab_size, d):
+            raise ValueError(f"lm_head_weight must be [{self.vocab_size}, {d}]")
+        if tuple(token_ids.shape) != tuple(hidden_states.shape[:-1]):
+            raise ValueError("token_ids must match hidden_states without its last dim")
+        if hidden_states.dtype != self.weight_dtype or lm_head_weight.dtype != self.weight_dtype:
+            raise ValueError("hidden_states and lm_head_weight must have the head's weight dtype")
+        if out_dtype not in _DT:
+            raise ValueError("out_dtype must be float32 or bfloat16")
+        _check_cuda(hidden_states, "hidden_states", self.device)
+        _check_cuda(lm_head_weight, "lm_head_weight", self.device)
+        ids = (token_ids if token_ids.dtype == torch.int64 else token_ids.long()).contiguous()
+        _check_cuda(ids, "token_ids", self.device)
+        shape = tuple(hidden_states.shape[:-1]) + (self.vocab_size,)
+        if out is None:
+            out = torch.empty(shape, dtype=out_dtype, device=self.device)
+        else:
+            if tuple(out.shape) != shape or out.dtype != out_dtype:
+                raise ValueError("out must be (..., V) of out_dtype")
+            _check_cuda(out, "out", self.device)
+        rows = hidden_states.numel() // d
+        if rows == 0:
+            return out
+        code = self._lib.dspark_markov_fused_lm_head_logits(
+            hidden_states.data_ptr(), ids.data_ptr(), rows, d, self.vocab_size, lm_head_weight.data_ptr(),
+            self.markov_w1.data_ptr(), self.markov_w2.data_ptr(), self.markov_rank, out.data_ptr(), _DT[out_dtype],
+            _DT[self.weight_dtype], _stream_ptr(self.device))
+        N.check(code, "dspark_markov_fused_lm_head_logits")
+        return out
+
     def apply_step_logits(self, logits: torch.Tensor, *, token_ids: torch.Tensor,
                           hidden_states: Optional[torch.Tensor] = None) -> torch.Tensor:
         """One position (B, V) with its (B,) previous tokens."""
@@ -293,6 +333,12 @@ def launch_count() -> int:
 
 def last_algo() -> int:
     return int(N.load().dspark_markov_last_algo())
+
+
+def last_variant() -> int:
+    """DSPARK_VARIANT_* bits of the tensor-core variants the last call on this
+    thread launched."""
+    return int(N.load().dspark_markov_last_variant())
 
 
 def set_debug(flags: int, wait_limit_ns: int = 0) -> None:

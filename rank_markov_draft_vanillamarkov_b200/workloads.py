@@ -42,7 +42,9 @@ class Workload:
     base-logit tensor serves as the incoming gradient), ``"transition"``
     (the bias alone and the embeddings of the same rows, no base logits) or
     ``"sample"`` (left-to-right, ``batch`` blocks of ``proposal_len``
-    positions).
+    positions) or ``"fused"`` (teacher-forced, with the base logits made
+    from hidden states of width ``hidden`` by an LM-head weight [V, hidden];
+    ``logits_dtype`` is then the output dtype).
     """
 
     name: str
@@ -63,6 +65,9 @@ class Workload:
     temperature: float = 0.0
     philox_seed: int = 0
     data_seed: int = 0
+    hidden: int = 0  # fused: width of the hidden states
+    hidden_std: float = 1.0  # fused: hidden states ~N(0, hidden_std)
+    lm_std: float = 0.02  # fused: LM-head weight ~N(0, lm_std)
 
     @property
     def rows(self) -> int:
@@ -83,6 +88,10 @@ class Workload:
             r = self.rows
             return r * self.vocab * lb + self.vocab * self.rank * wb + r * self.rank * wb + r * 8 \
                 + 2 * self.vocab * self.rank * 4
+        if self.mode == "fused":  # hidden in, LM head and W2 once, W1 rows, ids, logits out
+            r = self.rows
+            return (r * self.hidden * wb + self.vocab * self.hidden * wb + self.vocab * self.rank * wb
+                    + r * self.rank * wb + r * 8 + r * self.vocab * lb)
         if self.mode == "transition":  # bias out, W2, W1 rows in and embeddings out, ids
             r = self.rows
             return r * self.vocab * wb + self.vocab * self.rank * wb + 2 * r * self.rank * wb + r * 8
@@ -91,6 +100,8 @@ class Workload:
                 + self.batch * 8 + r * 8)
 
     def flops(self) -> int:
+        if self.mode == "fused":
+            return 2 * self.rows * self.vocab * (self.hidden + self.rank)
         r = self.rows if self.mode in ("apply", "transition") else self.batch * self.proposal_len
         if self.mode == "backward":  # dW2 and dW1 each cost one product per (row, id, rank) term
             return 4 * self.rows * self.vocab * self.rank
@@ -121,6 +132,13 @@ TRANSITION_320 = Workload("transition_r320_v129280_k128", "transition", vocab=12
 APPLY_2560 = Workload("apply_r2560_v129280_k256_pad20", "apply", vocab=129280, rank=256, batch=8,
                       num_blocks=64, block_size=5, logit_std=2.0, weight_std=0.02,
                       prev_dist="zipf1.1", pad_frac=0.2, data_seed=0)
+
+# The fused producer on the 320-row layout: hidden width 5120 and the LM head
+# [129280, 5120] of DeepseekV41TextConfig (hidden_size, vocab_size), fp32
+# output as compute_logits gives.
+FUSED_320 = Workload("fused_lmhead_r320_d5120_v129280_k128", "fused", vocab=129280, rank=128, batch=4,
+                     num_blocks=16, block_size=5, logits_dtype="fp32", weight_std=0.02, prev_dist="zipf1.1",
+                     hidden=5120, hidden_std=1.0, lm_std=0.02, data_seed=0)
 
 GREEDY_BATCHES = (1, 8, 32, 64)
 
@@ -162,12 +180,20 @@ def make_inputs(wl: Workload) -> dict:
 
     apply:  base [B, nb, bs, V], prev_ids [B, nb, bs] int64, pad_mask [B, nb]
     sample: base [B, M, V], first_prev [B] int64
+    fused:  hidden [B, nb, bs, d], lm_head [V, d], prev_ids [B, nb, bs] int64
     plus w1, w2 [V, r].
     """
     g = torch.Generator().manual_seed(wl.data_seed)
     w1, w2 = make_weights(wl, g)
     out = {"w1": w1, "w2": w2}
-    if wl.mode == "transition":
+    if wl.mode == "fused":
+        n = wl.rows
+        ids = zipf_ids(g, n, wl.vocab, 1.1) if wl.prev_dist == "zipf1.1" else uniform_ids(g, n, wl.vocab)
+        out["prev_ids"] = ids.view(wl.batch, wl.num_blocks, wl.block_size)
+        out["hidden"] = _normal(g, (wl.batch, wl.num_blocks, wl.block_size, wl.hidden), wl.hidden_std,
+                                wl.weight_dtype)
+        out["lm_head"] = _normal(g, (wl.vocab, wl.hidden), wl.lm_std, wl.weight_dtype)
+    elif wl.mode == "transition":
         n = wl.rows
         ids = zipf_ids(g, n, wl.vocab, 1.1) if wl.prev_dist == "zipf1.1" else uniform_ids(g, n, wl.vocab)
         out["prev_ids"] = ids.view(wl.batch, wl.num_blocks, wl.block_size)

@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import oracle
-from rank_markov_draft_vanillamarkov_b200 import VanillaMarkov, device_status, last_algo, set_algo
+from rank_markov_draft_vanillamarkov_b200 import VanillaMarkov, device_status, last_algo, last_variant, set_algo
 from rank_markov_draft_vanillamarkov_b200 import _native as N
 from rank_markov_draft_vanillamarkov_b200 import workloads as W
 from rank_markov_draft_vanillamarkov_b200.build import build
@@ -66,8 +66,9 @@ def _run(w1, w2, dout, ids, algo, **kw):
     set_algo(algo)
     head = VanillaMarkov(w1.cuda(), w2.cuda())
     gw1, gw2 = head.apply_block_logits_backward(dout.cuda(), token_ids=ids.cuda(), **kw)
+    used = last_algo()
     torch.cuda.synchronize()
-    return gw1, gw2, last_algo()
+    return gw1, gw2, used
 
 
 @pytest.mark.parametrize("algo", [TC, GEN], ids=["tc", "generic"])
@@ -83,6 +84,28 @@ def test_backward_small(rows, vocab, rank, algo):
     gw1, gw2, used = _run(w1, w2, dout, ids, algo)
     assert used == (2 if algo == TC else 1)
     assert device_status() == 0
+    _check(w1, w2, dout, ids, gw1, gw2)
+
+
+@pytest.mark.parametrize("rows,rank,accumulate,resident", [
+    (130, 256, False, True),    # rank 256: four W1 boxes per row beside the resident block, the widest MMA
+    (192, 256, True, True),     # the largest row count that keeps rank 256 resident; TMA reduce-add epilogue
+    (193, 256, False, False),   # one more stage no longer fits: per-stage gathers
+    (330, 128, True, True),
+])
+def test_backward_resident_w1_choice(rows, rank, accumulate, resident):
+    """The tensor-core dW2 keeps every row's W1 row resident exactly when the
+    block fits beside three gradient stages; both forms match the oracle."""
+    w1, w2, dout, ids = _inputs(rows, 2056, rank, seed=rows + rank)
+    kw = {}
+    if accumulate:
+        kw = dict(grad_w1=torch.full((2056, rank), 0.5, device="cuda"),
+                  grad_w2=torch.full((2056, rank), -0.25, device="cuda"), accumulate=True)
+    gw1, gw2, used = _run(w1, w2, dout, ids, TC, **kw)
+    assert used == 2 and device_status() == 0
+    assert bool(last_variant() & N.DSPARK_VARIANT_BWD_RESIDENT_W1) == resident
+    if accumulate:
+        gw1, gw2 = kw["grad_w1"] - 0.5, kw["grad_w2"] + 0.25
     _check(w1, w2, dout, ids, gw1, gw2)
 
 

@@ -13,7 +13,8 @@ from scipy.special import softmax
 
 import oracle
 from oracle.checks import check_logits, check_sampled_block
-from rank_markov_draft_vanillamarkov_b200 import VanillaMarkov, device_status, last_algo, set_algo, set_debug
+from rank_markov_draft_vanillamarkov_b200 import (VanillaMarkov, device_status, last_algo, last_variant, set_algo,
+                                                 set_debug)
 from rank_markov_draft_vanillamarkov_b200 import _native as N
 from rank_markov_draft_vanillamarkov_b200 import workloads as W
 from rank_markov_draft_vanillamarkov_b200.build import build
@@ -34,14 +35,24 @@ def _lib():
     set_debug(0, 0)
 
 
+_VARIANT = {}
+
+
 def _sample(d, algo, temperature, seed=0, base=None, first=None):
     set_algo(algo)
     head = VanillaMarkov(d["w1"].cuda(), d["w2"].cuda())
     base = (d["base"] if base is None else base).cuda()
     first = (d["first_prev"] if first is None else first).cuda()
     toks, corr = head.sample_block_tokens(base, first_prev_token_ids=first, temperature=temperature, seed=seed)
+    _VARIANT["last"] = last_variant()
     torch.cuda.synchronize()
     return toks, corr, last_algo(), device_status()
+
+
+def _rows_kernel_ran() -> bool:
+    """The tensor-core sampler ran in its row layout (batch on the MMA's M
+    side), not the tile layout (vocabulary ids on M)."""
+    return bool(_VARIANT["last"] & N.DSPARK_VARIANT_SAMPLE_ROWS)
 
 
 def _check(d, toks, corr, temperature, seed, dtype="bf16", rows=None):
@@ -58,12 +69,17 @@ def _small(batch, vocab=1000, rank=64, m=5, wstd=0.3, seed=21, spike=6.0):
 
 
 @pytest.mark.parametrize("algo", [TC, GEN], ids=["tc", "generic"])
-@pytest.mark.parametrize("batch,vocab,rank", [(1, 1000, 64), (5, 2056, 128), (33, 1000, 192), (70, 4096, 256)])
+@pytest.mark.parametrize("batch,vocab,rank", [(1, 1000, 64), (5, 2056, 128), (33, 1000, 192), (70, 4096, 256),
+                                              (128, 2056, 64), (150, 4096, 128), (256, 1000, 64)])
 def test_greedy_small(batch, vocab, rank, algo):
+    """Batches up to 128 take the row-layout kernel (32, 64 or 128 padded
+    rows); 150 and 256 the tile-layout one."""
     wl = _small(batch, vocab, rank)
     d = W.make_inputs(wl)
     toks, corr, used, st = _sample(d, algo, 0.0)
     assert used == (2 if algo == TC else 1) and st == 0
+    if algo == TC:
+        assert _rows_kernel_ran() == (batch <= 128)
     # invariant: each token is the first argmax of its own corrected row
     assert torch.equal(toks, corr.float().argmax(-1))
     _check(d, toks, corr, 0.0, 0)
@@ -75,8 +91,31 @@ def test_greedy_full_size(batch):
     wl = W.greedy(batch)
     d = W.make_inputs(wl)
     toks, corr, used, st = _sample(d, AUTO, 0.0)
-    assert used == 2 and st == 0
+    assert used == 2 and st == 0 and _rows_kernel_ran()
     assert torch.equal(toks, corr.float().argmax(-1))
+    _check(d, toks, corr, 0.0, 0)
+
+
+@pytest.mark.parametrize("temperature", [0.0, 0.8])
+@pytest.mark.parametrize("rank", [192, 256])
+def test_row_kernel_streams_w2_at_large_ranks(rank, temperature):
+    """Full vocabulary at ranks 192 and 256: a CTA's W2 chunks do not all fit
+    in shared memory, so most stream from L2 through the two-slot ring every
+    step. Weights that move tokens; every (b, k) against the oracle."""
+    wl = W.greedy(24).with_(rank=rank, weight_std=0.3, spike=0.0, proposal_len=3, data_seed=30 + rank)
+    d = W.make_inputs(wl)
+    toks, corr, used, st = _sample(d, AUTO, temperature, seed=11)
+    assert used == 2 and st == 0 and _rows_kernel_ran()
+    _check(d, toks, corr, temperature, 11)
+
+
+def test_tile_kernel_full_vocabulary():
+    """Batch 140 (above the row layout's 128) at full vocabulary and rank 64:
+    the tile-layout kernel, every (b, k) against the oracle."""
+    wl = W.greedy(140).with_(rank=64, weight_std=0.3, spike=0.0, proposal_len=2, data_seed=41)
+    d = W.make_inputs(wl)
+    toks, corr, used, st = _sample(d, AUTO, 0.0)
+    assert used == 2 and st == 0 and not _rows_kernel_ran()
     _check(d, toks, corr, 0.0, 0)
 
 
@@ -97,7 +136,7 @@ def test_temperature_full_size():
     wl = W.TEMPERATURE
     d = W.make_inputs(wl)
     toks, corr, used, st = _sample(d, AUTO, wl.temperature, seed=wl.philox_seed)
-    assert used == 2 and st == 0
+    assert used == 2 and st == 0 and _rows_kernel_ran()
     rep = _check(d, toks, corr, wl.temperature, wl.philox_seed)
     assert rep.exact_required > 0.9 * wl.batch * wl.proposal_len
 
