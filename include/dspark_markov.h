@@ -251,9 +251,14 @@ int64_t dspark_markov_launch_count(void);
  * out and reports DSPARK_STATUS_TIMEOUT; no GPU fault is involved.
  */
 #define DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL 1u
-/* flags bit 1: the tensor-core apply uses 128-id units even where 256-id
- * units apply (both kernels stay testable). */
-#define DSPARK_DEBUG_APPLY_NARROW 2u
+/* flags bit 1: the tensor-core apply uses 256-id units where they apply
+ * (bf16 logits with a base, out != base_logits) instead of 128-id units.
+ * flags bit 2: the tensor-core sampler uses the row layout (batch on the MMA's
+ * M side) where it applies instead of the tile layout. Without these bits
+ * each call takes the variant that measured fastest on these shapes; both
+ * stay testable. */
+#define DSPARK_DEBUG_APPLY_WIDE 2u
+#define DSPARK_DEBUG_SAMPLE_ROWS 4u
 int dspark_markov_set_debug(uint32_t flags, uint64_t wait_limit_ns);
 
 /* Which kernel the last call on this thread selected: 0 none, 1 generic, 2 tensor core. */
@@ -269,14 +274,14 @@ int32_t dspark_markov_last_algo(void);
 #define DSPARK_VARIANT_BWD_RESIDENT_W1 1
 /*
  *   DSPARK_VARIANT_SAMPLE_ROWS: the tensor-core sampler ran with the batch on
- *     the MMA's M side and 256 vocabulary ids per MMA (batch <= 128);
+ *     the MMA's M side and 256 vocabulary ids per MMA (batch <= 128; chosen by
+ *     DSPARK_DEBUG_SAMPLE_ROWS, or where the tile layout does not fit);
  *     otherwise it ran with vocabulary ids on M and the batch on N.
  */
 #define DSPARK_VARIANT_SAMPLE_ROWS 2
 /*
  *   DSPARK_VARIANT_APPLY_WIDE: the tensor-core apply ran with units of 128 rows
- *     x 256 ids (bf16 logits with a base, out != base_logits); otherwise with
- *     128 x 128.
+ *     x 256 ids (chosen by DSPARK_DEBUG_APPLY_WIDE); otherwise with 128 x 128.
  */
 #define DSPARK_VARIANT_APPLY_WIDE 4
 int32_t dspark_markov_last_variant(void);

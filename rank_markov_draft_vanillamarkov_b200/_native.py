@@ -28,7 +28,8 @@ DSPARK_ALGO_GENERIC = 1
 DSPARK_ALGO_TENSOR_CORE = 2
 
 DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL = 1
-DSPARK_DEBUG_APPLY_NARROW = 2
+DSPARK_DEBUG_APPLY_WIDE = 2
+DSPARK_DEBUG_SAMPLE_ROWS = 4
 
 DSPARK_NOALLOC_MAX_KEYS = 8192
 

@@ -190,10 +190,9 @@ int dspark_markov_apply_block_logits(const void* base_logits, void* out, const i
     TcApplyArgs a{base_logits, out, prev_token_ids, rows, vocab, w1, w2, rank, d->status, g_wait_limit_ns.load(),
                   logits_dtype == DSPARK_DTYPE_FP32 ? 1 : 0};
     t_last_algo = 2;
-    // In-place calls (out == base) keep the 128-id kernel, whose unit reads
-    // and writes the same tile; the 256-id kernel takes the rest it supports.
-    const bool narrow = (g_debug_flags.load() & DSPARK_DEBUG_APPLY_NARROW) != 0 || out == base_logits;
-    if (!narrow && tc_apply_wide_supported(rows, vocab, rank, logits_dtype, weight_dtype, true)) {
+    // The 256-id kernel on request (in-place calls keep the 128-id one).
+    const bool wide = (g_debug_flags.load() & DSPARK_DEBUG_APPLY_WIDE) != 0 && out != base_logits;
+    if (wide && tc_apply_wide_supported(rows, vocab, rank, logits_dtype, weight_dtype, true)) {
       t_last_variant = DSPARK_VARIANT_APPLY_WIDE;
       return cuda_code(launch_tc_apply_wide(a, d->num_sms, s));
     }
@@ -368,7 +367,8 @@ int dspark_markov_sample_block(const void* base_logits, const int64_t* first_pre
     a.debug_flags = g_debug_flags.load();
     t_last_algo = 2;
     int variant = 0;
-    const cudaError_t e = launch_tc_sample(a, d->num_sms, s, &variant);
+    const bool rows = (g_debug_flags.load() & DSPARK_DEBUG_SAMPLE_ROWS) != 0;
+    const cudaError_t e = launch_tc_sample(a, d->num_sms, s, rows, &variant);
     t_last_variant = variant;
     return cuda_code(e);
   }
@@ -465,7 +465,8 @@ int dspark_markov_sample_block_noalloc(const void* base_logits, const int64_t* f
   a.debug_flags = g_debug_flags.load();
   t_last_algo = 2;
   int variant = 0;
-  const cudaError_t e = launch_tc_sample(a, st->num_sms, s, &variant);
+  const bool rows = (g_debug_flags.load() & DSPARK_DEBUG_SAMPLE_ROWS) != 0;
+  const cudaError_t e = launch_tc_sample(a, st->num_sms, s, rows, &variant);
   t_last_variant = variant;
   return cuda_code(e);
 }

@@ -313,7 +313,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;               // TMEM lane quarter this warp may access
     const int row = 32 * q + lane;
     const uint32_t bar_id = 1 + g;
-    int prev_s = -1;  // the stage of this group's previous unit, released one store later
     int64_t it = g;
     for (int64_t u = u_begin + g; u < u_end; u += 2, it += 2) {
       const int32_t n = (int32_t)(u / MT), m = (int32_t)(u % MT);
@@ -385,20 +384,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int bx = 0; bx < kUStageBytes / kAtomBytes; ++bx)
           tma_store_2d(&maps.out, st + bx * kAtomBytes, n * kBN + bx * kBoxIds, m * kBM);
         bulk_commit_group();
-        // The previous unit's stage may be refilled once its store has read
-        // it; this unit's store stays in flight while the group moves on.
-        if (prev_s >= 0) {
-          bulk_wait_group_read<1>();
-          mbar_arrive(&sh->u_empty[prev_s]);
-        }
-        prev_s = s;
+        bulk_wait_group_read<0>();  // the stage may be refilled once the store has read it
+        mbar_arrive(&sh->u_empty[s]);
       }
       __syncwarp();
     }
-    if (et == 0) {
-      bulk_wait_group<0>();
-      if (prev_s >= 0) mbar_arrive(&sh->u_empty[prev_s]);
-    }
+    if (et == 0) bulk_wait_group<0>();
   }
 
   // Single-lane roles and lane-0 branches leave warps diverged; bar.sync is

@@ -750,10 +750,13 @@ bool tc_sample_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_
          tile_sample_supported(batch, vocab, rank, logits_dtype, weight_dtype, num_sms);
 }
 
-// The row-layout kernel where it applies (batch up to 128), else this file's
-// tile kernel (vocabulary ids on the MMA's M side, batch up to 256).
-cudaError_t launch_tc_sample(const TcSampleArgs& a, int num_sms, cudaStream_t s, int* variant) {
-  if (tc_sample_rows_supported(a.batch, a.vocab, a.rank, DSPARK_DTYPE_BF16, DSPARK_DTYPE_BF16, num_sms)) {
+// This file's tile kernel (vocabulary ids on the MMA's M side, batch up to
+// 256), or the row-layout kernel (batch up to 128) on request or where the
+// tile kernel's on-chip plan does not fit.
+cudaError_t launch_tc_sample(const TcSampleArgs& a, int num_sms, cudaStream_t s, bool prefer_rows, int* variant) {
+  const bool rows_ok = tc_sample_rows_supported(a.batch, a.vocab, a.rank, DSPARK_DTYPE_BF16, DSPARK_DTYPE_BF16, num_sms);
+  const bool tile_ok = tile_sample_supported(a.batch, a.vocab, a.rank, DSPARK_DTYPE_BF16, DSPARK_DTYPE_BF16, num_sms);
+  if (rows_ok && (prefer_rows || !tile_ok)) {
     *variant |= DSPARK_VARIANT_SAMPLE_ROWS;
     return launch_tc_sample_rows(a, num_sms, s);
   }

@@ -37,11 +37,11 @@ def _lib():
 _VARIANT = {}
 
 
-@pytest.fixture(params=["wide", "narrow"])
+@pytest.fixture(params=["narrow", "wide"])
 def kernel(request):
-    """The tensor-core apply with 256-id units (the default for bf16 logits
-    with a base) or forced to 128-id units."""
-    set_debug(N.DSPARK_DEBUG_APPLY_NARROW if request.param == "narrow" else 0, 0)
+    """The tensor-core apply with 128-id units (the default) or, on request,
+    256-id units."""
+    set_debug(N.DSPARK_DEBUG_APPLY_WIDE if request.param == "wide" else 0, 0)
     yield request.param
     set_debug(0, 0)
 

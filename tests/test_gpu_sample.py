@@ -49,6 +49,15 @@ def _sample(d, algo, temperature, seed=0, base=None, first=None):
     return toks, corr, last_algo(), device_status()
 
 
+@pytest.fixture(params=["tile", "rows"])
+def layout(request):
+    """The tensor-core sampler in its tile layout (the default) or, on
+    request, its row layout."""
+    set_debug(N.DSPARK_DEBUG_SAMPLE_ROWS if request.param == "rows" else 0, 0)
+    yield request.param
+    set_debug(0, 0)
+
+
 def _rows_kernel_ran() -> bool:
     """The tensor-core sampler ran in its row layout (batch on the MMA's M
     side), not the tile layout (vocabulary ids on M)."""
@@ -71,27 +80,27 @@ def _small(batch, vocab=1000, rank=64, m=5, wstd=0.3, seed=21, spike=6.0):
 @pytest.mark.parametrize("algo", [TC, GEN], ids=["tc", "generic"])
 @pytest.mark.parametrize("batch,vocab,rank", [(1, 1000, 64), (5, 2056, 128), (33, 1000, 192), (70, 4096, 256),
                                               (128, 2056, 64), (150, 4096, 128), (256, 1000, 64)])
-def test_greedy_small(batch, vocab, rank, algo):
-    """Batches up to 128 take the row-layout kernel (32, 64 or 128 padded
-    rows); 150 and 256 the tile-layout one."""
+def test_greedy_small(batch, vocab, rank, algo, layout):
+    """The row layout takes batches up to 128 (32, 64 or 128 padded rows);
+    150 and 256 always take the tile layout."""
     wl = _small(batch, vocab, rank)
     d = W.make_inputs(wl)
     toks, corr, used, st = _sample(d, algo, 0.0)
     assert used == (2 if algo == TC else 1) and st == 0
     if algo == TC:
-        assert _rows_kernel_ran() == (batch <= 128)
+        assert _rows_kernel_ran() == (layout == "rows" and batch <= 128)
     # invariant: each token is the first argmax of its own corrected row
     assert torch.equal(toks, corr.float().argmax(-1))
     _check(d, toks, corr, 0.0, 0)
 
 
 @pytest.mark.parametrize("batch", W.GREEDY_BATCHES)
-def test_greedy_full_size(batch):
+def test_greedy_full_size(batch, layout):
     """M = 5, V = 129280, rank 128, peaked logits, every (b, k)."""
     wl = W.greedy(batch)
     d = W.make_inputs(wl)
     toks, corr, used, st = _sample(d, AUTO, 0.0)
-    assert used == 2 and st == 0 and _rows_kernel_ran()
+    assert used == 2 and st == 0 and _rows_kernel_ran() == (layout == "rows")
     assert torch.equal(toks, corr.float().argmax(-1))
     _check(d, toks, corr, 0.0, 0)
 
@@ -104,7 +113,11 @@ def test_row_kernel_streams_w2_at_large_ranks(rank, temperature):
     step. Weights that move tokens; every (b, k) against the oracle."""
     wl = W.greedy(24).with_(rank=rank, weight_std=0.3, spike=0.0, proposal_len=3, data_seed=30 + rank)
     d = W.make_inputs(wl)
-    toks, corr, used, st = _sample(d, AUTO, temperature, seed=11)
+    set_debug(N.DSPARK_DEBUG_SAMPLE_ROWS, 0)
+    try:
+        toks, corr, used, st = _sample(d, AUTO, temperature, seed=11)
+    finally:
+        set_debug(0, 0)
     assert used == 2 and st == 0 and _rows_kernel_ran()
     _check(d, toks, corr, temperature, 11)
 
@@ -131,12 +144,12 @@ def test_greedy_strong_bias_changes_tokens():
     assert (toks.cpu() != unbiased).float().mean() > 0.2
 
 
-def test_temperature_full_size():
+def test_temperature_full_size(layout):
     """B = 32, M = 8, V = 151936, rank 64, T = 0.7, Philox seed 1234."""
     wl = W.TEMPERATURE
     d = W.make_inputs(wl)
     toks, corr, used, st = _sample(d, AUTO, wl.temperature, seed=wl.philox_seed)
-    assert used == 2 and st == 0 and _rows_kernel_ran()
+    assert used == 2 and st == 0 and _rows_kernel_ran() == (layout == "rows")
     rep = _check(d, toks, corr, wl.temperature, wl.philox_seed)
     assert rep.exact_required > 0.9 * wl.batch * wl.proposal_len
 
@@ -371,7 +384,7 @@ def test_gumbel_noise_every_word_within_bound():
 
 @pytest.mark.parametrize("temperature", [0.0, 0.9])
 @pytest.mark.parametrize("batch", [1, 3, 4])
-def test_small_batches_full_vocabulary(batch, temperature):
+def test_small_batches_full_vocabulary(batch, temperature, layout):
     """Batches of one to four on the tensor-core sampler at full vocabulary,
     rank 128 (so a CTA keeps W2 tiles in both shared and tensor memory),
     with weights that move tokens: every (b, k) against the oracle."""
