@@ -274,7 +274,7 @@ int32_t dspark_markov_last_algo(void);
 #define DSPARK_VARIANT_BWD_RESIDENT_W1 1
 /*
  *   DSPARK_VARIANT_SAMPLE_ROWS: the tensor-core sampler ran with the batch on
- *     the MMA's M side and 256 vocabulary ids per MMA (batch <= 128; chosen by
+ *     the MMA's M side and 256 vocabulary ids per MMA (batch <= 64; chosen by
  *     DSPARK_DEBUG_SAMPLE_ROWS, or where the tile layout does not fit);
  *     otherwise it ran with vocabulary ids on M and the batch on N.
  */

@@ -107,7 +107,7 @@ bool tc_sample_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_
 // when the row-layout kernel runs.
 cudaError_t launch_tc_sample(const TcSampleArgs& a, int num_sms, cudaStream_t s, bool prefer_rows, int* variant);
 // The row-layout sampler (sample_rows_tc.cu): batch on the MMA's M side,
-// batch <= 128.
+// batch <= 64.
 bool tc_sample_rows_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype,
                               int num_sms);
 cudaError_t launch_tc_sample_rows(const TcSampleArgs& a, int num_sms, cudaStream_t s);

@@ -7,36 +7,43 @@
 //              or argmax_v c_k[b, v] / T + g(b, k, v)   (Gumbel-max, Philox noise)
 //
 // with x_{-1} = first_prev, in one cooperative persistent launch for all M
-// steps. CTA c owns a contiguous range of vocabulary ids (a multiple of 16),
-// cut into chunks of up to 256 ids.
+// steps. CTA c owns a contiguous range of vocabulary ids (whole 64-id spans,
+// so that no TMA box of logits crosses into a neighbour's range), cut into
+// chunks of up to 256 ids.
 //
 // Why this layout. A tcgen05.mma costs the same time whatever its N (16 to
 // 256) on this part, so the ids go on N, 256 at a time, and the batch on M:
 // D[lane][id] = X[lane] . W2[id]^T with A = X = W1[x_{k-1}] rows in shared
-// memory and B = a W2 chunk. M is 128, so the batch (padded to BP = 32, 64 or
-// 128 rows) is repeated REP = 128 / BP times down the lanes; each repeat
-// serves a different part of the chunk's columns, so that all four TMEM lane
-// quarters (one per epilogue warp quarter) carry useful rows. An epilogue
-// thread owns one batch row and runs along contiguous ids: 16-byte loads of
-// U and stores of the corrected logits straight to global memory, a
-// thread-local running maximum, and one Philox call per four ids.
+// memory and B = a W2 chunk. M is 128, so the batch (padded to BP = 32 or 64
+// rows) is repeated REP = 128 / BP times down the lanes; each repeat serves a
+// different part of the chunk's columns, so that all four TMEM lane quarters
+// (one per epilogue warp quarter) carry useful rows.
+//
+// Why every logit moves by TMA. A tcgen05.wait::ld also waits for the
+// thread's global loads still in flight (a few dozen cycles alone, over a
+// thousand behind outstanding loads), so the epilogue threads issue no global
+// loads or stores at all: a loader warp brings each chunk's U into shared
+// memory (boxes of 64 ids x B rows, 128-byte swizzle) through a ring of
+// stages, the epilogue adds the bias and rounds in place, and the same warp
+// stores the stage back to the corrected-logit tensor. U does not depend on
+// the chain, so the loads run ahead of the MMAs (and L2 prefetches one step
+// ahead of them).
 //
 // W2 stays on chip: the CTA's chunks are loaded into shared memory once; when
-// they do not all fit (rank 128 and above), the rest stream from L2 through a
-// two-slot ring every step, ordered so that their loads hide behind the
-// resident chunks' MMAs and the grid barrier. U is prefetched into L2 one step
-// ahead with bulk prefetches (it does not depend on the chain).
+// they do not all fit, the rest stream from L2 through a two-slot ring every
+// step, ordered so that their loads hide behind the resident chunks' MMAs and
+// the grid barrier.
 //
-// Per step: the gather warp waits at the grid barrier (bounded), decodes
-// x_{k-1} from the global keys and gathers X by TMA tile::gather4; the MMA
-// warp runs the chunks into two alternating 256-column accumulators; the
-// epilogue rounds, stores and selects; the CTA's per-row maxima go to the
-// global keys with one red.max each, and one release-add arrives at the
-// barrier.
+// Per step: warp 3 waits at the grid barrier (bounded), decodes x_{k-1} from
+// the global keys and gathers X with TMA row gathers; the MMA warp runs the
+// chunks into two alternating 256-column accumulators; the epilogue rounds
+// and selects; the CTA's per-row maxima go to the global keys with one
+// red.max each, and one release-add arrives at the barrier.
 //
 // Warp roles (640 threads): 0 W2 loader and ring producer; 1 TMEM owner and
-// MMA issuer; 3 grid barrier, key decode, X gather and U prefetch; 4-19
-// epilogue (warp 4 + 4e + q reads TMEM lane quarter q); 2 has no role.
+// MMA issuer; 2 U loader and corrected-logit storer; 3 grid barrier, key
+// decode, X gather and U prefetch; 4-19 epilogue (warp 4 + 4e + q reads TMEM
+// lane quarter q).
 #include <type_traits>
 
 #include "common.cuh"
@@ -47,7 +54,11 @@ namespace dspark {
 namespace {
 
 constexpr int kChunk = 256;                      // ids per chunk (MMA N at most)
+constexpr int kSpan = 64;                        // ids per logit box; CTA ranges are whole spans
+constexpr int kBoxesPerChunk = kChunk / kSpan;
 constexpr int kGroup = 16;                       // ids per epilogue piece (one tcgen05.ld x16)
+constexpr int kMaxStages = 3;                    // logit stages in shared memory
+constexpr int kMaxRowsBatch = 64;                // batch rows the stages hold
 constexpr int kEpiWarps = 16;
 constexpr int kEpiPerQuarter = kEpiWarps / 4;    // E
 constexpr int kThreads = 128 + kEpiWarps * 32;
@@ -61,23 +72,25 @@ struct __align__(64) RowsMaps {
   CUtensorMap w2;     // [vocab, rank] bf16, box 64 x 256, 128B swizzle
   CUtensorMap w2_16;  // same tensor, box 64 x 16 (the last, partial chunk)
   CUtensorMap w1;     // [vocab, rank] bf16, box 64 x 1 (row gathers), 128B swizzle
+  CUtensorMap u;      // base logits [B, M, V] as (v, k, b), box 64 x 1 x B, 128B swizzle
+  CUtensorMap out;    // corrected logits, the same layout
 };
 
 struct RowsParams {
-  const __nv_bfloat16* base;  // [B, M, V]
-  __nv_bfloat16* out;         // [B, M, V]
+  const __nv_bfloat16* base;  // [B, M, V] (L2 prefetch)
   const int64_t* first_prev;
-  const __nv_bfloat16* w1;
+  const __nv_bfloat16* w1;    // [V, r] (L2 prefetch of the next rows)
   int64_t* tokens;
   unsigned long long* keys;
   uint32_t* barrier;
   uint32_t* status;
   int64_t vocab;
   int32_t batch, bp, steps, ka;
-  int32_t groups;        // 16-id groups of the vocabulary
+  int32_t spans;         // 64-id spans of the vocabulary
   int32_t resident_full; // full chunks a CTA keeps in shared memory (the rest stream)
   uint32_t w2_bytes;     // shared memory reserved for resident W2 blocks
   int32_t ring;          // 1 when the streaming ring exists
+  int32_t stages;        // logit stages (2 or 3)
   float temperature;
   PhiloxRoundKeys round_keys;
   uint64_t wait_limit_ns;
@@ -87,7 +100,8 @@ struct RowsParams {
 struct RowsTail {
   uint64_t w2_full;
   uint64_t ring_full[2], ring_empty[2];
-  uint64_t x_full, x_empty;
+  uint64_t x_full;
+  uint64_t u_full[kMaxStages], tile_ready[kMaxStages];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t drain;
   int32_t xid[128];
@@ -104,16 +118,20 @@ struct Range {
     const int64_t w = ((v1 - v0 + 15) & ~15ll) - (int64_t)kChunk * j;
     return w < kChunk ? (int)w : kChunk;  // MMA N: a multiple of 16
   }
+  __device__ int boxes(int j) const { return (width(j) + kSpan - 1) / kSpan; }
 };
 
+// CTA c owns spans [S c / G, S (c + 1) / G); only the last range can end
+// inside a span (at the vocabulary's end), where the boxes' extra ids fall
+// outside the tensor: zeros on load, dropped on store.
 __device__ __forceinline__ Range cta_range(const RowsParams& p) {
   Range r;
-  const int64_t g0 = (int64_t)p.groups * blockIdx.x / gridDim.x;
-  const int64_t g1 = (int64_t)p.groups * (blockIdx.x + 1) / gridDim.x;
-  r.v0 = g0 * kGroup;
-  r.v1 = g1 * kGroup < p.vocab ? g1 * kGroup : p.vocab;
-  // Chunks are counted on the length rounded up to 16 ids, as the plan does
-  // (the last range can end 8 ids short of a group; those rows read as zero).
+  const int64_t s0 = (int64_t)p.spans * blockIdx.x / gridDim.x;
+  const int64_t s1 = (int64_t)p.spans * (blockIdx.x + 1) / gridDim.x;
+  r.v0 = s0 * kSpan;
+  r.v1 = s1 * kSpan < p.vocab ? s1 * kSpan : p.vocab;
+  // Chunks are counted on the length rounded up to 16 ids (the last range
+  // can end 8 ids short of a group; those W2 rows read as zero).
   const int64_t n16 = (r.v1 - r.v0 + 15) & ~15ll;
   r.nchunks = (int)((n16 + kChunk - 1) / kChunk);
   r.nfull = (int)(n16 / kChunk);
@@ -190,19 +208,6 @@ __device__ __forceinline__ unsigned long long ld_relaxed_gpu(const unsigned long
   return v;
 }
 
-__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-}
-
-__device__ __forceinline__ void st_stream_v4(void* p, uint4 v) {
-  asm volatile("st.global.cs.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-               : "memory");
-}
-
 // A warp-uniform bounded wait: lane 0 waits, the warp follows its verdict, and
 // the other lanes then observe the (already completed) phase themselves.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl, int lane) {
@@ -263,10 +268,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_sample_rows_kernel(const __grid_constant__ RowsMaps maps, const RowsParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* w2_smem = smem;                                     // resident W2 blocks
-  uint8_t* ring_smem = w2_smem + p.w2_bytes;                   // 2 x 32 KB when streaming
+  const uint32_t box_bytes = (uint32_t)p.bp * 128u;               // one box: BP rows of 64 ids
+  const uint32_t stage_bytes = kBoxesPerChunk * box_bytes;        // one chunk of logits
+  uint8_t* w2_smem = smem;                                        // resident W2 blocks
+  uint8_t* ring_smem = w2_smem + p.w2_bytes;                      // 2 x 32 KB when streaming
   uint8_t* x_smem = ring_smem + (p.ring ? 2 * kFullBlockBytes : 0u);  // KA atoms of 16 KB
-  unsigned long long* red = reinterpret_cast<unsigned long long*>(x_smem + KA * kXAtomBytes);  // [128]
+  uint8_t* u_smem = x_smem + KA * kXAtomBytes;                    // p.stages logit stages
+  unsigned long long* red = reinterpret_cast<unsigned long long*>(u_smem + (uint32_t)p.stages * stage_bytes);
   RowsTail* sh = reinterpret_cast<RowsTail*>(red + 128);
 
   const int warp = threadIdx.x >> 5;
@@ -275,6 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int M = p.steps;
   const int B = p.batch;
   const int BP = p.bp;
+  const int NS = p.stages;
   const Range rg = cta_range(p);
   const int res = resident_full_of(rg, p);
   const int nc = rg.nchunks;
@@ -288,8 +297,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sh->acc_full[i], 1);
       mbar_init(&sh->acc_empty[i], kEpiWarps);
     }
-    mbar_init(&sh->x_full, 1);
-    mbar_init(&sh->x_empty, 1);
+    for (int i = 0; i < kMaxStages; ++i) {
+      mbar_init(&sh->u_full[i], 1);                // the chunk's logits have landed
+      mbar_init(&sh->tile_ready[i], kEpiWarps);    // the epilogue has rewritten the stage
+    }
+    mbar_init(&sh->x_full, 1);                     // the step's X rows have landed
     mbar_init(&sh->drain, 1);
     sh->abort_flag = 0;
     fence_barrier_init();
@@ -360,10 +372,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       int64_t t = 0, gs = 0;
       for (int k = 0; k < M && ok; ++k) {
         if (!mbar_wait(&sh->x_full, (uint32_t)k & 1u, ctl)) break;
+        tc_fence_after_sync();
         for (int i = 0; i < nc && ok; ++i, ++t) {
           const int j = chunk_at(i, rg, res);
           const int buf = (int)(t & 1);
-          if (!mbar_wait(&sh->acc_empty[buf], ((uint32_t)(t >> 1) & 1u) ^ 1u, ctl)) {
+          // The previous chunk's accumulator has been read into registers (and
+          // so, in order, every earlier one): the epilogue's tensor-memory
+          // loads never wait behind MMAs in flight.
+          if (t > 0 && !mbar_wait(&sh->acc_empty[(t - 1) & 1], (uint32_t)((t - 1) >> 1) & 1u, ctl)) {
             ok = false;
             break;
           }
@@ -397,31 +413,77 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (ok) umma_commit(&sh->acc_full[buf]);
         }
-        if (ok) umma_commit(&sh->x_empty);
       }
       umma_commit(&sh->drain);
       mbar_wait(&sh->drain, 0, drain_ctl);
     }
+  } else if (warp == 2) {
+    // ----------------------- logits in and out through the stages ----
+    // Chunk t (step t / nc, position t % nc) uses stage t % NS. Its boxes
+    // load once the stage's previous chunk has been stored (the store has
+    // read the stage), so the loads run up to NS chunks ahead of the
+    // epilogue, across step boundaries.
+    if (lane == 0) {
+      prefetch_tensormap(&maps.u);
+      prefetch_tensormap(&maps.out);
+      const uint64_t pol = policy_evict_first();
+      const int64_t T = (int64_t)M * nc;
+      const uint32_t box_tx = (uint32_t)B * 128u;
+      auto chunk_x = [&](int64_t t, int& k, int& nb) {
+        k = (int)(t / nc);
+        const int j = chunk_at((int)(t % nc), rg, res);
+        nb = rg.boxes(j);
+        return (int32_t)(rg.v0 + (int64_t)kChunk * j);
+      };
+      auto load = [&](int64_t t) {
+        int k, nb;
+        const int32_t x = chunk_x(t, k, nb);
+        const int s = (int)(t % NS);
+        mbar_arrive_expect_tx(&sh->u_full[s], (uint32_t)nb * box_tx);
+        for (int bx = 0; bx < nb; ++bx)
+          tma_load_3d(u_smem + (uint32_t)s * stage_bytes + (uint32_t)bx * box_bytes, &maps.u, &sh->u_full[s],
+                      x + bx * kSpan, k, 0, pol);
+      };
+      int64_t issued = 0;
+      for (; issued < T && issued < NS; ++issued) load(issued);
+      for (int64_t t = 0; t < T; ++t) {
+        const int s = (int)(t % NS);
+        if (!mbar_wait(&sh->tile_ready[s], (uint32_t)(t / NS) & 1u, ctl)) break;
+        int k, nb;
+        const int32_t x = chunk_x(t, k, nb);
+        for (int bx = 0; bx < nb; ++bx)
+          tma_store_3d(&maps.out, u_smem + (uint32_t)s * stage_bytes + (uint32_t)bx * box_bytes, x + bx * kSpan, k,
+                       0);
+        bulk_commit_group();
+        if (issued < T) {
+          bulk_wait_group_read<0>();  // the stage may be refilled once the store has read it
+          load(issued);
+          ++issued;
+        }
+      }
+      bulk_wait_group<0>();
+      // On an abort, the loads still in flight land before the CTA exits.
+      for (int64_t t = (issued > NS ? issued - NS : 0); t < issued; ++t)
+        mbar_wait(&sh->u_full[t % NS], (uint32_t)(t / NS) & 1u, drain_ctl);
+    }
   } else if (warp == 3) {
-    // ------------------------- grid barrier, X gather, U prefetch ----
-    const uint64_t pol_w1 = policy_evict_last();
-    if (lane == 0) prefetch_tensormap(&maps.w1);
+    // ------------- grid barrier, previous tokens, X gather, U prefetch ----
     // U of step k is prefetched into L2 (bulk prefetch of each row's range)
     // one step ahead: it does not depend on the chain.
+    if (lane == 0) prefetch_tensormap(&maps.w1);
+    const uint64_t pol_w1 = policy_evict_last();
     const uint32_t row_bytes = (uint32_t)((rg.v1 - rg.v0) * 2);
     auto prefetch_u = [&](int k) {
       for (int b = lane; b < B && row_bytes; b += 32)
         bulk_prefetch_l2(p.base + ((int64_t)b * M + k) * p.vocab + rg.v0, row_bytes);
     };
     prefetch_u(0);
-    int armed = -1;  // the last step whose gather was issued
     for (int k = 0; k < M; ++k) {
-      if (!warp_wait(&sh->x_empty, ((uint32_t)k & 1u) ^ 1u, ctl, lane)) break;
       // Every CTA has merged its step k-1 maxima once the counter reaches k * G.
       if (k > 0 && !grid_wait(p.barrier, (uint32_t)k * (uint32_t)G, ctl, lane)) break;
       bool bad = false;
       for (int b = lane; b < BP; b += 32) {
-        int32_t row = (int32_t)p.vocab;  // outside the tensor: the gather reads zeros
+        int32_t row = (int32_t)p.vocab;  // outside W1: the gather reads zeros
         if (b < B) {
           const int64_t id =
               k == 0 ? p.first_prev[b] : (int64_t)key_token(ld_relaxed_gpu(&p.keys[(size_t)(k - 1) * B + b]));
@@ -435,16 +497,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (bad) report_status(p.status, DSPARK_STATUS_TOKEN_RANGE);
       __syncwarp();
+      // X row L is W1[x_{k-1}[L % BP]]: lane l gathers rows 4l .. 4l + 3 of
+      // every 64-column atom into the 128-byte-swizzle K-major layout. The
+      // previous step's MMAs are complete (this CTA's epilogue read their
+      // accumulators before it arrived at the barrier just passed).
       if (lane == 0) mbar_arrive_expect_tx(&sh->x_full, (uint32_t)KA * kXAtomBytes);
-      armed = k;
       __syncwarp();
-      // Lane L of the operand holds batch row L % BP; lane i gathers lanes 4i..4i+3.
-#pragma unroll
-      for (int a = 0; a < KA; ++a) {
+      {
         const int l0 = 4 * lane;
-        tma_gather4(x_smem + (uint32_t)a * kXAtomBytes + (uint32_t)l0 * 128u, &maps.w1, &sh->x_full, a * 64,
-                    sh->xid[l0 % BP], sh->xid[(l0 + 1) % BP], sh->xid[(l0 + 2) % BP], sh->xid[(l0 + 3) % BP],
-                    pol_w1);
+        const int32_t r0 = sh->xid[l0 % BP], r1 = sh->xid[(l0 + 1) % BP];
+        const int32_t r2 = sh->xid[(l0 + 2) % BP], r3 = sh->xid[(l0 + 3) % BP];
+#pragma unroll
+        for (int a = 0; a < KA; ++a)
+          tma_gather4(x_smem + (uint32_t)a * kXAtomBytes + (uint32_t)l0 * 128u, &maps.w1, &sh->x_full, a * 64, r0, r1,
+                      r2, r3, pol_w1);
       }
       __syncwarp();
       if (k + 1 < M) prefetch_u(k + 1);
@@ -455,9 +521,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             p.tokens[(size_t)b * M + (M - 1)] = (int64_t)key_token(ld_relaxed_gpu(&p.keys[(size_t)(M - 1) * B + b]));
       }
     }
-    // The last gather has landed before the CTA may exit (it has unless a
-    // wait gave up before the MMAs consumed it).
-    if (lane == 0 && armed >= 0) mbar_wait(&sh->x_full, (uint32_t)armed & 1u, drain_ctl);
   } else if (warp >= 4) {
     // -------------------------------------------------- epilogue ----
     const int ew = warp - 4;
@@ -473,63 +536,52 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int te = threadIdx.x - 128;
     const uint32_t all_n = kEpiWarps * 32;
     const float inv_t = GREEDY ? 0.0f : 1.0f / p.temperature;
-    // The pieces (step k, chunk position i, 16-id group g) this thread works
-    // on, in order; U of the next piece is loaded one piece ahead (across
-    // chunk and step boundaries), so its latency hides behind the current
-    // piece and the accumulator waits.
-    struct Cursor {
-      int k, i, g;
-    };
-    auto settle = [&](Cursor& c) {  // move to the first existing piece at or after c
-      while (c.k < M) {
-        if (c.g < rg.width(chunk_at(c.i, rg, res)) / kGroup) return;
-        c.g = slot;
-        if (++c.i == nc) {
-          c.i = 0;
-          ++c.k;
-        }
-      }
-    };
-    auto load_u = [&](const Cursor& c, uint4& a0, uint4& a1) {
-      if (!row_ok || c.k >= M) return;
-      const int64_t v = rg.v0 + (int64_t)kChunk * chunk_at(c.i, rg, res) + (int64_t)kGroup * c.g;
-      const __nv_bfloat16* src = p.base + ((size_t)b * M + c.k) * (size_t)p.vocab + v;
-      a0 = ld_stream_v4(src);
-      if (v + kGroup <= p.vocab) a1 = ld_stream_v4(src + 8);
-    };
-    Cursor nxt{0, 0, slot};
-    settle(nxt);
-    uint4 nu0 = make_uint4(0u, 0u, 0u, 0u), nu1 = nu0;
-    load_u(nxt, nu0, nu1);
+    // Row b of a box sits at b * 128 bytes; its 16-byte piece c at (c ^ (b & 7)) * 16.
+    const uint32_t row_smem = (uint32_t)b * 128u;
+    const uint32_t swz = (uint32_t)(b & 7);
     int64_t t = 0;
     bool ok = true;
     for (int k = 0; k < M && ok; ++k) {
-      const size_t row_off = ((size_t)b * M + k) * (size_t)p.vocab;
       uint32_t best = 0u;      // greedy: (ordered bf16 bits, 0xFFFF - local id); temperature: ordered score
       uint32_t best_lid = 0u;  // temperature: the CTA-local id of `best`
       for (int i = 0; i < nc; ++i, ++t) {
         const int j = chunk_at(i, rg, res);
         const int buf = (int)(t & 1);
+        const int s = (int)(t % NS);
         const int ngroups = rg.width(j) / kGroup;
         const int64_t c0 = rg.v0 + (int64_t)kChunk * j;
-        if (!warp_wait(&sh->acc_full[buf], (uint32_t)(t >> 1) & 1u, ctl, lane)) {
+        uint8_t* stage = u_smem + (uint32_t)s * stage_bytes;
+        if (!warp_wait(&sh->u_full[s], (uint32_t)(t / NS) & 1u, ctl, lane) ||
+            !warp_wait(&sh->acc_full[buf], (uint32_t)(t >> 1) & 1u, ctl, lane)) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
+        // The accumulator goes back to the MMA warp right after this warp's
+        // last tensor-memory load of the chunk (at once if it has none).
+        if (slot >= ngroups) {
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh->acc_empty[buf]);
+        }
         for (int g = slot; g < ngroups; g += nslots) {
-          const int64_t v = c0 + (int64_t)kGroup * g;  // first id of the piece (== nxt)
+          const int64_t v = c0 + (int64_t)kGroup * g;  // first id of the piece
           const bool full = v + kGroup <= p.vocab;     // else only the first 8 ids exist
-          const uint4 u0 = nu0, u1 = nu1;
-          nxt.g += nslots;
-          settle(nxt);
-          nu1 = make_uint4(0u, 0u, 0u, 0u);
-          load_u(nxt, nu0, nu1);
           uint32_t d[16];
           __syncwarp();  // tcgen05.ld is warp-aligned
           tmem_ld_32x32b_x16(lane_base + (uint32_t)(buf * kChunk + kGroup * g), d);
           tmem_ld_wait();
+          if (g + nslots >= ngroups) {
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh->acc_empty[buf]);
+          }
           if (!row_ok) continue;
+          uint8_t* rowp = stage + (uint32_t)(g >> 2) * box_bytes + row_smem;
+          const uint32_t pc = (uint32_t)(g & 3) * 2u;
+          uint4* p0 = reinterpret_cast<uint4*>(rowp + ((pc ^ swz) << 4));
+          uint4* p1 = reinterpret_cast<uint4*>(rowp + (((pc + 1u) ^ swz) << 4));
+          const uint4 u0 = *p0, u1 = *p1;
           uint32_t c[8];
           c[0] = add_round2(u0.x, d[0], d[1]);
           c[1] = add_round2(u0.y, d[2], d[3]);
@@ -539,8 +591,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           c[5] = add_round2(u1.y, d[10], d[11]);
           c[6] = add_round2(u1.z, d[12], d[13]);
           c[7] = add_round2(u1.w, d[14], d[15]);
-          st_stream_v4(p.out + row_off + v, make_uint4(c[0], c[1], c[2], c[3]));
-          if (full) st_stream_v4(p.out + row_off + v + 8, make_uint4(c[4], c[5], c[6], c[7]));
+          *p0 = make_uint4(c[0], c[1], c[2], c[3]);
+          *p1 = make_uint4(c[4], c[5], c[6], c[7]);
           const int nid = full ? 16 : 8;
           const uint32_t lid0 = (uint32_t)(v - rg.v0);
           if constexpr (GREEDY) {
@@ -572,9 +624,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        tc_fence_before_sync();
+        // The stage goes to the storer: the rewritten logits are made visible
+        // to the async proxy first.
+        fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sh->acc_empty[buf]);
+        if (lane == 0) mbar_arrive(&sh->tile_ready[s]);
       }
       // The epilogue warps agree to go on (an abort anywhere ends every step).
       if (!barrier_and(ok, 1, all_n)) break;
@@ -618,29 +672,43 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 struct RowsPlan {
-  int bp, resident_full, ring;
+  int bp, resident_full, ring, stages;
   uint32_t w2_bytes;
   size_t smem;
   bool ok;
 };
 
-RowsPlan rows_plan(int64_t batch, int64_t vocab, int32_t rank, int grid) {
+// The shared-memory plan for `stages` logit stages: resident W2 chunks, the
+// streaming ring when they do not all fit, X, the stages and the tail.
+RowsPlan rows_plan_stages(int64_t batch, int64_t vocab, int32_t rank, int grid, int stages) {
   RowsPlan c{};
-  if (batch < 1 || batch > 128 || rank % 64 != 0 || rank < 64 || rank > 256 || vocab % 8 != 0 || grid < 1) return c;
-  c.bp = batch <= 32 ? 32 : batch <= 64 ? 64 : 128;
+  if (batch < 1 || batch > kMaxRowsBatch || rank % 64 != 0 || rank < 64 || rank > 256 || vocab % 8 != 0 ||
+      grid < 1 || stages < 2 || stages > kMaxStages)
+    return c;
+  c.bp = batch <= 32 ? 32 : 64;
+  c.stages = stages;
   const int ka = rank / 64;
-  const int64_t groups = (vocab + 15) / 16;
-  // CTA ranges hold floor or ceil(groups / grid) groups of 16 ids.
-  const int64_t nmin = 16 * (groups / grid), nmax = 16 * ((groups + grid - 1) / grid);
-  if (nmin < 16 || nmax > 65535 || (nmax + kChunk - 1) / kChunk > kMaxChunks) return c;
+  const int64_t spans = (vocab + kSpan - 1) / kSpan;
+  if (grid > spans) return c;
+  // Every CTA's range as the kernel cuts it: the most chunks, the most full
+  // chunks and the widest partial chunk over all of them.
+  int64_t nmax = 0;
+  int64_t part_w = 0;
+  for (int g = 0; g < grid; ++g) {
+    const int64_t v0 = spans * g / grid * kSpan;
+    const int64_t e = spans * (g + 1) / grid * kSpan;
+    const int64_t v1 = e < vocab ? e : vocab;
+    if (v1 <= v0) return c;
+    const int64_t n16 = (v1 - v0 + 15) & ~15ll;
+    nmax = n16 > nmax ? n16 : nmax;
+    part_w = n16 % kChunk > part_w ? n16 % kChunk : part_w;
+  }
+  if (nmax > 65535 || (nmax + kChunk - 1) / kChunk > kMaxChunks) return c;
   const int nfull = (int)(nmax / kChunk);
   const uint32_t full_bytes = (uint32_t)ka * kFullBlockBytes;
-  uint32_t part_bytes = 0;  // the larger partial chunk of the two range sizes
-  for (int64_t n : {nmin, nmax}) {
-    const uint32_t pb = (uint32_t)ka * (uint32_t)(n % kChunk) * 128u;
-    part_bytes = pb > part_bytes ? pb : part_bytes;
-  }
-  const size_t fixed = 1024 + (size_t)ka * kXAtomBytes + 128 * 8 + sizeof(RowsTail) + 64;
+  const uint32_t part_bytes = (uint32_t)ka * (uint32_t)part_w * 128u;
+  const size_t stage_bytes = (size_t)kBoxesPerChunk * c.bp * 128;
+  const size_t fixed = 1024 + (size_t)ka * kXAtomBytes + (size_t)stages * stage_bytes + 128 * 8 + sizeof(RowsTail) + 64;
   if (fixed >= kSmemLimit) return c;
   const size_t budget = kSmemLimit - fixed;
   const size_t ring_bytes = 2 * (size_t)kFullBlockBytes;
@@ -660,6 +728,14 @@ RowsPlan rows_plan(int64_t batch, int64_t vocab, int32_t rank, int grid) {
   return c;
 }
 
+// Three stages where they cost no resident W2 chunk, else two.
+RowsPlan rows_plan(int64_t batch, int64_t vocab, int32_t rank, int grid) {
+  const RowsPlan two = rows_plan_stages(batch, vocab, rank, grid, 2);
+  const RowsPlan three = rows_plan_stages(batch, vocab, rank, grid, 3);
+  if (three.ok && (!two.ok || (three.resident_full >= two.resident_full && three.ring <= two.ring))) return three;
+  return two;
+}
+
 template <int KA, bool GREEDY>
 cudaError_t launch_rows_ka(const TcSampleArgs& a, const RowsPlan& c, int grid, cudaStream_t stream) {
   RowsMaps maps;
@@ -667,17 +743,23 @@ cudaError_t launch_rows_ka(const TcSampleArgs& a, const RowsPlan& c, int grid, c
   const uint64_t wstr[1] = {(uint64_t)a.rank * 2};
   const uint32_t box[2] = {64, (uint32_t)kChunk};
   const uint32_t box16[2] = {64, 16};
-  const uint32_t rbox[2] = {64, 1};
+  const uint32_t box1[2] = {64, 1};
+  const uint64_t udim[3] = {(uint64_t)a.vocab, (uint64_t)a.steps, (uint64_t)a.batch};
+  const uint64_t ustr[2] = {(uint64_t)a.vocab * 2, (uint64_t)a.vocab * 2 * (uint64_t)a.steps};
+  const uint32_t ubox[3] = {(uint32_t)kSpan, 1u, (uint32_t)a.batch};
   if (!encode_tensor_map(&maps.w2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.w2, wdim, wstr, box,
                          CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tensor_map(&maps.w2_16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.w2, wdim, wstr, box16,
                          CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tensor_map(&maps.w1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.w1, wdim, wstr, rbox,
+      !encode_tensor_map(&maps.w1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.w1, wdim, wstr, box1,
+                         CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tensor_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.base, udim, ustr, ubox,
+                         CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tensor_map(&maps.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.corrected, udim, ustr, ubox,
                          CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   RowsParams p{};
   p.base = static_cast<const __nv_bfloat16*>(a.base);
-  p.out = static_cast<__nv_bfloat16*>(a.corrected);
   p.first_prev = a.first_prev;
   p.w1 = static_cast<const __nv_bfloat16*>(a.w1);
   p.tokens = a.tokens;
@@ -689,10 +771,11 @@ cudaError_t launch_rows_ka(const TcSampleArgs& a, const RowsPlan& c, int grid, c
   p.bp = c.bp;
   p.steps = (int32_t)a.steps;
   p.ka = KA;
-  p.groups = (int32_t)((a.vocab + 15) / 16);
+  p.spans = (int32_t)((a.vocab + kSpan - 1) / kSpan);
   p.resident_full = c.resident_full;
   p.w2_bytes = c.w2_bytes;
   p.ring = c.ring;
+  p.stages = c.stages;
   p.temperature = a.temperature;
   p.round_keys = round_keys_for(a.seed);
   p.wait_limit_ns = a.wait_limit_ns;
@@ -728,8 +811,8 @@ cudaError_t launch_rows_mode(const TcSampleArgs& a, const RowsPlan& c, int grid,
 }
 
 int rows_grid(int64_t vocab, int num_sms) {
-  const int64_t groups = (vocab + 15) / 16;
-  return (int)(groups < num_sms ? groups : num_sms);
+  const int64_t spans = (vocab + kSpan - 1) / kSpan;
+  return (int)(spans < num_sms ? spans : num_sms);
 }
 
 }  // namespace

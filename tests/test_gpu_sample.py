@@ -81,14 +81,14 @@ def _small(batch, vocab=1000, rank=64, m=5, wstd=0.3, seed=21, spike=6.0):
 @pytest.mark.parametrize("batch,vocab,rank", [(1, 1000, 64), (5, 2056, 128), (33, 1000, 192), (70, 4096, 256),
                                               (128, 2056, 64), (150, 4096, 128), (256, 1000, 64)])
 def test_greedy_small(batch, vocab, rank, algo, layout):
-    """The row layout takes batches up to 128 (32, 64 or 128 padded rows);
-    150 and 256 always take the tile layout."""
+    """The row layout takes batches up to 64 (32 or 64 padded rows); 70,
+    128, 150 and 256 always take the tile layout."""
     wl = _small(batch, vocab, rank)
     d = W.make_inputs(wl)
     toks, corr, used, st = _sample(d, algo, 0.0)
     assert used == (2 if algo == TC else 1) and st == 0
     if algo == TC:
-        assert _rows_kernel_ran() == (layout == "rows" and batch <= 128)
+        assert _rows_kernel_ran() == (layout == "rows" and batch <= 64)
     # invariant: each token is the first argmax of its own corrected row
     assert torch.equal(toks, corr.float().argmax(-1))
     _check(d, toks, corr, 0.0, 0)
@@ -123,7 +123,7 @@ def test_row_kernel_streams_w2_at_large_ranks(rank, temperature):
 
 
 def test_tile_kernel_full_vocabulary():
-    """Batch 140 (above the row layout's 128) at full vocabulary and rank 64:
+    """Batch 140 (above the row layout's 64) at full vocabulary and rank 64:
     the tile-layout kernel, every (b, k) against the oracle."""
     wl = W.greedy(140).with_(rank=64, weight_std=0.3, spike=0.0, proposal_len=2, data_seed=41)
     d = W.make_inputs(wl)
