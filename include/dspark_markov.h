@@ -254,11 +254,14 @@ int64_t dspark_markov_launch_count(void);
 /* flags bit 1: the tensor-core apply uses 256-id units where they apply
  * (bf16 logits with a base, out != base_logits) instead of 128-id units.
  * flags bit 2: the tensor-core sampler uses the row layout (batch on the MMA's
- * M side) where it applies instead of the tile layout. Without these bits
- * each call takes the variant that measured fastest on these shapes; both
- * stay testable. */
+ * M side) where it applies. flags bit 3: the tensor-core sampler uses the
+ * tile layout (vocabulary ids on M) where it applies; bit 2 wins when both are
+ * set. Without these bits each call takes the variant that measured fastest
+ * on these shapes (row layout for temperature sampling, tile layout for
+ * greedy decoding); every variant stays testable. */
 #define DSPARK_DEBUG_APPLY_WIDE 2u
 #define DSPARK_DEBUG_SAMPLE_ROWS 4u
+#define DSPARK_DEBUG_SAMPLE_TILE 8u
 int dspark_markov_set_debug(uint32_t flags, uint64_t wait_limit_ns);
 
 /* Which kernel the last call on this thread selected: 0 none, 1 generic, 2 tensor core. */
@@ -274,8 +277,9 @@ int32_t dspark_markov_last_algo(void);
 #define DSPARK_VARIANT_BWD_RESIDENT_W1 1
 /*
  *   DSPARK_VARIANT_SAMPLE_ROWS: the tensor-core sampler ran with the batch on
- *     the MMA's M side and 256 vocabulary ids per MMA (batch <= 64; chosen by
- *     DSPARK_DEBUG_SAMPLE_ROWS, or where the tile layout does not fit);
+ *     the MMA's M side and 256 vocabulary ids per MMA (batch <= 64; chosen for
+ *     temperature > 0, by DSPARK_DEBUG_SAMPLE_ROWS, or where the tile layout
+ *     does not fit; not under DSPARK_DEBUG_SAMPLE_TILE where the tile fits);
  *     otherwise it ran with vocabulary ids on M and the batch on N.
  */
 #define DSPARK_VARIANT_SAMPLE_ROWS 2

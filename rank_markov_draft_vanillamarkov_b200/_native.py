@@ -30,6 +30,7 @@ DSPARK_ALGO_TENSOR_CORE = 2
 DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL = 1
 DSPARK_DEBUG_APPLY_WIDE = 2
 DSPARK_DEBUG_SAMPLE_ROWS = 4
+DSPARK_DEBUG_SAMPLE_TILE = 8
 
 DSPARK_NOALLOC_MAX_KEYS = 8192
 

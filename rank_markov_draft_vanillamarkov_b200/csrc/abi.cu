@@ -91,6 +91,14 @@ unsigned char* workspace(DeviceState* d, size_t bytes) {
   return d->workspace;
 }
 
+// The sampler layout the debug flags force, if any (rows wins over tile).
+int sample_layout() {
+  const uint32_t f = g_debug_flags.load();
+  if (f & DSPARK_DEBUG_SAMPLE_ROWS) return kSampleRows;
+  if (f & DSPARK_DEBUG_SAMPLE_TILE) return kSampleTile;
+  return kSampleAuto;
+}
+
 // ---------------------------------------------------------------------------
 // Fixed scratch of dspark_markov_sample_block_noalloc, for callers that cannot
 // allocate device memory during the call. It lives in this module's static
@@ -367,8 +375,7 @@ int dspark_markov_sample_block(const void* base_logits, const int64_t* first_pre
     a.debug_flags = g_debug_flags.load();
     t_last_algo = 2;
     int variant = 0;
-    const bool rows = (g_debug_flags.load() & DSPARK_DEBUG_SAMPLE_ROWS) != 0;
-    const cudaError_t e = launch_tc_sample(a, d->num_sms, s, rows, &variant);
+    const cudaError_t e = launch_tc_sample(a, d->num_sms, s, sample_layout(), &variant);
     t_last_variant = variant;
     return cuda_code(e);
   }
@@ -465,8 +472,7 @@ int dspark_markov_sample_block_noalloc(const void* base_logits, const int64_t* f
   a.debug_flags = g_debug_flags.load();
   t_last_algo = 2;
   int variant = 0;
-  const bool rows = (g_debug_flags.load() & DSPARK_DEBUG_SAMPLE_ROWS) != 0;
-  const cudaError_t e = launch_tc_sample(a, st->num_sms, s, rows, &variant);
+  const cudaError_t e = launch_tc_sample(a, st->num_sms, s, sample_layout(), &variant);
   t_last_variant = variant;
   return cuda_code(e);
 }

@@ -102,10 +102,13 @@ struct TcSampleArgs {
 };
 bool tc_sample_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype,
                          int num_sms);
-// The tile-layout kernel, or the row-layout one when `prefer_rows` is set or
-// the tile layout does not fit; sets DSPARK_VARIANT_SAMPLE_ROWS in *variant
-// when the row-layout kernel runs.
-cudaError_t launch_tc_sample(const TcSampleArgs& a, int num_sms, cudaStream_t s, bool prefer_rows, int* variant);
+// Sampler layout request: the measured-faster layout for the mode (row layout
+// for temperature sampling, tile layout for greedy decoding), or one forced.
+enum SampleLayout { kSampleAuto = 0, kSampleRows = 1, kSampleTile = 2 };
+// The tile-layout or the row-layout kernel as `layout` asks, each only where
+// it fits (else the other); sets DSPARK_VARIANT_SAMPLE_ROWS in *variant when
+// the row-layout kernel runs.
+cudaError_t launch_tc_sample(const TcSampleArgs& a, int num_sms, cudaStream_t s, int layout, int* variant);
 // The row-layout sampler (sample_rows_tc.cu): batch on the MMA's M side,
 // batch <= 64.
 bool tc_sample_rows_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_dtype, int weight_dtype,

@@ -19,31 +19,39 @@
 // different part of the chunk's columns, so that all four TMEM lane quarters
 // (one per epilogue warp quarter) carry useful rows.
 //
-// Why every logit moves by TMA. A tcgen05.wait::ld also waits for the
-// thread's global loads still in flight (a few dozen cycles alone, over a
-// thousand behind outstanding loads), so the epilogue threads issue no global
-// loads or stores at all: a loader warp brings each chunk's U into shared
-// memory (boxes of 64 ids x B rows, 128-byte swizzle) through a ring of
-// stages, the epilogue adds the bias and rounds in place, and the same warp
-// stores the stage back to the corrected-logit tensor. U does not depend on
-// the chain, so the loads run ahead of the MMAs (and L2 prefetches one step
-// ahead of them).
+// Why the epilogue warps keep off global memory. A tcgen05.wait::ld, and a
+// proxy fence, also wait for the thread's global accesses still in flight:
+// a few dozen cycles alone, a thousand and more behind outstanding loads or
+// behind reductions that 148 CTAs aim at the same keys. So the epilogue
+// threads issue no global stores or reductions and no loads that are still
+// in flight at a tensor-memory load: a loader warp brings each chunk's U into
+// shared memory (boxes of 64 ids x B rows, 128-byte swizzle) through a ring
+// of stages, the epilogue adds the bias and rounds in place, and the same
+// warp stores the stage back to the corrected-logit tensor; the per-row
+// maxima leave through shared memory and warp 3 merges them into the global
+// keys. U does not depend on the chain, so its loads run ahead of the MMAs
+// (and L2 prefetches one step ahead of them). The one global read the
+// epilogue makes is X's rows at the start of a step, and those loads have
+// landed (their values are stored to shared memory) before any tensor-memory
+// load.
 //
 // W2 stays on chip: the CTA's chunks are loaded into shared memory once; when
 // they do not all fit, the rest stream from L2 through a two-slot ring every
 // step, ordered so that their loads hide behind the resident chunks' MMAs and
 // the grid barrier.
 //
-// Per step: warp 3 waits at the grid barrier (bounded), decodes x_{k-1} from
-// the global keys and gathers X with TMA row gathers; the MMA warp runs the
-// chunks into two alternating 256-column accumulators; the epilogue rounds
-// and selects; the CTA's per-row maxima go to the global keys with one
-// red.max each, and one release-add arrives at the barrier.
+// Per step: warp 3 waits at the grid barrier (bounded) and decodes x_{k-1}
+// from the global keys; the epilogue warps gather X (each loads its rows'
+// share of W1[x_{k-1}] and stores it in the swizzled operand layout); the MMA
+// warp runs the chunks into two alternating 256-column accumulators, one
+// chunk ahead of the epilogue; the epilogue rounds and selects and leaves its
+// per-row maxima in shared memory; warp 3 merges them into the global keys
+// (one red.max per row) and arrives at the barrier with one release-add.
 //
 // Warp roles (640 threads): 0 W2 loader and ring producer; 1 TMEM owner and
-// MMA issuer; 2 U loader and corrected-logit storer; 3 grid barrier, key
-// decode, X gather and U prefetch; 4-19 epilogue (warp 4 + 4e + q reads TMEM
-// lane quarter q).
+// MMA issuer; 2 U loader and corrected-logit storer; 3 key merge, grid
+// barrier, key decode and U prefetch; 4-19 X gather and epilogue (warp
+// 4 + 4e + q reads TMEM lane quarter q).
 #include <type_traits>
 
 #include "common.cuh"
@@ -71,7 +79,6 @@ constexpr size_t kSmemLimit = 232448;
 struct __align__(64) RowsMaps {
   CUtensorMap w2;     // [vocab, rank] bf16, box 64 x 256, 128B swizzle
   CUtensorMap w2_16;  // same tensor, box 64 x 16 (the last, partial chunk)
-  CUtensorMap w1;     // [vocab, rank] bf16, box 64 x 1 (row gathers), 128B swizzle
   CUtensorMap u;      // base logits [B, M, V] as (v, k, b), box 64 x 1 x B, 128B swizzle
   CUtensorMap out;    // corrected logits, the same layout
 };
@@ -79,9 +86,9 @@ struct __align__(64) RowsMaps {
 struct RowsParams {
   const __nv_bfloat16* base;  // [B, M, V] (L2 prefetch)
   const int64_t* first_prev;
-  const __nv_bfloat16* w1;    // [V, r] (L2 prefetch of the next rows)
+  const __nv_bfloat16* w1;    // [V, r]
   int64_t* tokens;
-  unsigned long long* keys;
+  unsigned long long* keys;   // [M, B] step maxima
   uint32_t* barrier;
   uint32_t* status;
   int64_t vocab;
@@ -100,7 +107,7 @@ struct RowsParams {
 struct RowsTail {
   uint64_t w2_full;
   uint64_t ring_full[2], ring_empty[2];
-  uint64_t x_full;
+  uint64_t xid_ready, x_full, merge_ready;
   uint64_t u_full[kMaxStages], tile_ready[kMaxStages];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t drain;
@@ -170,16 +177,6 @@ __device__ __forceinline__ uint32_t resident_offset(int j, int a, const Range& r
   return (uint32_t)res * ka * kFullBlockBytes + (uint32_t)a * pw * 128u;
 }
 
-__device__ __forceinline__ bool barrier_and(bool v, uint32_t id, uint32_t n) {
-  uint32_t out;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(out)
-      : "r"((uint32_t)v), "r"(id), "r"(n)
-      : "memory");
-  return out != 0;
-}
-
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -194,10 +191,6 @@ __device__ __forceinline__ void red_add_release_gpu(uint32_t* p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p) : "memory");
-}
-
 __device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
@@ -206,6 +199,12 @@ __device__ __forceinline__ unsigned long long ld_relaxed_gpu(const unsigned long
   unsigned long long v;
   asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
+}
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
 }
 
 // A warp-uniform bounded wait: lane 0 waits, the warp follows its verdict, and
@@ -301,7 +300,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sh->u_full[i], 1);                // the chunk's logits have landed
       mbar_init(&sh->tile_ready[i], kEpiWarps);    // the epilogue has rewritten the stage
     }
-    mbar_init(&sh->x_full, 1);                     // the step's X rows have landed
+    mbar_init(&sh->xid_ready, 1);                  // the step's previous tokens are in xid
+    mbar_init(&sh->x_full, kEpiWarps);             // the epilogue warps have gathered X
+    mbar_init(&sh->merge_ready, kEpiWarps);        // the step's maxima are in red[]
     mbar_init(&sh->drain, 1);
     sh->abort_flag = 0;
     fence_barrier_init();
@@ -376,10 +377,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < nc && ok; ++i, ++t) {
           const int j = chunk_at(i, rg, res);
           const int buf = (int)(t & 1);
-          // The previous chunk's accumulator has been read into registers (and
-          // so, in order, every earlier one): the epilogue's tensor-memory
-          // loads never wait behind MMAs in flight.
-          if (t > 0 && !mbar_wait(&sh->acc_empty[(t - 1) & 1], (uint32_t)((t - 1) >> 1) & 1u, ctl)) {
+          // The buffer's previous chunk (t - 2) has been read into registers,
+          // so this chunk's MMAs run while the epilogue works on chunk t - 1.
+          if (t > 1 && !mbar_wait(&sh->acc_empty[buf], (uint32_t)((t - 2) >> 1) & 1u, ctl)) {
             ok = false;
             break;
           }
@@ -467,23 +467,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&sh->u_full[t % NS], (uint32_t)(t / NS) & 1u, drain_ctl);
     }
   } else if (warp == 3) {
-    // ------------- grid barrier, previous tokens, X gather, U prefetch ----
+    // ---------- key merge, grid barrier, previous tokens, U prefetch ----
     // U of step k is prefetched into L2 (bulk prefetch of each row's range)
     // one step ahead: it does not depend on the chain.
-    if (lane == 0) prefetch_tensormap(&maps.w1);
-    const uint64_t pol_w1 = policy_evict_last();
     const uint32_t row_bytes = (uint32_t)((rg.v1 - rg.v0) * 2);
     auto prefetch_u = [&](int k) {
       for (int b = lane; b < B && row_bytes; b += 32)
         bulk_prefetch_l2(p.base + ((int64_t)b * M + k) * p.vocab + rg.v0, row_bytes);
     };
+    // This CTA's step-k maxima (left in red[] by the epilogue) into the global
+    // keys, one red.max per row, then the CTA's arrival: the release-add is
+    // cumulative over the lanes' reductions, which __syncwarp orders before
+    // it. Each candidate's W1 row then goes into L2, in case it wins (after
+    // the arrival, so that the release does not wait for the prefetches).
+    auto merge = [&](int k) -> bool {
+      if (!warp_wait(&sh->merge_ready, (uint32_t)k & 1u, ctl, lane)) return false;
+      unsigned long long* part = p.keys + (size_t)k * B;
+      unsigned long long key0 = 0ull, key1 = 0ull;  // rows lane and lane + 32 (B <= 64)
+      if (lane < B) {
+        key0 = red[lane];
+        red[lane] = 0ull;
+        if (key0) red_max_gpu(part + lane, key0);
+      }
+      if (lane + 32 < B) {
+        key1 = red[lane + 32];
+        red[lane + 32] = 0ull;
+        if (key1) red_max_gpu(part + lane + 32, key1);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        const bool skip = (p.debug_flags & DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL) && blockIdx.x == 0 && k == 0;
+        if (!skip) red_add_release_gpu(p.barrier, 1u);
+      }
+      __syncwarp();
+      if (k + 1 < M) {
+        if (key0) bulk_prefetch_l2(p.w1 + (size_t)key_token(key0) * (size_t)(KA * 64), (uint32_t)KA * 128u);
+        if (key1) bulk_prefetch_l2(p.w1 + (size_t)key_token(key1) * (size_t)(KA * 64), (uint32_t)KA * 128u);
+      }
+      return true;
+    };
     prefetch_u(0);
     for (int k = 0; k < M; ++k) {
-      // Every CTA has merged its step k-1 maxima once the counter reaches k * G.
-      if (k > 0 && !grid_wait(p.barrier, (uint32_t)k * (uint32_t)G, ctl, lane)) break;
+      if (k > 0) {
+        if (!merge(k - 1)) break;
+        // Every CTA has merged its step k-1 maxima once the counter reaches k * G.
+        if (!grid_wait(p.barrier, (uint32_t)k * (uint32_t)G, ctl, lane)) break;
+      }
       bool bad = false;
       for (int b = lane; b < BP; b += 32) {
-        int32_t row = (int32_t)p.vocab;  // outside W1: the gather reads zeros
+        int32_t row = (int32_t)p.vocab;  // outside W1: the gather writes zeros
         if (b < B) {
           const int64_t id =
               k == 0 ? p.first_prev[b] : (int64_t)key_token(ld_relaxed_gpu(&p.keys[(size_t)(k - 1) * B + b]));
@@ -497,24 +529,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (bad) report_status(p.status, DSPARK_STATUS_TOKEN_RANGE);
       __syncwarp();
-      // X row L is W1[x_{k-1}[L % BP]]: lane l gathers rows 4l .. 4l + 3 of
-      // every 64-column atom into the 128-byte-swizzle K-major layout. The
-      // previous step's MMAs are complete (this CTA's epilogue read their
-      // accumulators before it arrived at the barrier just passed).
-      if (lane == 0) mbar_arrive_expect_tx(&sh->x_full, (uint32_t)KA * kXAtomBytes);
-      __syncwarp();
-      {
-        const int l0 = 4 * lane;
-        const int32_t r0 = sh->xid[l0 % BP], r1 = sh->xid[(l0 + 1) % BP];
-        const int32_t r2 = sh->xid[(l0 + 2) % BP], r3 = sh->xid[(l0 + 3) % BP];
-#pragma unroll
-        for (int a = 0; a < KA; ++a)
-          tma_gather4(x_smem + (uint32_t)a * kXAtomBytes + (uint32_t)l0 * 128u, &maps.w1, &sh->x_full, a * 64, r0, r1,
-                      r2, r3, pol_w1);
-      }
+      if (lane == 0) mbar_arrive(&sh->xid_ready);
       __syncwarp();
       if (k + 1 < M) prefetch_u(k + 1);
-      if (k == M - 1 && blockIdx.x == 0) {
+      if (k == M - 1 && merge(M - 1) && blockIdx.x == 0) {
         // The last step's tokens, once every CTA has merged its maxima.
         if (grid_wait(p.barrier, (uint32_t)M * (uint32_t)G, ctl, lane))
           for (int b = lane; b < B; b += 32)
@@ -533,8 +551,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nslots = rep * kEpiPerQuarter;
     const bool row_ok = b < B;
     const uint32_t lane_base = tmem_base + ((uint32_t)(32 * q) << 16);
-    const int te = threadIdx.x - 128;
-    const uint32_t all_n = kEpiWarps * 32;
     const float inv_t = GREEDY ? 0.0f : 1.0f / p.temperature;
     // Row b of a box sits at b * 128 bytes; its 16-byte piece c at (c ^ (b & 7)) * 16.
     const uint32_t row_smem = (uint32_t)b * 128u;
@@ -542,6 +558,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     int64_t t = 0;
     bool ok = true;
     for (int k = 0; k < M && ok; ++k) {
+      // X for this step: row L of the operand is W1[x_{k-1}[L % BP]], in the
+      // 128-byte swizzle layout (16-byte chunk j of row L at chunk j ^ (L & 7)
+      // of its atom). Each distinct 16-byte piece is loaded once per CTA (a
+      // warp reads whole rows, so every W1 line is one request; all CTAs read
+      // the same rows at once) and stored into every repeat of its row (BP is
+      // a multiple of 8, so the repeats share the swizzle). The previous
+      // step's MMAs are complete: warp 3 publishes xid only after every
+      // epilogue warp has finished the previous step.
+      if (!warp_wait(&sh->xid_ready, (uint32_t)k & 1u, ctl, lane)) {
+        ok = false;
+        break;
+      }
+      {
+        constexpr int kPieces = 8 * KA;  // 16-byte pieces of a W1 row
+        const int te = ew * 32 + lane;
+        for (int i = te; i < BP * kPieces; i += kEpiWarps * 32) {
+          const int row = i / kPieces, c = i % kPieces;
+          const int32_t id = sh->xid[row];
+          const uint4 val = id < p.vocab
+                                ? ld_nc_v4(reinterpret_cast<const uint4*>(p.w1 + (size_t)id * (KA * 64)) + c)
+                                : make_uint4(0u, 0u, 0u, 0u);
+          uint8_t* dst = x_smem + (uint32_t)(c >> 3) * kXAtomBytes + (uint32_t)row * 128u +
+                         (uint32_t)(((c & 7) ^ (row & 7)) << 4);
+          for (int r = 0; r < rep; ++r) *reinterpret_cast<uint4*>(dst + (uint32_t)(r * BP) * 128u) = val;
+        }
+        fence_proxy_async_smem();  // read by the tensor cores
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->x_full);
+      }
       uint32_t best = 0u;      // greedy: (ordered bf16 bits, 0xFFFF - local id); temperature: ordered score
       uint32_t best_lid = 0u;  // temperature: the CTA-local id of `best`
       for (int i = 0; i < nc; ++i, ++t) {
@@ -630,10 +675,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh->tile_ready[s]);
       }
-      // The epilogue warps agree to go on (an abort anywhere ends every step).
-      if (!barrier_and(ok, 1, all_n)) break;
-      // This CTA's maximum per row: one shared 64-bit atomic per thread, then
-      // one global red.max per row (orderable score, complement of the id).
+      if (!ok) break;
+      // This CTA's maximum per row, through one shared 64-bit atomic per
+      // thread (orderable score, complement of the id); warp 3 takes it on.
       if (row_ok) {
         unsigned long long key;
         if constexpr (GREEDY) {
@@ -645,22 +689,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (key) atomicMax(&red[b], key);
       }
-      named_barrier_sync(1, all_n);
-      if (te < B) {
-        const unsigned long long key = red[te];
-        red[te] = 0ull;
-        if (key) {
-          red_max_gpu(&p.keys[(size_t)k * B + te], key);
-          if (k + 1 < M) prefetch_l2(p.w1 + (size_t)key_token(key) * (size_t)(KA * 64));
-        }
-      }
-      // The maxima are merged before the arrival: the release below is
-      // cumulative over the other threads' reductions ordered by this barrier.
-      named_barrier_sync(1, all_n);
-      if (te == 0) {
-        const bool skip = (p.debug_flags & DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL) && blockIdx.x == 0 && k == 0;
-        if (!skip) red_add_release_gpu(p.barrier, 1u);
-      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->merge_ready);
     }
   }
 
@@ -743,15 +773,12 @@ cudaError_t launch_rows_ka(const TcSampleArgs& a, const RowsPlan& c, int grid, c
   const uint64_t wstr[1] = {(uint64_t)a.rank * 2};
   const uint32_t box[2] = {64, (uint32_t)kChunk};
   const uint32_t box16[2] = {64, 16};
-  const uint32_t box1[2] = {64, 1};
   const uint64_t udim[3] = {(uint64_t)a.vocab, (uint64_t)a.steps, (uint64_t)a.batch};
   const uint64_t ustr[2] = {(uint64_t)a.vocab * 2, (uint64_t)a.vocab * 2 * (uint64_t)a.steps};
   const uint32_t ubox[3] = {(uint32_t)kSpan, 1u, (uint32_t)a.batch};
   if (!encode_tensor_map(&maps.w2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.w2, wdim, wstr, box,
                          CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tensor_map(&maps.w2_16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.w2, wdim, wstr, box16,
-                         CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tensor_map(&maps.w1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.w1, wdim, wstr, box1,
                          CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tensor_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.base, udim, ustr, ubox,
                          CU_TENSOR_MAP_SWIZZLE_128B) ||

@@ -751,12 +751,16 @@ bool tc_sample_supported(int64_t batch, int64_t vocab, int32_t rank, int logits_
 }
 
 // This file's tile kernel (vocabulary ids on the MMA's M side, batch up to
-// 256), or the row-layout kernel (batch up to 128) on request or where the
-// tile kernel's on-chip plan does not fit.
-cudaError_t launch_tc_sample(const TcSampleArgs& a, int num_sms, cudaStream_t s, bool prefer_rows, int* variant) {
+// 256) or the row-layout kernel (batch up to 64). Unforced, temperature
+// sampling takes the row layout and greedy decoding the tile layout: on the
+// V = 129280 .. 151936 shapes the row layout's epilogue spreads the Philox
+// and Gumbel arithmetic over all its threads and wins, while the greedy
+// chain is shorter in the tile layout.
+cudaError_t launch_tc_sample(const TcSampleArgs& a, int num_sms, cudaStream_t s, int layout, int* variant) {
   const bool rows_ok = tc_sample_rows_supported(a.batch, a.vocab, a.rank, DSPARK_DTYPE_BF16, DSPARK_DTYPE_BF16, num_sms);
   const bool tile_ok = tile_sample_supported(a.batch, a.vocab, a.rank, DSPARK_DTYPE_BF16, DSPARK_DTYPE_BF16, num_sms);
-  if (rows_ok && (prefer_rows || !tile_ok)) {
+  const bool want_rows = layout == kSampleRows || (layout == kSampleAuto && !a.greedy);
+  if (rows_ok && (want_rows || !tile_ok)) {
     *variant |= DSPARK_VARIANT_SAMPLE_ROWS;
     return launch_tc_sample_rows(a, num_sms, s);
   }

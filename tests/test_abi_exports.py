@@ -39,7 +39,7 @@ def test_header_constants_match_binding():
                  "DSPARK_ALGO_AUTO", "DSPARK_ALGO_GENERIC", "DSPARK_ALGO_TENSOR_CORE",
                  "DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL", "DSPARK_NOALLOC_MAX_KEYS", "DSPARK_VARIANT_BWD_RESIDENT_W1",
                  "DSPARK_VARIANT_SAMPLE_ROWS", "DSPARK_VARIANT_APPLY_WIDE", "DSPARK_DEBUG_APPLY_WIDE",
-                 "DSPARK_DEBUG_SAMPLE_ROWS"]:
+                 "DSPARK_DEBUG_SAMPLE_ROWS", "DSPARK_DEBUG_SAMPLE_TILE"]:
         m = re.search(rf"#define {name} (\d+)", text)
         assert m, name
         assert int(m.group(1)) == getattr(N, name), name

@@ -51,11 +51,26 @@ def _sample(d, algo, temperature, seed=0, base=None, first=None):
 
 @pytest.fixture(params=["tile", "rows"])
 def layout(request):
-    """The tensor-core sampler in its tile layout (the default) or, on
-    request, its row layout."""
-    set_debug(N.DSPARK_DEBUG_SAMPLE_ROWS if request.param == "rows" else 0, 0)
+    """The tensor-core sampler forced into its tile layout or its row layout
+    (each only where it fits)."""
+    set_debug(N.DSPARK_DEBUG_SAMPLE_ROWS if request.param == "rows" else N.DSPARK_DEBUG_SAMPLE_TILE, 0)
     yield request.param
     set_debug(0, 0)
+
+
+@pytest.mark.parametrize("temperature", [0.0, 0.7])
+def test_default_layout_by_mode(temperature):
+    """Unforced, temperature sampling takes the row layout and greedy decoding
+    the tile layout (the measured faster of the two on the full-vocabulary
+    shapes); batch 70, above the row layout's 64, takes the tile layout
+    either way. Both against the oracle."""
+    set_debug(0, 0)
+    for batch, want_rows in [(8, temperature > 0), (70, False)]:
+        wl = _small(batch, 2056, 128, m=3, wstd=0.3)
+        d = W.make_inputs(wl)
+        toks, corr, used, st = _sample(d, AUTO, temperature, seed=3)
+        assert used == 2 and st == 0 and _rows_kernel_ran() == want_rows
+        _check(d, toks, corr, temperature, 3)
 
 
 def _rows_kernel_ran() -> bool:
