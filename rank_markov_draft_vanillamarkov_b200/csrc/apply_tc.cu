@@ -4,27 +4,31 @@
 //     out[i, v] = round_bf16( U[i, v] + sum_j W1[prev_i, j] * W2[v, j] )
 //
 // One persistent CTA per SM walks a contiguous run of 128-row x 128-id output
-// tiles ("units"), vocab-tile major: all row tiles of one vocab tile, then the
-// next. The W2 tile [128 ids x rank] is loaded by TMA once per vocab tile and
-// stays in shared memory while the CTA walks that tile's rows.
-//
-// The gathered rows W1[prev] (the MMA's A operand, [128 rows x rank]) live in
-// tensor memory, loaded with tcgen05.st by four gather warps: resident for
-// the whole launch when every row tile fits (at rank 128 up to 512 rows),
-// otherwise double-buffered per unit. Shared memory then holds only W2 and a
-// deep ring of U tiles, which is what keeps enough HBM reads in flight.
+// tiles ("units"). The gathered rows W1[prev] (the MMA's A operand, [128 rows
+// x rank]) live in tensor memory, loaded with tcgen05.st by four gather
+// warps. When every row tile fits there (at rank 128 up to 512 rows) they stay
+// for the whole launch and the units go vocab-tile major: all row tiles of one
+// vocab tile, then the next, so each W2 tile [128 ids x rank] is loaded by TMA
+// once and stays in shared memory while the CTA walks that tile's rows.
+// Otherwise A is double-buffered and the units go row-tile major, so that a
+// row tile is gathered once per CTA and the W2 tiles stream from L2 through
+// two slots. Shared memory holds only W2 and a deep ring of U tiles, which is
+// what keeps enough HBM reads in flight.
 //
 // Warp roles (512 threads):
-//   warp 0       TMA producer: W2 tiles and U tiles (two 64-id boxes of 128
+//   warp 0       TMA producer: W2 tiles (vocab-tile major) and U tiles (two 64-id boxes of 128
 //                rows each, 128-byte swizzle) into rings.
 //   warp 1       owns tensor memory (512 columns); lane 0 issues
 //                tcgen05.mma.kind::f16 with A in TMEM and B = the W2 tile in
 //                shared memory (M = 128, N = 128, K = 16 per instruction).
+//   warp 2       row-tile major only: each unit's W2 tile, one 128-id x 64-rank
+//                atom at a time, into a ring of atoms.
 //   warps 4-7    gather W1[prev] rows into TMEM (warp w owns lanes 32*(w%4)).
-//   warps 8-11   epilogue group 0 (even units, accumulator 0);
-//   warps 12-15  epilogue group 1 (odd units, accumulator 1): tcgen05.ld of
-//                the fp32 accumulator (thread = row), add the U tile in place
-//                in shared memory, round to bf16, TMA-store the tile.
+//   warps 8-11   epilogue group 0 (ids 0-63 of every unit);
+//   warps 12-15  epilogue group 1 (ids 64-127): tcgen05.ld of the fp32
+//                accumulator (thread = row; the two accumulators alternate
+//                between units), add the U tile in place in shared memory,
+//                round to bf16, TMA-store the half tile.
 //
 // Tensor memory: columns [0,128) and [128,256) are the two accumulators,
 // [256,512) holds A (rank/2 columns per 128-row tile; two bf16 per column).
@@ -50,6 +54,7 @@ constexpr int kTmemCols = 512;
 constexpr int kAccCols = 2 * kBN;     // accumulators occupy [0, 256)
 constexpr int kMaxStages = 8;
 constexpr int kMaxResidentTiles = 8;
+constexpr int kMaxW2Slots = 8;
 constexpr size_t kSmemLimit = 232448;
 
 struct __align__(64) ApplyMaps {
@@ -64,14 +69,15 @@ struct ApplyParams {
   int64_t rows, vocab;
   int32_t rank;
   int32_t row_tiles, vocab_tiles;
-  int32_t w2_slots, u_stages;
+  int32_t w2_slots, u_stages;  // W2 blocks in the ring (a whole tile each, or one atom when row-major)
   int32_t resident;  // all row tiles of A stay in tensor memory
+  int32_t row_major; // units walk the vocabulary tiles of one row tile, then the next
   uint32_t* status;
   uint64_t wait_limit_ns;
 };
 
 struct SharedTail {
-  uint64_t w2_full[2], w2_empty[2];
+  uint64_t w2_full[kMaxW2Slots], w2_empty[kMaxW2Slots];
   uint64_t a_full[kMaxResidentTiles], a_empty[2];
   uint64_t u_full[kMaxStages], u_empty[kMaxStages];
   uint64_t acc_full[2], acc_empty[2];
@@ -110,6 +116,21 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
   if (ok && lane != 0) mbar_wait(bar, parity, ctl);
   return ok;
+}
+
+// Unit u's row tile m and vocabulary tile n. Vocab-tile major (all row tiles
+// of a vocabulary tile, then the next) shares each W2 tile between row tiles;
+// row-tile major shares each A tile between vocabulary tiles, which is what
+// counts when A does not stay in tensor memory and must be gathered again
+// whenever the row tile changes.
+__device__ __forceinline__ void unit_coords(const ApplyParams& p, int64_t u, int32_t& n, int32_t& m) {
+  if (p.row_major) {
+    m = (int32_t)(u / p.vocab_tiles);
+    n = (int32_t)(u % p.vocab_tiles);
+  } else {
+    n = (int32_t)(u / p.row_tiles);
+    m = (int32_t)(u % p.row_tiles);
+  }
 }
 
 // One 128-row tile of A into tensor memory: thread `row` loads W1[prev] (rank
@@ -153,10 +174,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_apply_kernel(const __grid_constant__ ApplyMaps maps, const ApplyParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* w2_smem = smem;                                     // w2_slots x KA atoms
+  uint8_t* w2_smem = smem;  // w2_slots blocks of KA atoms (vocab-tile major) or of one atom (row-tile major)
   constexpr int kUStageBytes = u_stage_bytes(F32);
   constexpr int kBoxIds = F32 ? 32 : 64;  // ids per 128-byte box row
-  uint8_t* u_smem = w2_smem + (size_t)p.w2_slots * KA * kAtomBytes;  // u_stages x kUStageBytes
+  const int w2_block_atoms = p.row_major ? 1 : KA;
+  uint8_t* u_smem = w2_smem + (size_t)p.w2_slots * w2_block_atoms * kAtomBytes;  // u_stages x kUStageBytes
   SharedTail* sh = reinterpret_cast<SharedTail*>(u_smem + (size_t)p.u_stages * kUStageBytes);
 
   constexpr int kACols = KA * 32;  // TMEM columns of one A tile
@@ -168,17 +190,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int MT = p.row_tiles;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kMaxW2Slots; ++i) {
       mbar_init(&sh->w2_full[i], 1);
       mbar_init(&sh->w2_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&sh->a_empty[i], 1);
       mbar_init(&sh->acc_full[i], 1);
-      mbar_init(&sh->acc_empty[i], 4);
+      mbar_init(&sh->acc_empty[i], 8);  // every epilogue warp
     }
     for (int i = 0; i < kMaxResidentTiles; ++i) mbar_init(&sh->a_full[i], 4);  // one arrival per gather warp
     for (int i = 0; i < p.u_stages; ++i) {
       mbar_init(&sh->u_full[i], 1);
-      mbar_init(&sh->u_empty[i], 1);
+      mbar_init(&sh->u_empty[i], 2);  // both halves stored
     }
     mbar_init(&sh->drain, 1);
     sh->abort_flag = 0;
@@ -211,8 +235,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < kMaxStages; ++i) fills[i] = 0;
       int64_t it = 0;
       for (int64_t u = u_begin; u < u_end; ++u, ++it) {
-        const int32_t n = (int32_t)(u / MT), m = (int32_t)(u % MT);
-        if (n != cur_n) {
+        int32_t n, m;
+        unit_coords(p, u, n, m);
+        if (!p.row_major && n != cur_n) {  // (row-tile major: warp 2 streams W2)
           const int ws = (int)(w2_loads % p.w2_slots);
           if (!mbar_wait(&sh->w2_empty[ws], ((w2_loads / p.w2_slots) & 1u) ^ 1u, ctl)) break;
           mbar_arrive_expect_tx(&sh->w2_full[ws], KA * kAtomBytes);
@@ -243,6 +268,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (uint32_t j = (w2_loads > (uint32_t)p.w2_slots ? w2_loads - p.w2_slots : 0); j < w2_loads; ++j)
         mbar_wait(&sh->w2_full[j % p.w2_slots], (j / p.w2_slots) & 1u, drain_ctl);
     }
+  } else if (warp == 2) {
+    // ------------------------- W2 ring producer (row-tile major) ----
+    // A new W2 tile every unit, atom by atom through the ring, so the next
+    // unit's atoms load as soon as this unit's MMAs release theirs, whatever
+    // the U ring is waiting for.
+    if (lane == 0 && p.row_major) {
+      const uint64_t pol_keep = policy_evict_last();
+      uint32_t w2_loads = 0;
+      bool ok = true;
+      for (int64_t u = u_begin; u < u_end && ok; ++u) {
+        int32_t n, m;
+        unit_coords(p, u, n, m);
+        for (int ka = 0; ka < KA; ++ka, ++w2_loads) {
+          const int ws = (int)(w2_loads % p.w2_slots);
+          ok = mbar_wait(&sh->w2_empty[ws], ((w2_loads / p.w2_slots) & 1u) ^ 1u, ctl);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&sh->w2_full[ws], kAtomBytes);
+          tma_load_2d(w2_smem + ws * kAtomBytes, &maps.w2, &sh->w2_full[ws], ka * kAtomK, n * kBN, pol_keep);
+        }
+      }
+      for (uint32_t j = (w2_loads > (uint32_t)p.w2_slots ? w2_loads - p.w2_slots : 0); j < w2_loads; ++j)
+        mbar_wait(&sh->w2_full[j % p.w2_slots], (j / p.w2_slots) & 1u, drain_ctl);
+    }
   } else if (warp == 1) {
     // ------------------------------------------------- MMA issuer -----
     if (lane == 0) {
@@ -252,9 +300,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t w2_uses = 0;
       int ws = 0;
       int64_t it = 0;
+      int32_t cur_m = -1;
+      uint32_t a_seq = 0;  // row tiles gathered so far (double-buffered A)
       for (int64_t u = u_begin; u < u_end; ++u, ++it) {
-        const int32_t n = (int32_t)(u / MT), m = (int32_t)(u % MT);
-        if (n != cur_n) {
+        int32_t n, m;
+        unit_coords(p, u, n, m);
+        if (m != cur_m) {
+          ++a_seq;
+          cur_m = m;
+        }
+        if (!p.row_major && n != cur_n) {
           ws = (int)(w2_uses % p.w2_slots);
           if (!mbar_wait(&sh->w2_full[ws], (w2_uses / p.w2_slots) & 1u, ctl)) break;
           ++w2_uses;
@@ -262,21 +317,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int abuf = (int)(it & 1);
         if (!mbar_wait(&sh->acc_empty[abuf], ((uint32_t)(it >> 1) & 1u) ^ 1u, ctl)) break;
-        const int aslot = p.resident ? m : (int)(it & 1);
-        const uint32_t apar = p.resident ? 0u : (uint32_t)(it >> 1) & 1u;
+        const int aslot = p.resident ? m : (int)((a_seq - 1) & 1u);
+        const uint32_t apar = p.resident ? 0u : ((a_seq - 1) >> 1) & 1u;
         if (!mbar_wait(&sh->a_full[aslot], apar, ctl)) break;
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + (uint32_t)(abuf * kBN);
         const uint32_t a_tmem = tmem_base + (uint32_t)(kAccCols + aslot * kACols);
+        if (p.row_major) {
+          bool ok = true;
+          for (int ka = 0; ka < KA; ++ka, ++w2_uses) {
+            const int wr = (int)(w2_uses % p.w2_slots);
+            if (!mbar_wait(&sh->w2_full[wr], (w2_uses / p.w2_slots) & 1u, ctl)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after_sync();
+            const uint64_t bd0 = sw128_kmajor_desc(w2_addr + wr * kAtomBytes);
 #pragma unroll
-        for (int kk = 0; kk < KA * kAtomK / 16; ++kk) {
-          const uint64_t bd = sw128_kmajor_desc(w2_addr + (ws * KA + (kk >> 2)) * kAtomBytes + (kk & 3) * 32);
-          umma_bf16_ts(d_tmem, a_tmem + kk * 8, bd, idesc, kk != 0);
+            for (int k4 = 0; k4 < 4; ++k4)
+              umma_bf16_ts(d_tmem, a_tmem + (ka * 4 + k4) * 8, desc_advance(bd0, k4 * 32), idesc, (ka | k4) != 0);
+            umma_commit(&sh->w2_empty[wr]);
+          }
+          if (!ok) break;
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < KA * kAtomK / 16; ++kk) {
+            const uint64_t bd = sw128_kmajor_desc(w2_addr + (ws * KA + (kk >> 2)) * kAtomBytes + (kk & 3) * 32);
+            umma_bf16_ts(d_tmem, a_tmem + kk * 8, bd, idesc, kk != 0);
+          }
         }
         umma_commit(&sh->acc_full[abuf]);
-        if (!p.resident) umma_commit(&sh->a_empty[aslot]);
-        const int64_t next_n = (u + 1 < u_end) ? (u + 1) / MT : -1;
-        if (next_n != n) umma_commit(&sh->w2_empty[ws]);
+        int32_t next_n = -1, next_m = -1;
+        if (u + 1 < u_end) unit_coords(p, u + 1, next_n, next_m);
+        if (!p.resident && next_m != m) umma_commit(&sh->a_empty[aslot]);
+        if (!p.row_major && next_n != n) umma_commit(&sh->w2_empty[ws]);
       }
       // All MMAs issued by this thread are complete once `drain` flips.
       umma_commit(&sh->drain);
@@ -288,65 +362,86 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = 32 * q + lane;
     const uint32_t lane_base = tmem_base + ((uint32_t)(32 * q) << 16);
     if (p.resident) {
-      for (int m = 0; m < MT; ++m) {
+      // Every row tile, starting with the one this CTA's first unit needs.
+      int32_t n0 = 0, m0 = 0;
+      if (u_begin < u_end) unit_coords(p, u_begin, n0, m0);
+      for (int i = 0; i < MT; ++i) {
+        const int m = (m0 + i) % MT;
         gather_tile_to_tmem<KA>(p, m, row, lane_base + kAccCols + m * kACols);
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh->a_full[m]);
       }
     } else {
-      int64_t it = 0;
-      for (int64_t u = u_begin; u < u_end; ++u, ++it) {
-        const int aslot = (int)(it & 1);
-        if (!warp_wait(&sh->a_empty[aslot], ((uint32_t)(it >> 1) & 1u) ^ 1u, ctl, lane)) break;
+      // A new tile whenever the row tile changes, into the free buffer.
+      int32_t cur_m = -1;
+      uint32_t a_seq = 0;
+      for (int64_t u = u_begin; u < u_end; ++u) {
+        int32_t n, m;
+        unit_coords(p, u, n, m);
+        if (m == cur_m) continue;
+        cur_m = m;
+        const int aslot = (int)(a_seq & 1u);
+        if (!warp_wait(&sh->a_empty[aslot], ((a_seq >> 1) & 1u) ^ 1u, ctl, lane)) break;
         tc_fence_after_sync();
-        gather_tile_to_tmem<KA>(p, (int)(u % MT), row, lane_base + kAccCols + aslot * kACols);
+        gather_tile_to_tmem<KA>(p, m, row, lane_base + kAccCols + aslot * kACols);
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh->a_full[aslot]);
+        ++a_seq;
       }
     }
   } else if (warp >= 8) {
     // ------------------------------------------------- epilogue -------
-    const int g = (warp - 8) >> 2;        // group: even or odd units
+    // Both groups work on every unit: group g takes ids [64 g, 64 g + 64)
+    // of it (U box g, or fp32 boxes 2g and 2g + 1), so a unit's accumulator
+    // is read in half the time, and it goes back to the MMA warp as soon as
+    // the eight warps have loaded it, before the adds.
+    const int g = (warp - 8) >> 2;               // which half of the unit's ids
     const int et = threadIdx.x - 256 - 128 * g;  // 0..127 within the group
-    const int q = warp & 3;               // TMEM lane quarter this warp may access
+    const int q = warp & 3;                      // TMEM lane quarter this warp may access
     const int row = 32 * q + lane;
     const uint32_t bar_id = 1 + g;
-    int64_t it = g;
-    for (int64_t u = u_begin + g; u < u_end; u += 2, it += 2) {
-      const int32_t n = (int32_t)(u / MT), m = (int32_t)(u % MT);
+    constexpr int kGroupBoxes = kUStageBytes / kAtomBytes / 2;  // boxes per half unit
+    int64_t it = 0;
+    for (int64_t u = u_begin; u < u_end; ++u, ++it) {
+      int32_t n, m;
+      unit_coords(p, u, n, m);
       const int s = (int)(it % p.u_stages);
+      const int abuf = (int)(it & 1);
       const uint32_t acc_par = (uint32_t)(it >> 1) & 1u;
       const uint32_t u_par = (uint32_t)(it / p.u_stages) & 1u;
       bool ok = true;
-      if (et == 0) ok = mbar_wait(&sh->acc_full[g], acc_par, ctl) && mbar_wait(&sh->u_full[s], u_par, ctl);
+      if (et == 0) ok = mbar_wait(&sh->acc_full[abuf], acc_par, ctl) && mbar_wait(&sh->u_full[s], u_par, ctl);
       __syncwarp();
       if (!barrier_and(ok, bar_id, 128)) break;
       if (et != 0) {
-        mbar_wait(&sh->acc_full[g], acc_par, ctl);
+        mbar_wait(&sh->acc_full[abuf], acc_par, ctl);
         mbar_wait(&sh->u_full[s], u_par, ctl);
       }
       __syncwarp();  // tcgen05.ld below is warp-aligned
       tc_fence_after_sync();
       uint8_t* st = u_smem + s * kUStageBytes;
-      const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(g * kBN);
+      const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(abuf * kBN + 64 * g);
       // A lane quarter that holds only rows past the end (the ragged last row
       // tile) has nothing to add: its rows are not stored.
       const bool live = (int64_t)m * kBM + 32 * q < p.rows;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {  // the two 64-id boxes of the tile
-        if (!live) break;
-        uint32_t acc[64];
-        tmem_ld_32x32b_x32(tbase + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&acc[0]));
-        tmem_ld_32x32b_x32(tbase + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&acc[32]));
+      uint32_t acc[64];
+      if (live) {
+        tmem_ld_32x32b_x32(tbase, *reinterpret_cast<uint32_t(*)[32]>(&acc[0]));
+        tmem_ld_32x32b_x32(tbase + 32, *reinterpret_cast<uint32_t(*)[32]>(&acc[32]));
         tmem_ld_wait();
+      }
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->acc_empty[abuf]);
+      if (live) {
         if constexpr (F32) {
-          // The half's 64 ids are boxes 2h and 2h+1, 32 fp32 each: chunk c
-          // of a box row holds ids 4c .. 4c+3.
+          // Boxes 2g and 2g+1, 32 fp32 each: chunk c of a box row holds ids
+          // 4c .. 4c+3.
 #pragma unroll
           for (int sub = 0; sub < 2; ++sub) {
-            uint8_t* box = st + (2 * h + sub) * kAtomBytes + row * 128;
+            uint8_t* box = st + (2 * g + sub) * kAtomBytes + row * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
               float4* ptr = reinterpret_cast<float4*>(box + ((c ^ (row & 7)) << 4));
@@ -360,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         } else {
-          uint8_t* box = st + h * kAtomBytes + row * 128;
+          uint8_t* box = st + g * kAtomBytes + row * 128;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             uint4* ptr = reinterpret_cast<uint4*>(box + ((c ^ (row & 7)) << 4));
@@ -373,18 +468,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->acc_empty[g]);
-      __syncwarp();
       fence_proxy_async_smem();
       named_barrier_sync(bar_id, 128);
       if (et == 0) {
 #pragma unroll
-        for (int bx = 0; bx < kUStageBytes / kAtomBytes; ++bx)
-          tma_store_2d(&maps.out, st + bx * kAtomBytes, n * kBN + bx * kBoxIds, m * kBM);
+        for (int bx = 0; bx < kGroupBoxes; ++bx)
+          tma_store_2d(&maps.out, st + (g * kGroupBoxes + bx) * kAtomBytes,
+                       n * kBN + (g * kGroupBoxes + bx) * kBoxIds, m * kBM);
         bulk_commit_group();
-        bulk_wait_group_read<0>();  // the stage may be refilled once the store has read it
+        bulk_wait_group_read<0>();  // the stage may be refilled once both halves' stores have read it
         mbar_arrive(&sh->u_empty[s]);
       }
       __syncwarp();
@@ -402,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 struct ApplyConfig {
-  int w2_slots, u_stages, resident;
+  int w2_slots, u_stages, resident, row_major;
   size_t smem_bytes;
 };
 
@@ -411,19 +503,34 @@ ApplyConfig plan(int ka, int row_tiles, bool f32) {
   ApplyConfig c{};
   c.resident = (row_tiles <= kMaxResidentTiles && row_tiles * ka * 32 <= kTmemCols - kAccCols) ? 1 : 0;
   const size_t fixed = 1024 + sizeof(SharedTail) + 64;
-  // Two W2 slots hide the reload at a vocab-tile change, which comes every
-  // row_tiles units; with many row tiles one slot leaves room for more U.
-  c.w2_slots = row_tiles < 8 ? 2 : 1;
-  for (;;) {
-    const size_t w2 = (size_t)c.w2_slots * ka * kAtomBytes;
-    int stages = (int)((kSmemLimit - fixed - w2) / kUStageBytes);
-    if (stages > kMaxStages) stages = kMaxStages;
-    if (stages >= 3 || c.w2_slots == 1) {
-      c.u_stages = stages;
-      break;
-    }
-    c.w2_slots = 1;
+  auto stages_for = [&](int slots) {
+    const int st = (int)((kSmemLimit - fixed - (size_t)slots * ka * kAtomBytes) / kUStageBytes);
+    return st > kMaxStages ? kMaxStages : st;
+  };
+  // Row-tile major streams W2 through a ring of single atoms: four U stages
+  // (three where four leave no room for two atoms) and the rest of shared
+  // memory for the ring. On 2560 rows at rank 256 that split (six atoms)
+  // measured 309 us, against 313 us with three stages and eight atoms and
+  // 328 us with five stages and four atoms: the next tile's W2 atoms need
+  // to be in flight while the current tile's are still in use.
+  int ring_stages = 4;
+  while (ring_stages > 3 && fixed + (size_t)ring_stages * kUStageBytes + 2 * (size_t)kAtomBytes > kSmemLimit)
+    --ring_stages;
+  int ring = (int)((kSmemLimit - fixed - (size_t)ring_stages * kUStageBytes) / kAtomBytes);
+  if (ring > kMaxW2Slots) ring = kMaxW2Slots;
+  if (!c.resident && ring >= 2 && fixed + (size_t)ring_stages * kUStageBytes + (size_t)ring * kAtomBytes <= kSmemLimit) {
+    c.row_major = 1;
+    c.w2_slots = ring;
+    c.u_stages = ring_stages;
+    c.smem_bytes = fixed + (size_t)ring * kAtomBytes + (size_t)c.u_stages * kUStageBytes;
+    return c;
   }
+  // Vocab-tile major: two W2 slots hide the reload at a vocab-tile change,
+  // which comes every row_tiles units; with many row tiles, or where two
+  // slots leave fewer than three U stages, one slot leaves room for more U.
+  c.row_major = 0;
+  c.w2_slots = (row_tiles < 8 && stages_for(2) >= 3) ? 2 : 1;
+  c.u_stages = stages_for(c.w2_slots);
   c.smem_bytes = fixed + (size_t)c.w2_slots * ka * kAtomBytes + (size_t)c.u_stages * kUStageBytes;
   return c;
 }
@@ -460,6 +567,7 @@ cudaError_t launch_ka(const TcApplyArgs& a, int num_sms, cudaStream_t stream) {
   p.w2_slots = c.w2_slots;
   p.u_stages = c.u_stages;
   p.resident = c.resident;
+  p.row_major = c.row_major;
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns;
 
