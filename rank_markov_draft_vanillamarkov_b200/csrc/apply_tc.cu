@@ -24,11 +24,12 @@
 //   warp 2       row-tile major only: each unit's W2 tile, one 128-id x 64-rank
 //                atom at a time, into a ring of atoms.
 //   warps 4-7    gather W1[prev] rows into TMEM (warp w owns lanes 32*(w%4)).
-//   warps 8-11   epilogue group 0 (ids 0-63 of every unit);
-//   warps 12-15  epilogue group 1 (ids 64-127): tcgen05.ld of the fp32
-//                accumulator (thread = row; the two accumulators alternate
-//                between units), add the U tile in place in shared memory,
-//                round to bf16, TMA-store the half tile.
+//   warps 8-11   epilogue group 0, warps 12-15 group 1: tcgen05.ld of the
+//                fp32 accumulator (thread = row; the two accumulators
+//                alternate between units), add the U tile in place in shared
+//                memory, round to bf16, TMA-store the tile. Vocab-tile major:
+//                group g takes the units of parity g; row-tile major: both
+//                take every unit, group g ids [64 g, 64 g + 64).
 //
 // Tensor memory: columns [0,128) and [128,256) are the two accumulators,
 // [256,512) holds A (rank/2 columns per 128-row tile; two bf16 per column).
@@ -197,12 +198,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sh->a_empty[i], 1);
       mbar_init(&sh->acc_full[i], 1);
-      mbar_init(&sh->acc_empty[i], 8);  // every epilogue warp
+      mbar_init(&sh->acc_empty[i], p.row_major ? 8 : 4);  // the warps that read it
     }
     for (int i = 0; i < kMaxResidentTiles; ++i) mbar_init(&sh->a_full[i], 4);  // one arrival per gather warp
     for (int i = 0; i < p.u_stages; ++i) {
       mbar_init(&sh->u_full[i], 1);
-      mbar_init(&sh->u_empty[i], 2);  // both halves stored
+      mbar_init(&sh->u_empty[i], p.row_major ? 2 : 1);  // the groups that store from it
     }
     mbar_init(&sh->drain, 1);
     sh->abort_flag = 0;
@@ -393,18 +394,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 8) {
     // ------------------------------------------------- epilogue -------
-    // Both groups work on every unit: group g takes ids [64 g, 64 g + 64)
-    // of it (U box g, or fp32 boxes 2g and 2g + 1), so a unit's accumulator
-    // is read in half the time, and it goes back to the MMA warp as soon as
-    // the eight warps have loaded it, before the adds.
-    const int g = (warp - 8) >> 2;               // which half of the unit's ids
+    // Vocab-tile major: group g takes the units of parity g whole (the two
+    // groups' per-unit waits and stores overlap). Row-tile major: both groups
+    // take every unit, group g its ids [64 g, 64 g + 64), and the accumulator
+    // goes back to the MMA warp right after the tensor-memory loads (there,
+    // each unit waits for a freshly streamed W2 tile, and this halves the
+    // time an accumulator is held).
+    const bool split = p.row_major != 0;
+    const int g = (warp - 8) >> 2;               // group
     const int et = threadIdx.x - 256 - 128 * g;  // 0..127 within the group
     const int q = warp & 3;                      // TMEM lane quarter this warp may access
     const int row = 32 * q + lane;
     const uint32_t bar_id = 1 + g;
-    constexpr int kGroupBoxes = kUStageBytes / kAtomBytes / 2;  // boxes per half unit
-    int64_t it = 0;
-    for (int64_t u = u_begin; u < u_end; ++u, ++it) {
+    const int h0 = split ? g : 0, h1 = split ? g + 1 : 2;  // 64-id halves of the unit this group adds
+    constexpr int kHalfBoxes = kUStageBytes / kAtomBytes / 2;
+    const int64_t step = split ? 1 : 2;
+    int64_t it = split ? 0 : g;
+    for (int64_t u = u_begin + it; u < u_end; u += step, it += step) {
       int32_t n, m;
       unit_coords(p, u, n, m);
       const int s = (int)(it % p.u_stages);
@@ -422,26 +428,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();  // tcgen05.ld below is warp-aligned
       tc_fence_after_sync();
       uint8_t* st = u_smem + s * kUStageBytes;
-      const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(abuf * kBN + 64 * g);
+      const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(abuf * kBN);
       // A lane quarter that holds only rows past the end (the ragged last row
       // tile) has nothing to add: its rows are not stored.
       const bool live = (int64_t)m * kBM + 32 * q < p.rows;
-      uint32_t acc[64];
-      if (live) {
-        tmem_ld_32x32b_x32(tbase, *reinterpret_cast<uint32_t(*)[32]>(&acc[0]));
-        tmem_ld_32x32b_x32(tbase + 32, *reinterpret_cast<uint32_t(*)[32]>(&acc[32]));
-        tmem_ld_wait();
-      }
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->acc_empty[abuf]);
-      if (live) {
+      for (int h = h0; h < h1; ++h) {
+        uint32_t acc[64];
+        if (live) {
+          tmem_ld_32x32b_x32(tbase + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&acc[0]));
+          tmem_ld_32x32b_x32(tbase + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&acc[32]));
+          tmem_ld_wait();
+        }
+        if (split) {
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh->acc_empty[abuf]);
+        }
+        if (!live) continue;
         if constexpr (F32) {
-          // Boxes 2g and 2g+1, 32 fp32 each: chunk c of a box row holds ids
-          // 4c .. 4c+3.
+          // The half's 64 ids are boxes 2h and 2h+1, 32 fp32 each: chunk c
+          // of a box row holds ids 4c .. 4c+3.
 #pragma unroll
           for (int sub = 0; sub < 2; ++sub) {
-            uint8_t* box = st + (2 * g + sub) * kAtomBytes + row * 128;
+            uint8_t* box = st + (2 * h + sub) * kAtomBytes + row * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
               float4* ptr = reinterpret_cast<float4*>(box + ((c ^ (row & 7)) << 4));
@@ -455,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         } else {
-          uint8_t* box = st + g * kAtomBytes + row * 128;
+          uint8_t* box = st + h * kAtomBytes + row * 128;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             uint4* ptr = reinterpret_cast<uint4*>(box + ((c ^ (row & 7)) << 4));
@@ -468,15 +477,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      if (!split) {
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->acc_empty[abuf]);
+      }
+      __syncwarp();
       fence_proxy_async_smem();
       named_barrier_sync(bar_id, 128);
       if (et == 0) {
-#pragma unroll
-        for (int bx = 0; bx < kGroupBoxes; ++bx)
-          tma_store_2d(&maps.out, st + (g * kGroupBoxes + bx) * kAtomBytes,
-                       n * kBN + (g * kGroupBoxes + bx) * kBoxIds, m * kBM);
+        for (int bx = h0 * kHalfBoxes; bx < h1 * kHalfBoxes; ++bx)
+          tma_store_2d(&maps.out, st + bx * kAtomBytes, n * kBN + bx * kBoxIds, m * kBM);
         bulk_commit_group();
-        bulk_wait_group_read<0>();  // the stage may be refilled once both halves' stores have read it
+        bulk_wait_group_read<0>();  // the stage may be refilled once its stores have read it
         mbar_arrive(&sh->u_empty[s]);
       }
       __syncwarp();
