@@ -459,7 +459,7 @@ def config_block(n_gpus):
 
 
 PROFILE_TAGS = {"apply": "apply_tc_r320_v129280_k128", "greedy": "sample_tc_greedy_b32_m5_v129280_k128",
-                "temperature": "sample_tc_temp_b32_m8_v151936_k64"}
+                "temperature": "sample_rows_temp_b32_m8_v151936_k64"}
 
 
 def roofline_block(dom, tag, achieved, hbm_peak, peak_kind, partinfo):

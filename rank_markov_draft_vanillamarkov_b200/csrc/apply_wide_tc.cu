@@ -17,17 +17,20 @@
 // while the current unit's MMAs run.
 //
 // Warp roles (640 threads):
-//   warp 0      TMA producer: W2 tiles (rank/64 boxes of 64 x 256) and U
-//               half-units (two 64-id boxes of 128 rows, 128-byte swizzle).
+//   warp 0      TMA producer: W2 tiles (rank/64 boxes of 64 x 256,
+//               128-byte swizzle).
 //   warp 1      tensor-memory owner and MMA issuer (M = 128, N = 256, K = 16,
 //               A from tensor memory, B = the W2 tile in shared memory).
 //   warps 4-19  epilogue and gather. Warp 4 + 4e + q owns TMEM lane quarter q
-//               (rows 32q..32q+31) and ids [64e, 64e + 64) of the unit: one
-//               tcgen05.ld pass of 64 columns, after which the accumulator is
-//               handed back to the MMA warp at once; then it adds the U box in
-//               place in shared memory, rounds once, and the four warps of a
-//               box TMA-store it. The same warp gathers columns
-//               [e r/4, (e+1) r/4) of its rows' W1 rows with tcgen05.st.
+//               (rows 32q..32q+31) and ids [64e, 64e + 64) of the unit. Each
+//               thread loads its row's 64 U values (128 bytes) straight from
+//               global memory before the unit's MMAs finish, reads its 64
+//               accumulator columns in two tcgen05.ld halves (handing the
+//               accumulator back after the second), adds, rounds once and
+//               stores the 128 bytes with streaming stores. The same warp
+//               gathers columns [e r/4, (e+1) r/4) of its rows' W1 rows with
+//               tcgen05.st. Shared memory holds only W2 tiles, so it can keep
+//               two or three of them.
 //
 // Tensor memory: the accumulator in columns [0, 256), A in [256, 512) (rank/2
 // columns per row tile). Every wait is bounded.
@@ -42,52 +45,56 @@ constexpr int kBM = 128;
 constexpr int kBN = 256;
 constexpr int kAtomK = 64;
 constexpr uint32_t kW2AtomBytes = kBN * 128;  // 256 ids x 64 bf16
-constexpr uint32_t kBoxBytes = kBM * 128;     // 128 rows x 64 bf16 ids
-constexpr uint32_t kHalfBytes = 2 * kBoxBytes;  // one U stage: 128 ids of a unit
 constexpr int kEpiWarps = 16;
 constexpr int kThreads = 128 + kEpiWarps * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCols = kBN;
-constexpr int kMaxStages = 8;
+constexpr int kMaxW2Slots = 3;
 constexpr int kMaxResident = 8;
 constexpr size_t kSmemLimit = 232448;
 
 struct __align__(64) WideMaps {
-  CUtensorMap u;    // [rows, vocab] bf16, box 64 x 128, 128B swizzle
-  CUtensorMap out;  // same geometry
-  CUtensorMap w2;   // [vocab, rank] bf16, box 64 x 256, 128B swizzle
+  CUtensorMap w2;  // [vocab, rank] bf16, box 64 x 256, 128B swizzle
 };
 
 struct WideParams {
+  const __nv_bfloat16* base;  // [rows, vocab]
+  __nv_bfloat16* out;         // [rows, vocab]
   const int64_t* ids;
   const __nv_bfloat16* w1;
   int64_t rows, vocab;
   int32_t rank;
   int32_t row_tiles, id_tiles;
-  int32_t w2_slots, stages;
+  int32_t w2_slots;
   int32_t resident;
   uint32_t* status;
   uint64_t wait_limit_ns;
 };
 
 struct WideTail {
-  uint64_t w2_full[2], w2_empty[2];
+  uint64_t w2_full[kMaxW2Slots], w2_empty[kMaxW2Slots];
   uint64_t a_full[kMaxResident], a_empty[2];
-  uint64_t u_full[kMaxStages], u_empty[kMaxStages];
   uint64_t acc_full, acc_empty;
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
 
-__device__ __forceinline__ bool barrier_and(bool v, uint32_t id, uint32_t n) {
-  uint32_t out;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(out)
-      : "r"((uint32_t)v), "r"(id), "r"(n)
-      : "memory");
-  return out != 0;
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void st_stream_v4(void* p, uint4 v) {
+  asm volatile("st.global.cs.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
@@ -148,9 +155,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_apply_wide_kernel(const __grid_constant__ WideMaps maps, const WideParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* w2_smem = smem;                                              // w2_slots x KA atoms
-  uint8_t* u_smem = w2_smem + (size_t)p.w2_slots * KA * kW2AtomBytes;  // stages x half-units
-  WideTail* sh = reinterpret_cast<WideTail*>(u_smem + (size_t)p.stages * kHalfBytes);
+  uint8_t* w2_smem = smem;  // w2_slots x KA atoms
+  WideTail* sh = reinterpret_cast<WideTail*>(w2_smem + (size_t)p.w2_slots * KA * kW2AtomBytes);
 
   constexpr uint32_t kACols = KA * 32;  // TMEM columns of one A tile
   const int warp = threadIdx.x >> 5;
@@ -159,19 +165,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t u_begin = units * blockIdx.x / gridDim.x;
   const int64_t u_end = units * (blockIdx.x + 1) / gridDim.x;
   const int MT = p.row_tiles;
-  const int S = p.stages;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kMaxW2Slots; ++i) {
       mbar_init(&sh->w2_full[i], 1);
       mbar_init(&sh->w2_empty[i], 1);
-      mbar_init(&sh->a_empty[i], 1);
     }
+    for (int i = 0; i < 2; ++i) mbar_init(&sh->a_empty[i], 1);
     for (int i = 0; i < kMaxResident; ++i) mbar_init(&sh->a_full[i], kEpiWarps);
-    for (int i = 0; i < S; ++i) {
-      mbar_init(&sh->u_full[i], 1);
-      mbar_init(&sh->u_empty[i], 2);  // the two box stores of the half-unit
-    }
     mbar_init(&sh->acc_full, 1);
     mbar_init(&sh->acc_empty, kEpiWarps);
     mbar_init(&sh->drain, 1);
@@ -194,41 +195,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------ TMA producer ----
     if (lane == 0) {
-      prefetch_tensormap(&maps.u);
       prefetch_tensormap(&maps.w2);
-      prefetch_tensormap(&maps.out);
-      const uint64_t pol_stream = policy_evict_first();
       const uint64_t pol_keep = policy_evict_last();
       int64_t cur_n = -1;
       uint32_t w2_loads = 0;
-      int64_t g = 0;
-      bool ok = true;
-      for (int64_t u = u_begin; u < u_end && ok; ++u) {
-        const int32_t n = (int32_t)(u / MT), m = (int32_t)(u % MT);
-        if (n != cur_n) {
-          const int ws = (int)(w2_loads % p.w2_slots);
-          if (!mbar_wait(&sh->w2_empty[ws], ((w2_loads / p.w2_slots) & 1u) ^ 1u, ctl)) break;
-          mbar_arrive_expect_tx(&sh->w2_full[ws], KA * kW2AtomBytes);
+      for (int64_t u = u_begin; u < u_end; ++u) {
+        const int32_t n = (int32_t)(u / MT);
+        if (n == cur_n) continue;
+        const int ws = (int)(w2_loads % p.w2_slots);
+        if (!mbar_wait(&sh->w2_empty[ws], ((w2_loads / p.w2_slots) & 1u) ^ 1u, ctl)) break;
+        mbar_arrive_expect_tx(&sh->w2_full[ws], KA * kW2AtomBytes);
 #pragma unroll
-          for (int ka = 0; ka < KA; ++ka)
-            tma_load_2d(w2_smem + (size_t)(ws * KA + ka) * kW2AtomBytes, &maps.w2, &sh->w2_full[ws], ka * kAtomK,
-                        n * kBN, pol_keep);
-          ++w2_loads;
-          cur_n = n;
-        }
-        for (int h = 0; h < 2; ++h, ++g) {
-          const int s = (int)(g % S);
-          if (!mbar_wait(&sh->u_empty[s], ((uint32_t)(g / S) & 1u) ^ 1u, ctl)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&sh->u_full[s], kHalfBytes);
-          uint8_t* st = u_smem + (size_t)s * kHalfBytes;
-          tma_load_2d(st, &maps.u, &sh->u_full[s], n * kBN + h * 128, m * kBM, pol_stream);
-          tma_load_2d(st + kBoxBytes, &maps.u, &sh->u_full[s], n * kBN + h * 128 + 64, m * kBM, pol_stream);
-        }
+        for (int ka = 0; ka < KA; ++ka)
+          tma_load_2d(w2_smem + (size_t)(ws * KA + ka) * kW2AtomBytes, &maps.w2, &sh->w2_full[ws], ka * kAtomK,
+                      n * kBN, pol_keep);
+        ++w2_loads;
+        cur_n = n;
       }
-      for (int64_t j = (g > S ? g - S : 0); j < g; ++j) mbar_wait(&sh->u_full[j % S], (uint32_t)(j / S) & 1u, drain_ctl);
       for (uint32_t j = (w2_loads > (uint32_t)p.w2_slots ? w2_loads - p.w2_slots : 0); j < w2_loads; ++j)
         mbar_wait(&sh->w2_full[j % p.w2_slots], (j / p.w2_slots) & 1u, drain_ctl);
     }
@@ -274,12 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ew = warp - 4;
     const int q = ew & 3;     // TMEM lane quarter: rows 32q .. 32q + 31
     const int e = ew >> 2;    // ids [64e, 64e + 64) of the unit; W1 columns [e r/4, (e+1) r/4)
-    const int row = 32 * q + lane;
-    const int h = e >> 1, bx = e & 1;  // U half-stage and 64-id box of this warp
     const uint32_t lane_base = tmem_base + ((uint32_t)(32 * q) << 16);
-    const uint32_t bar_id = 1 + e;     // the four warps of box e
-    const bool store_thread = q == 0 && lane == 0;
-    int prev_s = -1;
     bool ok = true;
     // A for the first unit (or every row tile, when resident).
     if (u_begin < u_end) {
@@ -297,71 +275,78 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&sh->a_full[0]);
       }
     }
+    // U rows of a unit into L2 ahead of their loads: warps of e = 0 prefetch
+    // one 512-byte row range each (a row's 256 ids).
+    auto prefetch_unit = [&](int64_t uu) {
+      if (e != 0 || uu >= u_end) return;
+      const int64_t r = (uu % MT) * kBM + 32 * q + lane;
+      const int64_t i0 = (uu / MT) * kBN;
+      if (r < p.rows) {
+        const int64_t nid = p.vocab - i0 < kBN ? p.vocab - i0 : kBN;
+        bulk_prefetch_l2(p.base + r * p.vocab + i0, (uint32_t)(nid * 2));
+      }
+    };
+    prefetch_unit(u_begin);
+    prefetch_unit(u_begin + 1);
     int64_t it = 0;
-    for (int64_t u = u_begin; u < u_end; ++u, ++it) {
+    for (int64_t u = u_begin; u < u_end && ok; ++u, ++it) {
       const int32_t n = (int32_t)(u / MT), m = (int32_t)(u % MT);
+      prefetch_unit(u + 2);
+      const int64_t grow = (int64_t)m * kBM + 32 * q + lane;
+      const int64_t v0 = (int64_t)n * kBN + 64 * e;  // this thread's first id
+      // Ids of this thread's eight 8-id chunks that exist (vocab is a
+      // multiple of 8, so a chunk is wholly in or out).
+      const int64_t left = p.vocab - v0;
+      const int nchunk = grow < p.rows ? (left >= 64 ? 8 : (left > 0 ? (int)(left / 8) : 0)) : 0;
+      // U of this unit, issued before its MMAs are awaited.
+      uint4 uv[8];
+      const __nv_bfloat16* src = p.base + grow * p.vocab + v0;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) uv[c] = c < nchunk ? ld_stream_v4(src + 8 * c) : make_uint4(0u, 0u, 0u, 0u);
       if (!p.resident && u + 1 < u_end) {
         // The next unit's rows into the other slot, once the MMAs of the unit
         // before this one have read it; the current unit's MMAs run meanwhile.
         const int ns = (int)((it + 1) & 1);
         if (!warp_wait(&sh->a_empty[ns], ((uint32_t)((it + 1) >> 1) & 1u) ^ 1u, ctl, lane)) {
           ok = false;
-        } else {
-          tc_fence_after_sync();
-          gather_share<KA>(p, (int)((u + 1) % MT), q, e, lane, lane_base + kAccCols + (uint32_t)ns * kACols);
+          break;
+        }
+        tc_fence_after_sync();
+        gather_share<KA>(p, (int)((u + 1) % MT), q, e, lane, lane_base + kAccCols + (uint32_t)ns * kACols);
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->a_full[ns]);
+      }
+      if (!warp_wait(&sh->acc_full, (uint32_t)it & 1u, ctl, lane)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      __nv_bfloat16* dst = p.out + grow * p.vocab + v0;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t acc[32];
+        __syncwarp();  // tcgen05.ld is warp-aligned
+        tmem_ld_32x32b_x32(lane_base + (uint32_t)(64 * e + 32 * half), acc);
+        tmem_ld_wait();
+        if (half == 1) {
+          // Every accumulator column of this warp is in registers.
           tc_fence_before_sync();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&sh->a_full[ns]);
+          if (lane == 0) mbar_arrive(&sh->acc_empty);
         }
-      }
-      ok = ok && warp_wait(&sh->acc_full, (uint32_t)it & 1u, ctl, lane);
-      if (!barrier_and(ok, bar_id, 128)) break;
-      tc_fence_after_sync();
-      // Rows past the end (the ragged last row tile) are neither read nor stored.
-      const bool live = (int64_t)m * kBM + 32 * q < p.rows;
-      uint32_t acc[64];
-      if (live) {
-        tmem_ld_32x32b_x32(lane_base + (uint32_t)(64 * e), *reinterpret_cast<uint32_t(*)[32]>(&acc[0]));
-        tmem_ld_32x32b_x32(lane_base + (uint32_t)(64 * e + 32), *reinterpret_cast<uint32_t(*)[32]>(&acc[32]));
-        tmem_ld_wait();
-      }
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->acc_empty);  // the accumulator is free for the next unit
-      const int64_t gs = 2 * it + h;  // this warp's U stage fill
-      const int s = (int)(gs % S);
-      if (!warp_wait(&sh->u_full[s], (uint32_t)(gs / S) & 1u, ctl, lane)) ok = false;
-      uint8_t* box = u_smem + (size_t)s * kHalfBytes + bx * kBoxBytes;
-      if (ok && live) {
-        uint8_t* rp = box + row * 128;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4* ptr = reinterpret_cast<uint4*>(rp + ((c ^ (row & 7)) << 4));
-          uint4 x = *ptr;
-          x.x = add_round_pair(x.x, acc[c * 8 + 0], acc[c * 8 + 1]);
-          x.y = add_round_pair(x.y, acc[c * 8 + 2], acc[c * 8 + 3]);
-          x.z = add_round_pair(x.z, acc[c * 8 + 4], acc[c * 8 + 5]);
-          x.w = add_round_pair(x.w, acc[c * 8 + 6], acc[c * 8 + 7]);
-          *ptr = x;
+        for (int cc = 0; cc < 4; ++cc) {
+          const int c = 4 * half + cc;
+          if (c < nchunk) {
+            const uint4 x = uv[c];
+            const uint32_t* a8 = &acc[8 * cc];
+            st_stream_v4(dst + 8 * c, make_uint4(add_round_pair(x.x, a8[0], a8[1]), add_round_pair(x.y, a8[2], a8[3]),
+                                                 add_round_pair(x.z, a8[4], a8[5]),
+                                                 add_round_pair(x.w, a8[6], a8[7])));
+          }
         }
       }
-      fence_proxy_async_smem();
-      if (!barrier_and(ok, bar_id, 128)) break;
-      if (store_thread) {
-        tma_store_2d(&maps.out, box, n * kBN + 64 * e, m * kBM);
-        bulk_commit_group();
-        // The previous box's stage may be refilled once its store has read it.
-        if (prev_s >= 0) {
-          bulk_wait_group_read<1>();
-          mbar_arrive(&sh->u_empty[prev_s]);
-        }
-        prev_s = s;
-      }
-      __syncwarp();
-    }
-    if (store_thread) {
-      bulk_wait_group<0>();
-      if (prev_s >= 0) mbar_arrive(&sh->u_empty[prev_s]);
     }
   }
 
@@ -373,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 struct WidePlan {
-  int w2_slots, stages, resident;
+  int w2_slots, resident;
   size_t smem;
   bool ok;
 };
@@ -384,33 +369,20 @@ WidePlan wide_plan(int ka, int row_tiles) {
   c.resident = (row_tiles <= kMaxResident && (uint32_t)row_tiles * a_cols <= kTmemCols - kAccCols) ? 1 : 0;
   const size_t fixed = 1024 + sizeof(WideTail) + 64;
   const size_t w2_tile = (size_t)ka * kW2AtomBytes;
-  // Two W2 slots hide the reload at an id-tile change when it comes often
-  // (few row tiles); otherwise one slot leaves room for more U stages.
-  for (int slots = row_tiles < 8 ? 2 : 1; slots >= 1; --slots) {
-    if (fixed + slots * w2_tile >= kSmemLimit) continue;
-    int stages = (int)((kSmemLimit - fixed - slots * w2_tile) / kHalfBytes);
-    if (stages > kMaxStages) stages = kMaxStages;
-    if (stages < 3) continue;
-    c.w2_slots = slots;
-    c.stages = stages;
-    c.smem = fixed + slots * w2_tile + (size_t)stages * kHalfBytes;
-    c.ok = true;
-    return c;
-  }
+  // As many W2 slots as fit (up to three): the next id tile's W2 loads while
+  // the current one is in use.
+  int slots = (int)((kSmemLimit - fixed) / w2_tile);
+  if (slots > kMaxW2Slots) slots = kMaxW2Slots;
+  if (slots < 1) return c;
+  c.w2_slots = slots;
+  c.smem = fixed + (size_t)slots * w2_tile;
+  c.ok = true;
   return c;
 }
 
 template <int KA>
 cudaError_t launch_wide_ka(const TcApplyArgs& a, int num_sms, cudaStream_t stream) {
   WideMaps maps;
-  const uint64_t ldim[2] = {(uint64_t)a.vocab, (uint64_t)a.rows};
-  const uint64_t lstr[1] = {(uint64_t)a.vocab * 2};
-  const uint32_t ubox[2] = {64, (uint32_t)kBM};
-  if (!encode_tensor_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.base, ldim, lstr, ubox,
-                         CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tensor_map(&maps.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.out, ldim, lstr, ubox,
-                         CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
   const uint64_t wdim[2] = {(uint64_t)a.rank, (uint64_t)a.vocab};
   const uint64_t wstr[1] = {(uint64_t)a.rank * 2};
   const uint32_t wbox[2] = {64, (uint32_t)kBN};
@@ -418,6 +390,8 @@ cudaError_t launch_wide_ka(const TcApplyArgs& a, int num_sms, cudaStream_t strea
                          CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   WideParams p{};
+  p.base = static_cast<const __nv_bfloat16*>(a.base);
+  p.out = static_cast<__nv_bfloat16*>(a.out);
   p.ids = a.ids;
   p.w1 = static_cast<const __nv_bfloat16*>(a.w1);
   p.rows = a.rows;
@@ -428,7 +402,6 @@ cudaError_t launch_wide_ka(const TcApplyArgs& a, int num_sms, cudaStream_t strea
   const WidePlan c = wide_plan(KA, p.row_tiles);
   if (!c.ok) return cudaErrorInvalidValue;
   p.w2_slots = c.w2_slots;
-  p.stages = c.stages;
   p.resident = c.resident;
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns;
