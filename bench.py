@@ -231,11 +231,16 @@ class Part:
         return part_rows(self.wl)
 
 
+TIMED_LAUNCHES = {"last": 0}  # this library's kernel launches inside the last timed loop
+
+
 def time_region(parts, steps, warmup, world):
     """Warm up, then time exactly `steps` steps between a barrier and a device
     synchronise on both sides. Returns (region seconds max over ranks, per-part
-    mean kernel seconds)."""
+    mean kernel seconds); the launches of the timed loop alone go to
+    TIMED_LAUNCHES."""
     import torch.distributed as dist
+    from rank_markov_draft_vanillamarkov_b200 import launch_count
     for i in range(warmup):
         for p in parts:
             p.run(i)
@@ -246,6 +251,7 @@ def time_region(parts, steps, warmup, world):
     torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
+    n0 = launch_count()
     start.record()
     for i in range(steps):
         for p in parts:
@@ -256,6 +262,7 @@ def time_region(parts, steps, warmup, world):
             b.record()
             ev[p.name].append((a, b))
     end.record()
+    TIMED_LAUNCHES["last"] = launch_count() - n0
     torch.cuda.synchronize()
     region = start.elapsed_time(end) / 1e3
     per = {k: sum(a.elapsed_time(b) for a, b in v) / len(v) / 1e3 for k, v in ev.items()}
@@ -510,7 +517,6 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
 
     from rank_markov_draft_vanillamarkov_b200 import _native as N
-    from rank_markov_draft_vanillamarkov_b200 import launch_count
     from rank_markov_draft_vanillamarkov_b200.build import build
     if rank == 0:
         build()
@@ -535,9 +541,8 @@ def main():
 
     clocks = ClockSampler(local)
     clocks.start()
-    n0 = launch_count()
     region, per = time_region(parts, args.steps, args.warmup, world)
-    launches = launch_count() - n0
+    launches = TIMED_LAUNCHES["last"]
     clk = clocks.stop()
     extra_per = time_region(extra, max(20, args.steps // 20), 3, world)[1] if extra else {}
 
