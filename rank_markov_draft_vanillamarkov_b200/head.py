@@ -14,7 +14,9 @@ predecessor (``apply_block_logits``); inference samples left to right
 """
 from __future__ import annotations
 
+import functools
 import math
+import os
 from typing import Optional, Tuple
 
 import torch
@@ -22,6 +24,27 @@ import torch
 from . import _native as N
 
 _DT = {torch.float32: N.DSPARK_DTYPE_FP32, torch.bfloat16: N.DSPARK_DTYPE_BF16}
+
+# Every entry point runs inside an NVTX range named "dspark_markov.<method>",
+# so that a profiler's timeline shows the library's calls around its kernels.
+# DSPARK_NVTX=0 in the environment (read at import) leaves the ranges out.
+_NVTX = os.environ.get("DSPARK_NVTX", "1") != "0"
+
+
+def _ranged(fn):
+    name = "dspark_markov." + fn.__name__
+
+    @functools.wraps(fn)
+    def wrapper(*args, **kwargs):
+        if not _NVTX:
+            return fn(*args, **kwargs)
+        torch.cuda.nvtx.range_push(name)
+        try:
+            return fn(*args, **kwargs)
+        finally:
+            torch.cuda.nvtx.range_pop()
+
+    return wrapper
 
 
 def _stream_ptr(device: torch.device) -> int:
@@ -67,6 +90,7 @@ class VanillaMarkov:
         return self.markov_w1.dtype
 
     # ------------------------------------------------------------------ apply
+    @_ranged
     def apply_block_logits(self, base_logits: torch.Tensor, *, token_ids: torch.Tensor,
                            hidden_states: Optional[torch.Tensor] = None,
                            out: Optional[torch.Tensor] = None) -> torch.Tensor:
@@ -103,6 +127,7 @@ class VanillaMarkov:
         N.check(code, "dspark_markov_apply_block_logits")
         return out
 
+    @_ranged
     def fused_lm_head_logits(self, hidden_states: torch.Tensor, lm_head_weight: torch.Tensor, *,
                              token_ids: torch.Tensor, out_dtype: torch.dtype = torch.float32,
                              out: Optional[torch.Tensor] = None) -> torch.Tensor:
@@ -143,12 +168,14 @@ class VanillaMarkov:
         N.check(code, "dspark_markov_fused_lm_head_logits")
         return out
 
+    @_ranged
     def apply_step_logits(self, logits: torch.Tensor, *, token_ids: torch.Tensor,
                           hidden_states: Optional[torch.Tensor] = None) -> torch.Tensor:
         """One position (B, V) with its (B,) previous tokens."""
         return self.apply_block_logits(logits.unsqueeze(-2), token_ids=token_ids.unsqueeze(-1),
                                        hidden_states=hidden_states).squeeze(-2)
 
+    @_ranged
     def apply_block_logits_backward(self, grad_out: torch.Tensor, *, token_ids: torch.Tensor,
                                     grad_w1: Optional[torch.Tensor] = None, grad_w2: Optional[torch.Tensor] = None,
                                     accumulate: bool = False, want_w1: bool = True, want_w2: bool = True):
@@ -186,6 +213,7 @@ class VanillaMarkov:
         N.check(code, "dspark_markov_apply_block_logits_backward")
         return outs[0], outs[1]
 
+    @_ranged
     def transition_logits(self, token_ids: torch.Tensor, *, with_embeddings: bool = True,
                           out: Optional[torch.Tensor] = None,
                           out_embeddings: Optional[torch.Tensor] = None):
@@ -221,6 +249,7 @@ class VanillaMarkov:
         return out, emb
 
     # ----------------------------------------------------------------- sample
+    @_ranged
     def sample_block_tokens(self, base_logits: torch.Tensor, *, first_prev_token_ids: torch.Tensor,
                             hidden_states: Optional[torch.Tensor] = None, temperature: Optional[float] = 0.0,
                             seed: int = 0, out_tokens: Optional[torch.Tensor] = None,
@@ -259,6 +288,7 @@ class VanillaMarkov:
         N.check(code, "dspark_markov_sample_block")
         return tokens, corrected
 
+    @_ranged
     def sample_block_tokens_noalloc(self, base_logits: torch.Tensor, *, first_prev_token_ids: torch.Tensor,
                                     out_tokens: torch.Tensor, out_logits: torch.Tensor,
                                     temperature: Optional[float] = 0.0, seed: int = 0) -> None:
