@@ -531,7 +531,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->xid_ready);
       __syncwarp();
-      if (k + 1 < M) prefetch_u(k + 1);
+      // The next step's U goes into L2 once X has landed, out of the window
+      // where the epilogue warps wait for W1 rows.
+      if (k + 1 < M && warp_wait(&sh->x_full, (uint32_t)k & 1u, ctl, lane)) prefetch_u(k + 1);
       if (k == M - 1 && merge(M - 1) && blockIdx.x == 0) {
         // The last step's tokens, once every CTA has merged its maxima.
         if (grid_wait(p.barrier, (uint32_t)M * (uint32_t)G, ctl, lane))
