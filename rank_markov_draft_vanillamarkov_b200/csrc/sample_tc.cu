@@ -565,9 +565,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // The groups agree to go on (an abort anywhere ends every step here).
       if (!barrier_and(ok, allbar, all_n)) break;
       // Merge the partial maxima of each b, then this CTA's into the global
-      // keys (64-bit: orderable score, complement of the global id). The W1
-      // row of this CTA's candidate is prefetched into L2: if it wins, the
-      // next step's gather finds it there.
+      // keys (64-bit: orderable score, complement of the global id). The
+      // arrival below is a release by one thread after the CTA barrier, so
+      // it is cumulative over every thread's reduction ordered before it; a
+      // fence per thread would wait for each contended reduction in turn.
+      // The W1 row of this CTA's candidate goes into L2 after the arrival
+      // (a release also waits for the thread's earlier prefetches): if it
+      // wins, the next step's gather finds it there.
+      unsigned long long cand = 0ull;  // this thread's row candidate (B <= all_n rows)
       for (int b = te; b < B; b += (int)all_n) {
         Key m = 0;
         for (int r = 0; r < NG * 4; ++r) m = red[(size_t)r * BB + b] > m ? red[(size_t)r * BB + b] : m;
@@ -578,17 +583,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           gk = m;
         }
-        if (gk) {
-          red_max_gpu(&p.keys[(size_t)k * B + b], gk);
-          if (k + 1 < M) prefetch_l2(p.w1 + (size_t)key_token(gk) * p.rank);
-        }
-        __threadfence();  // the merge is performed before this CTA's arrival below
+        if (gk) red_max_gpu(&p.keys[(size_t)k * B + b], gk);
+        cand = gk;
       }
       named_barrier_sync(allbar, all_n);
       if (te == 0) {
         const bool skip = (p.debug_flags & DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL) && blockIdx.x == 0 && k == 0;
         if (!skip) red_add_release_gpu(p.barrier, 1u);
       }
+      if (cand && k + 1 < M) prefetch_l2(p.w1 + (size_t)key_token(cand) * p.rank);
     }
   }
 
