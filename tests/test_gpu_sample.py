@@ -58,6 +58,28 @@ def layout(request):
     set_debug(0, 0)
 
 
+@pytest.mark.parametrize("batch,vocab,rank,m,temperature", [
+    (1, 1000, 64, 1, 0.0),     # one step: the chain's first and last step at once
+    (64, 2056, 128, 2, 0.8),   # the largest batch (64 padded rows), the last range ends inside a span
+    (17, 4104, 256, 3, 0.0),   # rank 256, V not a multiple of 64
+    (40, 136, 64, 4, 1.1),     # three CTAs, the last with 8 ids
+    (32, 9600, 192, 5, 0.6),   # rank 192 with chunks of several widths
+])
+def test_row_layout_edge_shapes(batch, vocab, rank, m, temperature):
+    """The row-layout sampler at the edges of its plan (steps, batch, rank,
+    ranges that end inside a 64-id span, tiny grids), forced, every (b, k)
+    against the oracle with weights that move tokens."""
+    wl = _small(batch, vocab, rank, m=m, wstd=0.3, seed=50 + batch).with_(temperature=temperature)
+    d = W.make_inputs(wl)
+    set_debug(N.DSPARK_DEBUG_SAMPLE_ROWS, 0)
+    try:
+        toks, corr, used, st = _sample(d, TC, temperature, seed=9)
+    finally:
+        set_debug(0, 0)
+    assert used == 2 and st == 0 and _rows_kernel_ran()
+    _check(d, toks, corr, temperature, 9)
+
+
 @pytest.mark.parametrize("temperature", [0.0, 0.7])
 def test_default_layout_by_mode(temperature):
     """Unforced, temperature sampling takes the row layout and greedy decoding
@@ -271,20 +293,28 @@ def test_out_of_range_first_prev_reports_status(algo):
     assert st & N.DSPARK_STATUS_TOKEN_RANGE
 
 
-def test_barrier_timeout_is_reported_not_hung():
+@pytest.mark.parametrize("which", ["tile", "rows"])
+def test_barrier_timeout_is_reported_not_hung(which):
     """One CTA withholds its grid-barrier arrival (a host-set test flag):
     the other CTAs' bounded waits run out after 20 ms, the TIMEOUT bit is
-    set, the kernel returns, and the next call is correct again."""
+    set, the kernel returns, and the next call is correct again. Both
+    sampler layouts."""
     wl = W.greedy(8)
     d = W.make_inputs(wl)
-    set_debug(N.DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL, 20_000_000)
+    force = N.DSPARK_DEBUG_SAMPLE_ROWS if which == "rows" else N.DSPARK_DEBUG_SAMPLE_TILE
+    set_debug(N.DSPARK_DEBUG_SKIP_BARRIER_ARRIVAL | force, 20_000_000)
     try:
         _, _, used, st = _sample(d, TC, 0.0)
+        assert _rows_kernel_ran() == (which == "rows")
     finally:
         set_debug(0, 0)
     assert used == 2
     assert st & N.DSPARK_STATUS_TIMEOUT
-    toks, corr, used, st = _sample(d, TC, 0.0)
+    set_debug(force, 0)
+    try:
+        toks, corr, used, st = _sample(d, TC, 0.0)
+    finally:
+        set_debug(0, 0)
     assert st == 0
     _check(d, toks, corr, 0.0, 0)
 
@@ -329,12 +359,16 @@ def _edge_rows(vocab: int, m: int):
     return base.to(torch.bfloat16)
 
 
-@pytest.mark.parametrize("algo", [TC, GEN], ids=["tc", "generic"])
+@pytest.mark.parametrize("algo", [TC + 100, TC, GEN], ids=["tc_rows", "tc_tile", "generic"])
 @pytest.mark.parametrize("vocab", [129280, 1000])
 def test_greedy_ties_nan_signed_zero_and_inf(algo, vocab):
     """Greedy selection on exact ties, NaN, -0/+0 and all -inf: with W2 = 0
     every corrected logit is its base logit, so each token is numpy's argmax
-    (first NaN, else the lowest id among equal maxima) of its base row."""
+    (first NaN, else the lowest id among equal maxima) of its base row. The
+    tensor-core sampler in both layouts."""
+    rows_layout = algo == TC + 100
+    algo = TC if rows_layout else algo
+    set_debug(N.DSPARK_DEBUG_SAMPLE_ROWS if rows_layout else 0, 0)
     m, rank = 3, 64
     base = _edge_rows(vocab, m)
     g = torch.Generator().manual_seed(2)
@@ -342,8 +376,13 @@ def test_greedy_ties_nan_signed_zero_and_inf(algo, vocab):
     w2 = torch.zeros(vocab, rank, dtype=torch.bfloat16)
     first = torch.arange(base.shape[0], dtype=torch.long) * 13
     d = {"w1": w1, "w2": w2, "base": base, "first_prev": first}
-    toks, corr, used, st = _sample(d, algo, 0.0)
+    try:
+        toks, corr, used, st = _sample(d, algo, 0.0)
+    finally:
+        set_debug(0, 0)
     assert used == (2 if algo == TC else 1) and st == 0
+    if algo == TC:
+        assert _rows_kernel_ran() == rows_layout
     want = oracle.select_greedy(f64(base))
     np.testing.assert_array_equal(toks.cpu().numpy(), want)
     # the corrected logits are the base logits (-0 + 0 = +0, NaN stays NaN)
