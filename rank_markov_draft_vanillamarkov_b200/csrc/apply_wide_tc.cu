@@ -3,11 +3,11 @@
 //
 //     out[i, v] = round_bf16( U[i, v] + sum_j W1[prev_i, j] * W2[v, j] )
 //
-// A tcgen05.mma costs the same time at N = 256 as at N = 128 on this part, so
-// this kernel takes units of 128 rows x 256 ids: half the MMAs of the 128-id
-// kernel (apply_tc.cu), and half the W1 row gathers where the rows' W1 rows
-// cannot stay in tensor memory for the whole launch (many row tiles at
-// rank 256), which is what bounds that kernel there.
+// This kernel takes units of 128 rows x 256 ids: half the MMA instructions of
+// the 128-id kernel (apply_tc.cu), and half the W1 row gathers where the rows'
+// W1 rows cannot stay in tensor memory for the whole launch (many row tiles
+// at rank 256). It is an opt-in variant: on every workload measured here it
+// is slower than the 128-id kernel, whose per-unit stages move U by TMA.
 //
 // Persistent CTAs walk contiguous runs of units, id-tile major (all row tiles
 // of one id tile, then the next), so a W2 tile [256 ids x rank] is loaded

@@ -25,8 +25,8 @@
 // 4 + q reads accumulator lanes 32q..32q+31 (one row per thread), rounds and
 // stores the row's 256 values with streaming 16-byte stores. Tensor memory
 // holds two 256-column fp32 accumulators, so the epilogue of one unit overlaps
-// the MMAs of the next. An MMA costs the same at N = 256 as at N = 16 on this
-// part, hence the widest N.
+// the MMAs of the next. The widest N takes the fewest MMA instructions per id:
+// on this part a narrow MMA costs far more per column than a wide one.
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
